@@ -1,0 +1,528 @@
+"""Benchmark of the MoonEP hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid]
+                    [--impl reference] [--no-sweep]
+
+A step is one pass of the whole hot path over one MoE layer of the workload:
+moonep_plan -> moonep_prefetch -> moonep_dispatch -> moonep_combine ->
+moonep_reduce_grad (the combine gathers the dispatched rows themselves: the
+expert computation is out of scope).  Inputs are resident in HBM when the
+timed region starts and are larger than L2, so no flush is needed between
+steps.  Every kernel is timed with CUDA events on the launching stream;
+`value` is the dispatch+combine algorithmic bytes over their device time,
+summed over ranks; `e2e` is the same metric through the same calls with the
+router output and hidden states copied in from pinned host memory and the
+combined output copied back, inside the timed region.
+
+Under torchrun every rank runs its own independent replica of the workload
+("replicas only": the path is simulated on one GPU, with no exchange between
+GPUs); times are the max over ranks.  --impl reference times the CPU oracle
+(single-threaded C) on a bounded sample of the same workload, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from load_balancing_plan_b200 import inputs  # noqa: E402
+
+METRIC = "dispatch+combine GB/s vs HBM peak; plan µs; rows/s flat across maxvio sweep"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (per launch)
+# ---------------------------------------------------------------------------
+
+def alg_bytes(cfg, n_replicas=0, n_rx=0, w_elems=0, g_elems=0):
+    """Bytes each step must move at minimum.  T = R*S tokens.
+    dispatch: read x once, write K rows per token, read ids, write dest.
+    combine: read K rows per token, write one, read weights and dest.
+    prefetch: read and write P*H*I bf16 per used slot.
+    reduce_grad: read+write the home gradient of each replicated expert,
+    read+zero every replica (fp32).  plan: read the ids."""
+    T = cfg["R"] * cfg["S"]
+    K, H = cfg["K"], cfg["H"]
+    row = 2 * H
+    return dict(
+        dispatch=T * row + T * K * row + 8 * T * K,
+        combine=T * K * row + T * row + 8 * T * K,
+        prefetch=2 * 2 * w_elems * n_replicas,
+        reduce_grad=4 * g_elems * (2 * n_rx + 2 * n_replicas),
+        plan=4 * T * K,
+    )
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, or None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                if line.startswith("#") or not line.strip():
+                    continue
+                k, w, b = line.split()[:3]
+                if k == kernel and w == workload:
+                    return float(b)
+    except OSError:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, read only)
+# ---------------------------------------------------------------------------
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index, period=0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:
+                import torch
+                pr = torch.cuda.get_device_properties(device_index)
+                bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in _REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+
+def rank_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def reduce_over_ranks(local_ms, local_units, world):
+    """Max of the timed-region lengths and sum of the units over ranks (the
+    identity with one rank).  Returns (max_ms, total_units)."""
+    if world <= 1:
+        return float(local_ms), float(local_units)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=dev)
+    u = torch.tensor([float(local_units)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+class Runner:
+    def __init__(self, wl, maxvio, seed, with_weights=True):
+        import torch
+        from load_balancing_plan_b200 import harness
+        self.torch = torch
+        self.wl = wl
+        self.cfg = wl.cfg()
+        t0 = time.time()
+        self.route = inputs.routing(wl.R, wl.L, wl.S, wl.K, seed, maxvio=maxvio)
+        self.gen_s = time.time() - t0
+        we = wl.w_elems if with_weights else 0
+        ge = wl.g_elems if with_weights else 0
+        self.prob = harness.Problem(self.cfg, w_elems=we, g_elems=ge)
+        self.prob.set_routing(self.route.topk_idx, self.route.topk_w)
+        self.prob.fill_x(seed)
+        self.prob.fill_weights(seed)
+        self.prob.fill_g_rep(seed)
+        self.stream = torch.cuda.current_stream()
+        self.with_weights = with_weights
+        torch.cuda.synchronize()
+
+    def step(self, ev=None):
+        p = self.prob
+        s = self.stream
+        if ev is not None:
+            ev[0].record(s)
+        p.plan(s)
+        if ev is not None:
+            ev[1].record(s)
+        if self.with_weights:
+            p.prefetch(s)
+        if ev is not None:
+            ev[2].record(s)
+        p.dispatch(s)
+        if ev is not None:
+            ev[3].record(s)
+        p.combine(None, s)
+        if ev is not None:
+            ev[4].record(s)
+        if self.with_weights:
+            p.reduce_grad(s)
+        if ev is not None:
+            ev[5].record(s)
+
+    def launches_per_step(self):
+        return 5 if self.with_weights and self.cfg["B"] > 0 else 3
+
+    def timed(self, steps, warmup, world=1):
+        torch = self.torch
+        for _ in range(warmup):
+            self.step()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            start = torch.cuda.Event(enable_timing=True)
+            end = torch.cuda.Event(enable_timing=True)
+            start.record(self.stream)
+            for i in range(steps):
+                self.step(evs[i])
+            end.record(self.stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        total_ms = start.elapsed_time(end)
+        names = ["plan", "prefetch", "dispatch", "combine", "reduce_grad"]
+        per = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)] for j, n in enumerate(names)}
+        return total_ms, per, clk.summary()
+
+    def e2e(self, steps, warmup):
+        """Same calls with the step's inputs copied from pinned host memory
+        and the output copied back, all inside the timed region."""
+        torch = self.torch
+        p = self.prob
+        T, K = self.prob.T, self.cfg["K"]
+        ids_h = torch.from_numpy(self.route.topk_idx.reshape(-1).copy()).pin_memory()
+        w_h = torch.from_numpy(self.route.topk_w.reshape(-1).copy()).pin_memory()
+        x_h = p.x.cpu().pin_memory()
+        out_h = torch.empty_like(p.out, device="cpu").pin_memory()
+        s = self.stream
+
+        def one():
+            p.ids[:T * K].copy_(ids_h, non_blocking=True)
+            p.w[:T * K].copy_(w_h, non_blocking=True)
+            p.x.copy_(x_h, non_blocking=True)
+            self.step()
+            out_h.copy_(p.out, non_blocking=True)
+
+        for _ in range(warmup):
+            one()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(steps):
+            one()
+        b.record(s)
+        torch.cuda.synchronize()
+        h2d = ids_h.numel() * 4 + w_h.numel() * 4 + x_h.numel() * 2
+        d2h = out_h.numel() * 2
+        return a.elapsed_time(b), h2d, d2h
+
+
+def run_gpu(args):
+    import torch
+    rank, local_rank, world = rank_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    wl = inputs.WORKLOADS[args.workload]
+    target = wl.maxvio[0] if wl.maxvio else None
+    run = Runner(wl, target, seed=args.seed)
+    from load_balancing_plan_b200 import moonep as mp
+    info = mp.moonep_plan_read(run.cfg, run.prob.ws)   # also checks the status
+    run.step()
+    info = mp.moonep_plan_read(run.cfg, run.prob.ws)
+    if info["status"] & mp.ST_ERROR_MASK:
+        raise RuntimeError("plan failed: status 0x%x" % info["status"])
+    n_rx = len(set(np.asarray(mp.moonep_plan_read(run.cfg, run.prob.ws, tables=True)["rep_expert"]).tolist()))
+    ab = alg_bytes(run.cfg, info["n_replicas"], n_rx, run.prob.w_elems, run.prob.g_elems)
+
+    total_ms, per, clocks = run.timed(args.steps, args.warmup, world)
+    mean = {k: float(np.mean(v)) for k, v in per.items()}
+    dc_ms = sum(per["dispatch"]) + sum(per["combine"])
+    max_dc_ms, dc_bytes = reduce_over_ranks(dc_ms, (ab["dispatch"] + ab["combine"]) * args.steps, world)
+    max_total_ms, rows = reduce_over_ranks(total_ms, run.prob.T * run.cfg["K"] * args.steps, world)
+    value = dc_bytes / (max_dc_ms * 1e-3) / 1e9
+    ms_per_step = max_total_ms / args.steps
+
+    e2e_ms, h2d, d2h = run.e2e(max(3, args.steps // 4), 2)
+    e2e_steps = max(3, args.steps // 4)
+    max_e2e_ms, e2e_bytes = reduce_over_ranks(e2e_ms, (ab["dispatch"] + ab["combine"]) * e2e_steps, world)
+
+    peak, peak_kind = measured_peak()
+    shares = {k: sum(v) for k, v in per.items()}
+    dom = max(("dispatch", "combine", "prefetch", "reduce_grad"), key=lambda k: shares[k])
+    achieved = ab[dom] / (mean[dom] * 1e-3) / 1e9
+    kernel_gbs = {k: (ab[k] / (mean[k] * 1e-3) / 1e9 if mean[k] > 0 and ab[k] else None)
+                  for k in ("dispatch", "combine", "prefetch", "reduce_grad")}
+
+    sweep = None
+    if not args.no_sweep and world == 1:
+        sweep = run_sweep(args, peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(wl, run.route, args.cpu_seconds)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "%s: R=%d L=%d (N=%d experts) S=%d K=%d H=%d B=%d C=%d C_max=%d, "
+                               "router bias tuned to maxvio %.2f (achieved %.3f), seed %d"
+                               % (wl.name, wl.R, wl.L, wl.N, wl.S, wl.K, wl.H, wl.B, wl.C, wl.C_max,
+                                  target if target is not None else -1, run.route.maxvio, args.seed),
+                   "step": "plan -> prefetch -> dispatch -> combine -> reduce_grad",
+                   "weights_per_expert": "bf16 [%d x %d x %d]" % (wl.P, wl.H, wl.I),
+                   "grads_per_expert": "fp32 [%d x %d]" % (wl.H, wl.I),
+                   "accumulate": "fp32", "parallelism": "replicas%d" % world,
+                   "l2": "no flush: inputs larger than L2 (x %.2f GB, recv %.2f GB)"
+                         % (run.prob.x.numel() * 2 / 1e9, run.prob.recv.numel() * 2 / 1e9)},
+        "plan_us": round(mean["plan"] * 1e3, 2),
+        "kernel_us": {k: round(v * 1e3, 2) for k, v in mean.items()},
+        "kernel_gbs": {k: (round(v, 1) if v else None) for k, v in kernel_gbs.items()},
+        "rows_per_s": round(rows / (max_total_ms * 1e-3), 1),
+        "dispatch_combine_frac_of_peak": round(value / world / peak, 4),
+        "dispatch_combine_frac_of_8tbs": round(value / world / 8000.0, 4),
+        "plan_info": {"n_replicas": info["n_replicas"], "migrated_rows": info["migrated_rows"],
+                      "migrated_frac": round(info["migrated_rows"] / (run.prob.T * wl.K), 4),
+                      "fallback_rows": info["fallback_rows"], "replicated_experts": n_rx},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "algorithmic_bytes": ab[dom],
+                     "traffic": recorded_traffic(dom, wl.name)},
+        "e2e": {"value": round(e2e_bytes / (max_e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(max_e2e_ms / e2e_steps, 4)},
+        "gpu_launches": run.launches_per_step() * args.steps,
+        "clocks": clocks,
+    }
+    if sweep is not None:
+        out["sweep"] = sweep
+    if cpu is not None:
+        out["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_sweep(args, peak):
+    """plan / dispatch / combine over the skew-sweep workload at each target
+    maxvio (seed 0): rows/s should not move with the skew."""
+    import torch
+    wl = inputs.WORKLOADS["skew"]
+    res = {}
+    for mv in wl.maxvio:
+        run = Runner(wl, mv, seed=0, with_weights=False)
+        total_ms, per, _ = run.timed(args.sweep_steps, 3)
+        from load_balancing_plan_b200 import moonep as mp
+        info = mp.moonep_plan_read(run.cfg, run.prob.ws)
+        ab = alg_bytes(run.cfg)
+        d = float(np.mean(per["dispatch"]))
+        c = float(np.mean(per["combine"]))
+        res["%g" % mv] = {
+            "maxvio": round(run.route.maxvio, 3),
+            "plan_us": round(float(np.mean(per["plan"])) * 1e3, 2),
+            "dispatch_gbs": round(ab["dispatch"] / (d * 1e-3) / 1e9, 1),
+            "combine_gbs": round(ab["combine"] / (c * 1e-3) / 1e9, 1),
+            "dispatch_combine_frac": round((ab["dispatch"] + ab["combine"]) / ((d + c) * 1e-3) / 1e9 / peak, 4),
+            "rows_per_s": round(run.prob.T * wl.K / (total_ms / args.sweep_steps * 1e-3), 1),
+            "migrated_frac": round(info["migrated_rows"] / (run.prob.T * wl.K), 4),
+            "n_replicas": info["n_replicas"], "fallback_rows": info["fallback_rows"],
+        }
+        del run
+        torch.cuda.empty_cache()
+    rps = [v["rows_per_s"] for v in res.values()]
+    return {"workload": "skew: R=8 L=32 S=8192 K=8 H=7168 B=32, seed 0, step = plan -> dispatch -> combine",
+            "points": res, "rows_per_s_spread": round(max(rps) / min(rps) - 1.0, 4)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle arm (reference / cpu_baseline)
+# ---------------------------------------------------------------------------
+
+class OracleArm:
+    """The oracle (as it stands, single-threaded C) on a bounded sample of the
+    workload: one step is the plan over all T*K ids, then dispatch and
+    combine over the first n tokens (n calibrated once to a time budget)."""
+
+    def __init__(self, wl, route):
+        import oracle
+        oracle.build()
+        self.oracle = oracle
+        self.wl, self.route, self.cfg = wl, route, wl.cfg()
+        # host receive buffer: only the rows the sample touches get committed
+        self.recv = np.empty((wl.R * self.cfg["C_max"], wl.H), np.uint16)
+        self.x = None
+
+    def _inputs(self, n):
+        if self.x is None or self.x.shape[0] < n:
+            self.x = inputs.cb_bf16_np(0, inputs.STREAM_X, np.arange(n * self.wl.H)).reshape(n, self.wl.H)
+
+    def step(self, n):
+        o, wl = self.oracle, self.wl
+        T, K = wl.T, wl.K
+        self._inputs(n)
+        t0 = time.perf_counter()
+        pl = o.plan(self.cfg, self.route.topk_idx)
+        t1 = time.perf_counter()
+        d = np.ascontiguousarray(pl["dest"].reshape(T, K)[:n])
+        w = np.ascontiguousarray(self.route.topk_w.reshape(T, K)[:n])
+        t2 = time.perf_counter()
+        o.dispatch(self.cfg, d, self.x[:n], self.recv, n_tokens=n)
+        o.combine(self.cfg, d, self.recv, w, n_tokens=n)
+        t3 = time.perf_counter()
+        b = alg_bytes(dict(self.cfg, S=1, R=n))   # bytes of n tokens
+        return {"gbs": (b["dispatch"] + b["combine"]) / (t3 - t2) / 1e9, "plan_us": (t1 - t0) * 1e6,
+                "rows_per_s": n * K / (t3 - t2), "tokens": n, "seconds": (t1 - t0) + (t3 - t2)}
+
+    def calibrate(self, seconds):
+        n = min(self.wl.T, 128)
+        r = self.step(n)
+        per_tok = max(r["seconds"] - r["plan_us"] * 1e-6, 1e-7) / n
+        return int(max(1, min(self.wl.T, (seconds - r["plan_us"] * 1e-6) / per_tok)))
+
+
+def cpu_baseline(wl, route, seconds):
+    arm = OracleArm(wl, route)
+    n = arm.calibrate(seconds)
+    r = arm.step(n)
+    return {"value": round(r["gbs"], 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "plan_us": round(r["plan_us"], 1), "rows_per_s": round(r["rows_per_s"], 1),
+            "sample": "oracle plan over all %d ids, then dispatch+combine over the first %d of %d "
+                      "tokens (%.1f s, single-threaded C)" % (wl.T * wl.K, r["tokens"], wl.T, r["seconds"])}
+
+
+def run_reference(args):
+    rank, _, world = rank_env()
+    if rank != 0:
+        return
+    wl = inputs.WORKLOADS[args.workload]
+    target = wl.maxvio[0] if wl.maxvio else None
+    route = inputs.routing(wl.R, wl.L, wl.S, wl.K, args.seed, maxvio=target)
+    arm = OracleArm(wl, route)
+    n = arm.calibrate(args.cpu_seconds * 6.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        arm.step(n)
+    res = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        res.append(arm.step(n))
+    wall = time.perf_counter() - t0
+    gbs = float(np.mean([r["gbs"] for r in res]))
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "%s: R=%d L=%d S=%d K=%d H=%d B=%d, maxvio %.2f"
+                               % (wl.name, wl.R, wl.L, wl.S, wl.K, wl.H, wl.B, route.maxvio),
+                   "accumulate": "fp32", "parallelism": "cpu"},
+        "plan_us": round(float(np.mean([r["plan_us"] for r in res])), 1),
+        "rows_per_s": round(float(np.mean([r["rows_per_s"] for r in res])), 1),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "per step: oracle plan over all %d ids, dispatch+combine over the "
+                                   "first %d tokens" % (wl.T * wl.K, n)},
+        "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mid", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--sweep-steps", type=int, default=20)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU oracle sample budget (the reference arm uses 6x this over all its steps)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,230 @@
+/*
+ * moonep.h -- C ABI of the MoonEP hot path on NVIDIA B200 (sm_100a).
+ *
+ * MoonEP ("Moonshot AI Open-Sources MoonEP: A Perfectly Balanced Expert
+ * Parallelism Library for MoE Training", TL;DR) gives every expert-parallel
+ * rank exactly C = S*K rows per MoE layer, whatever the router skew, by
+ * planning a few redundant copies of hot experts online on the GPU and
+ * routing the overflow to them.  This library implements the data path of
+ * one layer for R expert-parallel ranks simulated as partitions of one
+ * symmetric buffer in a single GPU's memory:
+ *
+ *   moonep_plan         histogram of the router's top-K ids, keep/spill split,
+ *                       redundant-expert (spill) planner, all tables; one
+ *                       persistent kernel, no host synchronisation
+ *   moonep_dispatch     sender-side destination rows fused with the row
+ *                       scatter of the hidden states (zero-copy permute)
+ *   moonep_combine      gather of the expert outputs fused with the top-K
+ *                       weighted fp32 sum (unpermute)
+ *   moonep_prefetch     copy of the replicated experts' weights into the
+ *                       receivers' prefetch slots
+ *   moonep_reduce_grad  replica gradients added to the home experts'
+ *                       gradients, used slots cleared
+ *
+ * Notation.  R ranks; L experts per rank; N = R*L experts; expert e lives on
+ * home rank home(e) = e / L at local index e % L (the contiguous blocking of
+ * the weight tensor in "The Busiest Rank Sets Your Step Time: Running
+ * MoonEP's Planning Code Ourselves", section "Installation and integration");
+ * S tokens per rank, T = R*S tokens; K experts per token; H hidden size; B
+ * prefetch slots per rank; C = S*K rows per rank; C_max >= C rows allocated
+ * per rank (rows [C, C_max) are the headroom for fallback rows).  A routed
+ * copy has global index g = (r*S + s)*K + k for token s of rank r.
+ *
+ * Spill rule (the pages give no planning algorithm; this is the library's
+ * rule).  Each home rank keeps its rows in local-expert order up to C.  The
+ * overflow ("spilled chunks"), taken expert by expert in ascending expert
+ * order, goes to the lowest-index ranks that still have room below C and a
+ * free prefetch slot; each (expert, receiver) piece takes one slot.  Rows no
+ * receiver can take stay on the home rank in the headroom, from row C on.
+ * The copies of expert e are numbered j = 0, 1, ... in ascending g; copy j
+ * goes home while j < keep[e], then through e's replica pieces in ascending
+ * receiver order, then to the fallback rows.
+ *
+ * Row layout of rank r in the receive buffer recv[R][C_max][H] (the
+ * "cu_seqlens" the group GEMM consumes, twodots.gr "MoonEP balances AI
+ * experts in MoE models", memory-contract paragraphs): local segments of
+ * experts r*L .. r*L+L-1 packed from row 0, then slots b = 0..B-1 packed
+ * after them, then padding up to C (only if receivers ran out of slots),
+ * then fallback segments of r's own experts from row C.  When no row falls
+ * back every rank holds exactly C rows and rows [0, C) are all used.
+ *
+ * Ownership.  The caller allocates every device buffer, including the plan
+ * workspace; the library never allocates or frees device memory.  Device
+ * pointers must be 16-byte aligned (4-byte for int32/fp32 arrays); H must be
+ * a multiple of 8 so each bf16 row is a whole number of 16-byte vectors.
+ * Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) except moonep_plan_read, which synchronises it.  The
+ * receive buffer's rows are views valid until the next dispatch or combine
+ * into the same buffer (twodots.gr, zero-copy views); rows outside the
+ * plan's segments are never written.
+ *
+ * Errors.  Every call returns MOONEP_OK or a synchronous host error
+ * (MOONEP_ERR_ARG: bad configuration, null or misaligned pointer, size out
+ * of range; MOONEP_ERR_CUDA: a CUDA call failed; MOONEP_ERR_DEVICE: the
+ * device is not sm_100).  moonep_last_error() describes the last one on the
+ * calling thread.  Data-dependent errors are recorded on the device in the
+ * workspace status word without host synchronisation (MOONEP_ST_* bits); a
+ * call that finds an error bit set in the workspace writes nothing.
+ * moonep_plan_read returns the status to the host.
+ *
+ * Limits: 1 <= R <= 64; N <= 4096; 1 <= K <= 64; 8 <= H <= 1048576;
+ * 0 <= B <= 1024 and R*B <= 65536; T*K and R*C_max below 2^31.
+ */
+#ifndef MOONEP_H
+#define MOONEP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOONEP_API __attribute__((visibility("default")))
+#else
+#define MOONEP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+    int32_t R, L, S, K, H, B, C, C_max; /* C must equal S*K; C_max >= C */
+} moonep_cfg_t;
+
+typedef struct {
+    int32_t status;        /* MOONEP_ST_* bits                               */
+    int32_t fallback_rows; /* rows kept on their home rank beyond C          */
+    int32_t n_replicas;    /* replica pieces = used prefetch slots            */
+    int32_t migrated_rows; /* rows placed on a rank other than their home    */
+} moonep_plan_info_t;
+
+/* host return codes */
+#define MOONEP_OK 0
+#define MOONEP_ERR_ARG 1
+#define MOONEP_ERR_CUDA 2
+#define MOONEP_ERR_DEVICE 3
+
+/* device status bits (workspace word 0) */
+#define MOONEP_ST_EXPERT_ID 0x1   /* a top-K id outside [0, N)                          */
+#define MOONEP_ST_CAPACITY 0x2    /* fallback rows do not fit in [C, C_max)             */
+#define MOONEP_ST_TIMEOUT 0x4     /* a bounded device wait gave up                      */
+#define MOONEP_ST_DEST 0x8        /* combine met a destination outside [0, R*C_max)     */
+#define MOONEP_ST_CFG 0x10        /* workspace planned for another configuration        */
+#define MOONEP_ST_ERROR_MASK 0xFF
+#define MOONEP_ST_FALLBACK 0x100  /* informational: fallback_rows > 0                   */
+
+/* Workspace layout: offsets in int32 words from the workspace base.  The
+ * header occupies words [0, MOONEP_WS_HEADER_WORDS):
+ *   0 status, 1 fallback_rows, 2 n_replicas, 3 migrated_rows, 4 n_ranges,
+ *   5..12 the cfg it was planned for, 13 replicated-expert count.
+ * Tables ([N] unless noted): cnt = copies per expert (tokens_per_expert);
+ * keep, spill, home_off (row of e's local segment), fb_cnt, fb_off (row of
+ * e's fallback segment); [R]: load (copies homed on r), deficit (C - load,
+ * floored at 0), fill (rows used below C), slots_used; [R*B]: slot_expert
+ * (-1 = empty), slot_cnt, slot_off, slot_first_j (first copy index j held);
+ * rep_ptr [N+1] (CSR over pieces, pieces in ascending (expert, receiver)
+ * order) and per piece rep_expert, rep_recv, rep_slot, rep_first_j,
+ * rep_cnt; rx_expert (experts with >= 1 piece, ascending); route_ptr [N+1],
+ * route_end, route_base (copy j of e goes to flat row route_base[p] + j for
+ * the first entry p of e with j < route_end[p]); seg_off, seg_len
+ * [R][2L+B] (L local, B slot, L fallback segments per rank); alloc [N][R]
+ * (rows of expert e on rank r, fallback included: the allocation table);
+ * base [N][n_ranges] (copies of e in earlier token ranges; dispatch scratch).
+ * Tables from `cnt` up to, not including, `base` are contiguous. */
+#define MOONEP_WS_HEADER_WORDS 64
+typedef struct {
+    int64_t words;      /* total size in int32 words                  */
+    int64_t n_ranges;   /* token ranges of the dispatch grid           */
+    int64_t max_pieces; /* capacity of the per-piece arrays            */
+    int64_t cnt, keep, spill, home_off, fb_cnt, fb_off;
+    int64_t load, deficit, fill, slots_used;
+    int64_t slot_expert, slot_cnt, slot_off, slot_first_j;
+    int64_t rep_ptr, rep_expert, rep_recv, rep_slot, rep_first_j, rep_cnt;
+    int64_t rx_expert;
+    int64_t route_ptr, route_end, route_base;
+    int64_t seg_off, seg_len;
+    int64_t alloc;
+    int64_t tables_end; /* = base                                      */
+    int64_t base;
+} moonep_ws_layout_t;
+
+/* Per-rank buffer sizes in bytes, as a real deployment would allocate them
+ * ("The Busiest Rank Sets Your Step Time", memory-cost table): dispatch =
+ * C_max*H*2 (bf16 rows), prefetch = B*elems*2 (bf16 weights), reduce =
+ * B*elems*4 (fp32 gradients), for elems weight elements per expert. */
+typedef struct {
+    int64_t dispatch_bytes, prefetch_bytes, reduce_bytes;
+} moonep_rank_bytes_t;
+
+/* Validates cfg and fills the workspace layout.  MOONEP_OK or ERR_ARG. */
+MOONEP_API int moonep_ws_layout(const moonep_cfg_t *cfg, moonep_ws_layout_t *out);
+
+/* Workspace size in bytes for cfg (0 if cfg is invalid). */
+MOONEP_API size_t moonep_plan_workspace_bytes(const moonep_cfg_t *cfg);
+
+/* Per-rank buffer sizes for cfg and `elems_per_expert` weight elements. */
+MOONEP_API int moonep_rank_bytes(const moonep_cfg_t *cfg, int64_t elems_per_expert, moonep_rank_bytes_t *out);
+
+/* Plan ("The Busiest Rank Sets Your Step Time", section "What the technique
+ * is", flowchart: router output -> planning kernel).  topk_idx: device int32
+ * [R][S][K] expert ids.  ws: device workspace of moonep_plan_workspace_bytes
+ * bytes, 16-byte aligned, owned by the caller; fully rewritten.  One memset
+ * of the header and one persistent cooperative kernel; no host sync. */
+MOONEP_API int moonep_plan(const moonep_cfg_t *cfg, const int32_t *topk_idx, void *ws, void *stream);
+
+/* Dispatch (same flowchart: dispatch sends tokens straight to their final
+ * slot on the remote rank).  x: device bf16 [R*S][H] hidden states;
+ * topk_idx: the ids given to moonep_plan; recv: device bf16 [R][C_max][H];
+ * dest: device int32 [R][S][K], written with the flat row rank*C_max + row of
+ * every copy.  recv[dest[g]] = x[token(g)] bitwise. */
+MOONEP_API int moonep_dispatch(const moonep_cfg_t *cfg, void *ws, const void *x, const int32_t *topk_idx,
+                    void *recv, int32_t *dest, void *stream);
+
+/* Combine (same flowchart: combine gathers results back into token order).
+ * y: device bf16 [R][C_max][H] expert outputs in the dispatched layout;
+ * dest: from moonep_dispatch; topk_w: device fp32 [R][S][K] router weights;
+ * out: device bf16 [R*S][H].  out[t] = bf16_rne(acc), acc = 0.0f then
+ * acc = fmaf(w[t][k], float(y[dest[t][k]]), acc) for k = 0..K-1. */
+MOONEP_API int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32_t *dest,
+                   const float *topk_w, void *out, void *stream);
+
+/* Prefetch (twodots.gr: weights of the duplicated experts are loaded into
+ * the prefetch slots [E, E+B) before the experts run).  w_home: device bf16
+ * [N][elems_per_expert]; w_slot: device bf16 [R][B][elems_per_expert];
+ * w_slot[r][b] = w_home[slot_expert[r][b]] for used slots only.
+ * elems_per_expert must be a positive multiple of 8. */
+MOONEP_API int moonep_prefetch(const moonep_cfg_t *cfg, void *ws, const void *w_home, void *w_slot,
+                    int64_t elems_per_expert, void *stream);
+
+/* Replica gradient reduction (twodots.gr: reduce_grad adds the replica
+ * slots of a rank's own experts to the local parameter gradient and clears
+ * the used slots).  g_home: device fp32 [N][elems]; g_rep: device fp32
+ * [R][B][elems].  For each replicated expert, in ascending receiver order,
+ * g_home[e] = g_home[e] + g_rep[r][b] (fp32 adds); then g_rep[r][b] = 0.
+ * Unused slots are not touched: zero g_rep once after allocating it.
+ * elems_per_expert must be a positive multiple of 4. */
+MOONEP_API int moonep_reduce_grad(const moonep_cfg_t *cfg, void *ws, float *g_home, float *g_rep,
+                       int64_t elems_per_expert, void *stream);
+
+/* Reads the plan header (and, if host_tables is not NULL, the tables from
+ * `cnt` up to `base`, i.e. layout.tables_end - layout.cnt words, into
+ * host_tables) after synchronising `stream`. */
+MOONEP_API int moonep_plan_read(const moonep_cfg_t *cfg, const void *ws, moonep_plan_info_t *info,
+                     int32_t *host_tables, void *stream);
+
+/* Upper bound on polls of every bounded device wait (default 1 << 22).  A
+ * wait that runs out sets MOONEP_ST_TIMEOUT and the kernel returns. */
+MOONEP_API int moonep_set_wait_limit(int64_t polls);
+
+/* Token ranges (dispatch CTAs) used for T tokens. */
+MOONEP_API int64_t moonep_num_ranges(int64_t T);
+
+/* Description of the last host error on this thread ("" if none). */
+MOONEP_API const char *moonep_last_error(void);
+
+/* Library version string. */
+MOONEP_API const char *moonep_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOONEP_H */

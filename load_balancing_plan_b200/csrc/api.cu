@@ -1,0 +1,332 @@
+// api.cu -- the C ABI of the MoonEP hot path: argument validation, workspace
+// layout, launch configuration and error reporting.  Every compute step runs
+// in the kernels of plan.cu, dispatch.cu, combine.cu and weights.cu; this
+// file only checks arguments and launches them.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "moonep_internal.cuh"
+
+using namespace moonep;
+
+namespace {
+
+thread_local std::string g_err;
+std::atomic<int64_t> g_wait_limit{int64_t(1) << 22};
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(MOONEP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+struct DeviceInfo {
+    bool ready = false;
+    bool ok = false;
+    int sms = 0;
+    int plan_grid = 0;
+    int combine_grid = 0;
+    size_t plan_smem = 0;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+// Checks the current device once (sm_100, cooperative launch) and caches
+// launch sizes that depend on it.
+int device_info(int N, DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(MOONEP_ERR_DEVICE, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, coop = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        d.ok = (major == 10 && minor == 0 && coop != 0);
+        d.ready = true;
+        if (d.ok) {
+            int nb = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, (const void *)combine_kernel_ptr(), 256, 0);
+            if (e != cudaSuccess) return cuda_fail(e, "occupancy(combine)");
+            d.combine_grid = d.sms * (nb > 0 ? nb : 1);
+        }
+    }
+    if (!d.ok) return fail(MOONEP_ERR_DEVICE, "device %d is not an sm_100 GPU with cooperative launch", dev);
+    // plan kernel: shared memory depends on N
+    const size_t smem = plan_smem_bytes(N);
+    if (smem != d.plan_smem) {
+        e = cudaFuncSetAttribute(plan_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(plan)");
+        int nb = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, plan_kernel_ptr(), 512, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "occupancy(plan)");
+        if (nb < 1) return fail(MOONEP_ERR_DEVICE, "plan kernel does not fit an SM");
+        d.plan_grid = d.sms;  // one CTA per SM; co-resident by the cooperative launch
+        d.plan_smem = smem;
+    }
+    *out = &d;
+    return MOONEP_OK;
+}
+
+int check_cfg(const moonep_cfg_t *c) {
+    if (!c) return fail(MOONEP_ERR_ARG, "cfg is NULL");
+    if (c->R < 1 || c->R > 64) return fail(MOONEP_ERR_ARG, "R=%d outside [1, 64]", c->R);
+    if (c->L < 1) return fail(MOONEP_ERR_ARG, "L=%d < 1", c->L);
+    const int64_t N = (int64_t)c->R * c->L;
+    if (N > 4096) return fail(MOONEP_ERR_ARG, "N=R*L=%lld above 4096", (long long)N);
+    if (c->S < 0) return fail(MOONEP_ERR_ARG, "S=%d < 0", c->S);
+    if (c->K < 1 || c->K > 64) return fail(MOONEP_ERR_ARG, "K=%d outside [1, 64]", c->K);
+    if (c->H < 8 || c->H > (1 << 20) || (c->H % 8) != 0)
+        return fail(MOONEP_ERR_ARG, "H=%d must be a multiple of 8 in [8, 2^20]", c->H);
+    if (c->B < 0 || c->B > 1024 || (int64_t)c->R * c->B > 65536)
+        return fail(MOONEP_ERR_ARG, "B=%d outside [0, 1024] or R*B above 65536", c->B);
+    const int64_t C = (int64_t)c->S * c->K;
+    if (c->C != C) return fail(MOONEP_ERR_ARG, "C=%d must equal S*K=%lld", c->C, (long long)C);
+    if (c->C_max < c->C) return fail(MOONEP_ERR_ARG, "C_max=%d below C=%d", c->C_max, c->C);
+    const int64_t T = (int64_t)c->R * c->S;
+    if (T * c->K > INT32_MAX) return fail(MOONEP_ERR_ARG, "T*K above 2^31-1");
+    if ((int64_t)c->R * c->C_max > INT32_MAX) return fail(MOONEP_ERR_ARG, "R*C_max above 2^31-1");
+    return MOONEP_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_ptr(const void *p, uintptr_t a, const char *name, bool needed) {
+    if (!needed) return MOONEP_OK;
+    if (!p) return fail(MOONEP_ERR_ARG, "%s is NULL", name);
+    if (!aligned(p, a)) return fail(MOONEP_ERR_ARG, "%s is not %d-byte aligned", name, (int)a);
+    return MOONEP_OK;
+}
+
+#define TRY(x)                        \
+    do {                              \
+        int _rc = (x);                \
+        if (_rc != MOONEP_OK) return _rc; \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int moonep_ws_layout(const moonep_cfg_t *cfg, moonep_ws_layout_t *out) {
+    TRY(check_cfg(cfg));
+    if (!out) return fail(MOONEP_ERR_ARG, "out is NULL");
+    compute_layout(*cfg, *out);
+    return MOONEP_OK;
+}
+
+size_t moonep_plan_workspace_bytes(const moonep_cfg_t *cfg) {
+    if (check_cfg(cfg) != MOONEP_OK) return 0;
+    moonep_ws_layout_t l;
+    compute_layout(*cfg, l);
+    return (size_t)l.words * 4;
+}
+
+int moonep_rank_bytes(const moonep_cfg_t *cfg, int64_t elems_per_expert, moonep_rank_bytes_t *out) {
+    TRY(check_cfg(cfg));
+    if (!out) return fail(MOONEP_ERR_ARG, "out is NULL");
+    if (elems_per_expert < 0) return fail(MOONEP_ERR_ARG, "elems_per_expert < 0");
+    out->dispatch_bytes = (int64_t)cfg->C_max * cfg->H * 2;
+    out->prefetch_bytes = (int64_t)cfg->B * elems_per_expert * 2;
+    out->reduce_bytes = (int64_t)cfg->B * elems_per_expert * 4;
+    return MOONEP_OK;
+}
+
+int64_t moonep_num_ranges(int64_t T) { return T < 0 ? 0 : num_ranges(T); }
+
+int moonep_set_wait_limit(int64_t polls) {
+    if (polls < 0) return fail(MOONEP_ERR_ARG, "wait limit < 0");
+    g_wait_limit.store(polls);
+    return MOONEP_OK;
+}
+
+const char *moonep_last_error(void) { return g_err.c_str(); }
+
+const char *moonep_version(void) { return "moonep-b200 0.1 (sm_100a)"; }
+
+int moonep_plan(const moonep_cfg_t *cfg, const int32_t *topk_idx, void *ws, void *stream) {
+    TRY(check_cfg(cfg));
+    const int64_t T = (int64_t)cfg->R * cfg->S;
+    TRY(check_ptr(topk_idx, 4, "topk_idx", T > 0));
+    TRY(check_ptr(ws, 16, "ws", true));
+    const int N = cfg->R * cfg->L;
+    DeviceInfo *d = nullptr;
+    TRY(device_info(N, &d));
+    cudaStream_t s = (cudaStream_t)stream;
+    PlanParams p{};
+    p.cfg = *cfg;
+    p.N = N;
+    p.T = T;
+    compute_layout(*cfg, p.lay);
+    p.Q = p.lay.n_ranges;
+    p.ids = topk_idx;
+    p.ws = (int32_t *)ws;
+    p.wait_limit = g_wait_limit.load();
+    cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)(MOONEP_WS_HEADER_WORDS + N) * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(plan header)");
+    e = launch_plan(p, d->plan_grid, d->plan_smem, s);
+    if (e != cudaSuccess) return cuda_fail(e, "plan kernel launch");
+    return MOONEP_OK;
+}
+
+int moonep_dispatch(const moonep_cfg_t *cfg, void *ws, const void *x, const int32_t *topk_idx, void *recv,
+                    int32_t *dest, void *stream) {
+    TRY(check_cfg(cfg));
+    const int64_t T = (int64_t)cfg->R * cfg->S;
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(x, 16, "x", T > 0));
+    TRY(check_ptr(topk_idx, 4, "topk_idx", T > 0));
+    TRY(check_ptr(recv, 16, "recv", T > 0));
+    TRY(check_ptr(dest, 4, "dest", T > 0));
+    const int N = cfg->R * cfg->L;
+    DeviceInfo *d = nullptr;
+    TRY(device_info(N, &d));
+    if (T == 0) return MOONEP_OK;
+    DispatchParams p{};
+    p.cfg = *cfg;
+    p.N = N;
+    p.T = T;
+    compute_layout(*cfg, p.lay);
+    p.Q = p.lay.n_ranges;
+    p.row_bytes = (uint32_t)cfg->H * 2;
+    size_t smem = 0;
+    const int ctas_per_sm = (int)((p.Q + d->sms - 1) / d->sms);
+    cudaError_t e = dispatch_smem_config(N, p.row_bytes, ctas_per_sm < 1 ? 1 : ctas_per_sm, &p.piece_bytes, &p.npc,
+                                         &smem);
+    if (e != cudaSuccess) return fail(MOONEP_ERR_ARG, "dispatch: no shared-memory configuration for H=%d", cfg->H);
+    p.x = (const uint8_t *)x;
+    p.ids = topk_idx;
+    p.recv = (uint8_t *)recv;
+    p.dest = dest;
+    p.ws = (int32_t *)ws;
+    p.wait_limit = g_wait_limit.load();
+    e = launch_dispatch(p, smem, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch kernel launch");
+    return MOONEP_OK;
+}
+
+int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32_t *dest, const float *topk_w,
+                   void *out, void *stream) {
+    TRY(check_cfg(cfg));
+    const int64_t T = (int64_t)cfg->R * cfg->S;
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(y, 16, "y", T > 0));
+    TRY(check_ptr(dest, 4, "dest", T > 0));
+    TRY(check_ptr(topk_w, 4, "topk_w", T > 0));
+    TRY(check_ptr(out, 16, "out", T > 0));
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (T == 0) return MOONEP_OK;
+    CombineParams p{};
+    p.cfg = *cfg;
+    p.T = T;
+    p.hv = cfg->H / 8;
+    p.upt = (p.hv + 31) / 32;  // units of 32 16-byte vectors
+    p.units = T * p.upt;
+    p.rows_total = (int64_t)cfg->R * cfg->C_max;
+    p.y = (const uint4 *)y;
+    p.dest = dest;
+    p.w = topk_w;
+    p.out = (uint4 *)out;
+    p.ws = (int32_t *)ws;
+    int64_t grid = d->combine_grid;
+    const int64_t need = (p.units + 7) / 8;  // at least one unit per warp
+    if (grid > need) grid = need;
+    if (grid < 1) grid = 1;
+    cudaError_t e = launch_combine(p, (int)grid, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+    return MOONEP_OK;
+}
+
+int moonep_prefetch(const moonep_cfg_t *cfg, void *ws, const void *w_home, void *w_slot, int64_t elems_per_expert,
+                    void *stream) {
+    TRY(check_cfg(cfg));
+    if (elems_per_expert <= 0 || (elems_per_expert % 8) != 0)
+        return fail(MOONEP_ERR_ARG, "elems_per_expert=%lld must be a positive multiple of 8",
+                    (long long)elems_per_expert);
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(w_home, 16, "w_home", true));
+    TRY(check_ptr(w_slot, 16, "w_slot", cfg->B > 0));
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (cfg->B == 0) return MOONEP_OK;
+    CopyParams p{};
+    p.cfg = *cfg;
+    p.vecs = elems_per_expert * 2 / 16;
+    p.src = (const uint4 *)w_home;
+    p.dst = (uint4 *)w_slot;
+    p.ws = (int32_t *)ws;
+    compute_layout(*cfg, p.lay);
+    cudaError_t e = launch_prefetch(p, d->sms * 8, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "prefetch kernel launch");
+    return MOONEP_OK;
+}
+
+int moonep_reduce_grad(const moonep_cfg_t *cfg, void *ws, float *g_home, float *g_rep, int64_t elems_per_expert,
+                       void *stream) {
+    TRY(check_cfg(cfg));
+    if (elems_per_expert <= 0 || (elems_per_expert % 4) != 0)
+        return fail(MOONEP_ERR_ARG, "elems_per_expert=%lld must be a positive multiple of 4",
+                    (long long)elems_per_expert);
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(g_home, 16, "g_home", true));
+    TRY(check_ptr(g_rep, 16, "g_rep", cfg->B > 0));
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (cfg->B == 0) return MOONEP_OK;
+    CopyParams p{};
+    p.cfg = *cfg;
+    p.vecs = elems_per_expert * 4 / 16;
+    p.src = (const uint4 *)g_home;
+    p.dst = (uint4 *)g_rep;
+    p.ws = (int32_t *)ws;
+    compute_layout(*cfg, p.lay);
+    cudaError_t e = launch_reduce_grad(p, d->sms * 8, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "reduce_grad kernel launch");
+    return MOONEP_OK;
+}
+
+int moonep_plan_read(const moonep_cfg_t *cfg, const void *ws, moonep_plan_info_t *info, int32_t *host_tables,
+                     void *stream) {
+    TRY(check_cfg(cfg));
+    TRY(check_ptr(ws, 16, "ws", true));
+    if (!info && !host_tables) return fail(MOONEP_ERR_ARG, "nothing to read");
+    moonep_ws_layout_t l;
+    compute_layout(*cfg, l);
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t hdr[MOONEP_WS_HEADER_WORDS];
+    cudaError_t e = cudaMemcpyAsync(hdr, ws, sizeof hdr, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(header)");
+    if (host_tables) {
+        e = cudaMemcpyAsync(host_tables, (const int32_t *)ws + l.cnt, (size_t)(l.tables_end - l.cnt) * 4,
+                            cudaMemcpyDeviceToHost, s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(tables)");
+    }
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    if (info) {
+        info->status = hdr[HDR_STATUS];
+        info->fallback_rows = hdr[HDR_FALLBACK];
+        info->n_replicas = hdr[HDR_NREP];
+        info->migrated_rows = hdr[HDR_MIGRATED];
+    }
+    return MOONEP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,218 @@
+// dispatch.cu -- moonep_dispatch: sender-side destination rows fused with the
+// row scatter of the hidden states ("The Busiest Rank Sets Your Step Time:
+// Running MoonEP's Planning Code Ourselves", section "What the technique is":
+// the sending side computes the receiver's final per-expert position and
+// writes there, so no receive-buffer-to-compute-buffer copy exists;
+// agentlenshq "MoonshotAI/MoonEP", "How it works": fused permute).
+//
+// One CTA of one warp per token range (the ranges the plan counted).  The
+// warp numbers the range's copies in ascending g: for each group of 32 ids it
+// finds equal experts with __match_any_sync, ranks lanes within a group by
+// popcount, and adds a per-expert running counter kept in shared memory
+// (initialised from the plan's per-range prefix), which gives the copy index
+// j of every (token, k); j maps to a flat row through the expert's route
+// entries.  Lane 0 then moves the data with TMA bulk copies: each row piece
+// of x is loaded once into a shared-memory stage (mbarrier completion) and
+// stored K times straight to its destination rows (bulk async-groups), with
+// kLookahead loads in flight ahead of the stores.  Numbering runs just ahead
+// of the copies, so its cost hides under them.  No multicast.
+#include "moonep_internal.cuh"
+
+namespace moonep {
+
+namespace {
+
+constexpr int kStages = 8;      // shared-memory stages
+constexpr int kLookahead = 6;   // loads issued ahead of the stores
+constexpr int kRing = 2048;     // destination ring entries (ids)
+constexpr uint32_t kMaxPiece = 32768;
+static_assert(kStages - kLookahead - 1 >= 0, "stage reuse needs an older store group");
+
+struct Smem {
+    uint8_t *stages;
+    uint64_t *bars;
+    int32_t *ring;
+    int32_t *ctr;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t *base, uint32_t piece_bytes) {
+    Smem s;
+    s.stages = base;
+    s.bars = reinterpret_cast<uint64_t *>(base + (size_t)kStages * piece_bytes);
+    s.ring = reinterpret_cast<int32_t *>(s.bars + kStages);
+    s.ctr = s.ring + kRing;
+    return s;
+}
+
+// number the next 32 copies of the range (warp-wide)
+__device__ __forceinline__ bool rank_group(const DispatchParams &p, const Smem &sm, int64_t g0, int64_t l0,
+                                           int64_t nids) {
+    const int lane = threadIdx.x & 31;
+    const int32_t *ws = p.ws;
+    const int64_t l = l0 + lane;
+    const bool valid = l < nids;
+    int e = valid ? __ldg(p.ids + g0 + l) : -1;
+    bool bad = false;
+    if (valid && (unsigned)e >= (unsigned)p.N) {
+        e = -1;
+        bad = true;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rin = __popc(peers & lanemask_lt());
+    const int b = e >= 0 ? sm.ctr[e] : 0;
+    __syncwarp();
+    if (e >= 0 && rin == 0) sm.ctr[e] = b + __popc(peers);
+    __syncwarp();
+    int d = -1;
+    if (e >= 0) {
+        const int j = b + rin;
+        const int pb = __ldg(ws + p.lay.route_ptr + e), pe = __ldg(ws + p.lay.route_ptr + e + 1);
+        for (int x = pb; x < pe; ++x)
+            if (j < __ldg(ws + p.lay.route_end + x)) {
+                d = __ldg(ws + p.lay.route_base + x) + j;
+                break;
+            }
+        if (d < 0 || (int64_t)d >= (int64_t)p.cfg.R * p.cfg.C_max) {
+            d = -1;
+            bad = true;
+        }
+    }
+    if (valid) {
+        sm.ring[l % kRing] = d;
+        p.dest[g0 + l] = d;
+    }
+    __syncwarp();
+    return __any_sync(0xffffffffu, bad);
+}
+
+__global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__ DispatchParams p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const int lane = threadIdx.x;
+    int32_t *ws = p.ws;
+    const int64_t q = blockIdx.x;
+    if (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
+    if (!cfg_matches(ws, p.cfg, p.Q)) {
+        if (lane == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
+        return;
+    }
+    const Smem sm = carve(smem_raw, p.piece_bytes);
+    const int K = p.cfg.K, npc = p.npc;
+    for (int e = lane; e < p.N; e += 32) sm.ctr[e] = __ldg(ws + p.lay.base + (int64_t)e * p.Q + q);
+    if (lane == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&sm.bars[s], 1);
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    __syncwarp();
+
+    const int64_t t0 = range_begin(q, p.T, p.Q), t1 = range_begin(q + 1, p.T, p.Q);
+    const int64_t ntok = t1 - t0;
+    const int64_t g0 = t0 * K, nids = ntok * K;
+    const int64_t nunits = ntok * npc;
+    const uint32_t last_piece = p.row_bytes - (uint32_t)(npc - 1) * p.piece_bytes;
+    const uint64_t pol = policy_evict_first();
+
+    int64_t nranked = 0;
+    bool bad = false;
+    bool fail = false;
+    int64_t issued = 0, stored = 0;
+    for (int64_t it = 0; it < nunits + kLookahead; ++it) {
+        if (it < nunits) {
+            const int64_t i = it / npc;
+            while (nranked < (i + 1) * K) {
+                bad |= rank_group(p, sm, g0, nranked, nids);
+                nranked = min(nranked + 32, nids);
+            }
+            if (lane == 0) {
+                const int s = (int)(it % kStages);
+                const int pc = (int)(it - i * npc);
+                const uint32_t bytes = pc == npc - 1 ? last_piece : p.piece_bytes;
+                if (it >= kStages) bulk_wait_read<kStages - kLookahead - 1>();
+                mbar_arrive_expect_tx(&sm.bars[s], bytes);
+                bulk_g2s(sm.stages + (size_t)s * p.piece_bytes,
+                         p.x + (t0 + i) * (int64_t)p.row_bytes + (int64_t)pc * p.piece_bytes, bytes, &sm.bars[s],
+                         pol);
+            }
+            issued = it + 1;
+        }
+        const int64_t j = it - kLookahead;
+        if (j >= 0 && j < nunits) {
+            if (lane == 0) {
+                const int s = (int)(j % kStages);
+                const uint32_t par = (uint32_t)((j / kStages) & 1);
+                int64_t n = 0;
+                while (!mbar_try_wait(&sm.bars[s], par))
+                    if (++n > p.wait_limit) {
+                        fail = true;
+                        break;
+                    }
+                if (!fail) {
+                    const int64_t i = j / npc;
+                    const int pc = (int)(j - i * npc);
+                    const uint32_t bytes = pc == npc - 1 ? last_piece : p.piece_bytes;
+                    const uint8_t *src = sm.stages + (size_t)s * p.piece_bytes;
+                    for (int k = 0; k < K; ++k) {
+                        const int d = sm.ring[(i * K + k) % kRing];
+                        if (d >= 0)
+                            bulk_s2g(p.recv + (int64_t)d * p.row_bytes + (int64_t)pc * p.piece_bytes, src, bytes,
+                                     pol);
+                    }
+                    bulk_commit();
+                }
+            }
+            fail = __shfl_sync(0xffffffffu, (int)fail, 0) != 0;
+            if (fail) break;
+            stored = j + 1;
+        }
+    }
+    if (lane == 0) {
+        bulk_wait_all<0>();
+        if (fail) {
+            // let the loads still in flight land before the CTA exits (with a
+            // limit of its own, at least 2^20 polls, whatever wait_limit is)
+            const int64_t drain = p.wait_limit > (int64_t(1) << 20) ? p.wait_limit : (int64_t(1) << 20);
+            for (int64_t u = stored; u < issued; ++u) {
+                int64_t n = 0;
+                while (!mbar_try_wait(&sm.bars[u % kStages], (uint32_t)((u / kStages) & 1)))
+                    if (++n > drain) break;
+            }
+            atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
+        }
+        if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_DEST);
+    }
+}
+
+}  // namespace
+
+// Shared memory: kStages pieces + barriers + ring + N counters, sized so that
+// `ctas_per_sm` CTAs fit one SM (227 KB usable per SM on sm_100).
+cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uint32_t *piece_bytes, int *npc,
+                                 size_t *smem) {
+    const size_t budget = (size_t)(228 * 1024) / (size_t)ctas_per_sm - 1024;  // 1 KB reserved per CTA
+    const size_t fixed = (size_t)kStages * 8 + (size_t)kRing * 4 + (size_t)N * 4 + 128;
+    if (budget <= fixed) return cudaErrorInvalidValue;
+    size_t maxp = (budget - fixed) / kStages;
+    if (maxp > kMaxPiece) maxp = kMaxPiece;
+    maxp &= ~(size_t)127;
+    if (maxp < 128) return cudaErrorInvalidValue;
+    int n = (int)((row_bytes + maxp - 1) / maxp);
+    uint32_t pb = (uint32_t)(((row_bytes + n - 1) / n + 127) & ~127u);  // 128-byte aligned stages
+    while ((size_t)pb > maxp) {
+        ++n;
+        pb = (uint32_t)(((row_bytes + n - 1) / n + 127) & ~127u);
+    }
+    n = (int)((row_bytes + pb - 1) / pb);
+    *piece_bytes = pb;
+    *npc = n;
+    *smem = (size_t)kStages * pb + fixed;
+    return cudaSuccess;
+}
+
+cudaError_t launch_dispatch(const DispatchParams &p, size_t smem, cudaStream_t s) {
+    cudaError_t err = cudaFuncSetAttribute(dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    dispatch_kernel<<<(unsigned)p.Q, 32, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace moonep

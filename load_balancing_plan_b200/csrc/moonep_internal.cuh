@@ -1,0 +1,256 @@
+// moonep_internal.cuh -- shared pieces of the MoonEP sm_100a library:
+// workspace layout arithmetic (host and device), header word indices, kernel
+// parameter blocks, and inline-PTX wrappers for mbarriers and TMA bulk copies.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moonep.h"
+
+namespace moonep {
+
+// ---------------------------------------------------------------------------
+// workspace header words
+// ---------------------------------------------------------------------------
+enum : int {
+    HDR_STATUS = 0,
+    HDR_FALLBACK = 1,
+    HDR_NREP = 2,
+    HDR_MIGRATED = 3,
+    HDR_NRANGES = 4,
+    HDR_CFG = 5,  // 8 words: R L S K H B C C_max
+    HDR_NRX = 13,
+    HDR_BAR_COUNT = 16,
+    HDR_BAR_GEN = 17,
+    HDR_TOTAL_SPILL = 20,
+    HDR_PEND = 21,
+};
+
+// Token ranges of the dispatch grid: two per SM of a B200 (148 SMs).  The
+// plan counts copies per (expert, range) so each dispatch CTA can number its
+// copies without looking at other ranges.
+constexpr int64_t kRanges = 296;
+
+__host__ __device__ inline int64_t num_ranges(int64_t T) { return T < kRanges ? T : kRanges; }
+
+// token range q of Q: [q*T/Q, (q+1)*T/Q)
+__host__ __device__ inline int64_t range_begin(int64_t q, int64_t T, int64_t Q) { return q * T / Q; }
+
+__host__ __device__ inline int64_t max_pieces(int R, int L, int B) {
+    int64_t N = (int64_t)R * L;
+    int64_t a = (int64_t)R * B, b = N + R;
+    int64_t p = a < b ? a : b;
+    return p > 0 ? p : 1;
+}
+
+// Fills the layout; returns false if the configuration is out of range.
+__host__ __device__ inline void compute_layout(const moonep_cfg_t &c, moonep_ws_layout_t &l) {
+    const int64_t N = (int64_t)c.R * c.L, R = c.R, T = (int64_t)c.R * c.S;
+    const int64_t RB = (int64_t)c.R * c.B > 0 ? (int64_t)c.R * c.B : 1;
+    const int64_t P = max_pieces(c.R, c.L, c.B);
+    const int64_t NR = 2 * N + P;
+    const int64_t SEG = R * (2 * (int64_t)c.L + c.B);
+    int64_t o = MOONEP_WS_HEADER_WORDS;
+    l.n_ranges = num_ranges(T);
+    l.max_pieces = P;
+    l.cnt = o; o += N;
+    l.keep = o; o += N;
+    l.spill = o; o += N;
+    l.home_off = o; o += N;
+    l.fb_cnt = o; o += N;
+    l.fb_off = o; o += N;
+    l.load = o; o += R;
+    l.deficit = o; o += R;
+    l.fill = o; o += R;
+    l.slots_used = o; o += R;
+    l.slot_expert = o; o += RB;
+    l.slot_cnt = o; o += RB;
+    l.slot_off = o; o += RB;
+    l.slot_first_j = o; o += RB;
+    l.rep_ptr = o; o += N + 1;
+    l.rep_expert = o; o += P;
+    l.rep_recv = o; o += P;
+    l.rep_slot = o; o += P;
+    l.rep_first_j = o; o += P;
+    l.rep_cnt = o; o += P;
+    l.rx_expert = o; o += N;
+    l.route_ptr = o; o += N + 1;
+    l.route_end = o; o += NR;
+    l.route_base = o; o += NR;
+    l.seg_off = o; o += SEG;
+    l.seg_len = o; o += SEG;
+    l.alloc = o; o += N * R;
+    o = (o + 3) & ~(int64_t)3;
+    l.tables_end = o;
+    l.base = o;
+    o += N * (l.n_ranges > 0 ? l.n_ranges : 1);
+    o = (o + 3) & ~(int64_t)3;
+    l.words = o;
+}
+
+// ---------------------------------------------------------------------------
+// kernel parameter blocks
+// ---------------------------------------------------------------------------
+struct PlanParams {
+    moonep_cfg_t cfg;
+    int32_t N;
+    int64_t T, Q;
+    const int32_t *ids;
+    int32_t *ws;
+    moonep_ws_layout_t lay;
+    int64_t wait_limit;
+};
+
+struct DispatchParams {
+    moonep_cfg_t cfg;
+    int32_t N;
+    int32_t npc;          // pieces per row
+    int64_t T, Q;
+    uint32_t row_bytes;   // H * 2
+    uint32_t piece_bytes; // stage size; every piece but the last is this size
+    const uint8_t *x;
+    const int32_t *ids;
+    uint8_t *recv;
+    int32_t *dest;
+    int32_t *ws;
+    moonep_ws_layout_t lay;
+    int64_t wait_limit;
+};
+
+struct CombineParams {
+    moonep_cfg_t cfg;
+    int64_t T;
+    int64_t units;        // T * units_per_token
+    int32_t upt;          // units per token
+    int32_t hv;           // 16-byte vectors per row (H / 8)
+    int64_t rows_total;   // R * C_max
+    const uint4 *y;
+    const int32_t *dest;
+    const float *w;
+    uint4 *out;
+    int32_t *ws;
+};
+
+struct CopyParams {
+    moonep_cfg_t cfg;
+    int64_t vecs;         // 16-byte vectors per expert
+    const uint4 *src;
+    uint4 *dst;
+    int32_t *ws;
+    moonep_ws_layout_t lay;
+};
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+#ifdef __CUDACC__
+__device__ __forceinline__ int ld_cg(const int32_t *p) { return __ldcg(p); }
+
+__device__ __forceinline__ bool cfg_matches(const int32_t *ws, const moonep_cfg_t &c, int64_t Q) {
+    const int32_t *h = ws + HDR_CFG;
+    return __ldcg(h + 0) == c.R && __ldcg(h + 1) == c.L && __ldcg(h + 2) == c.S &&
+           __ldcg(h + 3) == c.K && __ldcg(h + 4) == c.H && __ldcg(h + 5) == c.B &&
+           __ldcg(h + 6) == c.C && __ldcg(h + 7) == c.C_max && __ldcg(ws + HDR_NRANGES) == (int32_t)Q;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// TMA bulk copy global -> shared, completion counted on an mbarrier
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32_t bytes, uint64_t *bar,
+                                         uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+
+// TMA bulk copy shared -> global, tracked by bulk async-groups
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src_smem, uint32_t bytes, uint64_t pol) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
+                 "r"(smem_u32(src_smem)), "r"(bytes), "l"(pol)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+#endif
+
+}  // namespace moonep
+
+// launchers (defined in the kernel files, called by the C ABI layer)
+namespace moonep {
+cudaError_t launch_plan(const PlanParams &p, int grid, size_t smem, cudaStream_t s);
+size_t plan_smem_bytes(int N);
+const void *plan_kernel_ptr();
+cudaError_t launch_dispatch(const DispatchParams &p, size_t smem, cudaStream_t s);
+cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uint32_t *piece_bytes,
+                                 int *npc, size_t *smem);
+cudaError_t launch_combine(const CombineParams &p, int grid, cudaStream_t s);
+const void *combine_kernel_ptr();
+cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s);
+cudaError_t launch_reduce_grad(const CopyParams &p, int grid, cudaStream_t s);
+}  // namespace moonep

@@ -1,0 +1,130 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every entry point the header declares, validates its arguments before any
+CUDA call, and sizes its buffers as the pages' memory-cost table does."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def mp():
+    from load_balancing_plan_b200 import build
+    build.build()
+    from load_balancing_plan_b200 import moonep
+    return moonep
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "moonep.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moonep_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(mp):
+    names = _declared()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(mp.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(mp.EXPORTS)
+
+
+def test_version(mp):
+    assert "sm_100a" in mp.version()
+
+
+def _cfg(**kw):
+    c = dict(R=4, L=4, S=64, K=2, H=128, B=4, C=128, C_max=128)
+    c.update(kw)
+    return c
+
+
+@pytest.mark.parametrize("bad", [
+    dict(R=0), dict(R=65), dict(L=0), dict(R=64, L=65), dict(K=0), dict(K=65),
+    dict(H=12), dict(H=0), dict(B=-1), dict(B=1025), dict(C=127), dict(C_max=100),
+    dict(S=-1, C=-2),
+])
+def test_bad_cfg_rejected(mp, bad):
+    c = _cfg(**bad)
+    with pytest.raises(mp.MoonepError) as ei:
+        mp.moonep_ws_layout(c)
+    assert ei.value.code == mp.ERR_ARG
+    assert mp.last_error()
+    assert mp._lib.moonep_plan_workspace_bytes(ctypes.byref(mp.cfg_of(c))) == 0
+    with pytest.raises(mp.MoonepError) as ei:
+        mp.moonep_plan(c, 16, 256, stream=0)
+    assert ei.value.code == mp.ERR_ARG
+
+
+def test_null_and_misaligned_pointers_rejected(mp):
+    c = _cfg()
+    for args in [(None, 256), (16, None), (16, 258), (18, 256)]:
+        with pytest.raises(mp.MoonepError) as ei:
+            mp.moonep_plan(c, *args, stream=0)
+        assert ei.value.code == mp.ERR_ARG
+    with pytest.raises(mp.MoonepError):
+        mp.moonep_dispatch(c, 256, 8, 16, 256, 16, stream=0)      # x misaligned
+    with pytest.raises(mp.MoonepError):
+        mp.moonep_combine(c, 256, 256, 16, 16, 264, stream=0)     # out misaligned
+    with pytest.raises(mp.MoonepError):
+        mp.moonep_prefetch(c, 256, 256, 256, 12, stream=0)        # elems not a multiple of 8
+    with pytest.raises(mp.MoonepError):
+        mp.moonep_reduce_grad(c, 256, 256, 256, 6, stream=0)      # elems not a multiple of 4
+    with pytest.raises(mp.MoonepError):
+        mp.moonep_set_wait_limit(-1)
+
+
+def test_layout_is_consistent(mp):
+    for c in [_cfg(), dict(R=8, L=32, S=8192, K=8, H=7168, B=32, C=65536, C_max=65536),
+              dict(R=16, L=24, S=2048, K=8, H=7168, B=4, C=16384, C_max=20480),
+              _cfg(S=0, C=0, C_max=0), _cfg(B=0)]:
+        lay = mp.moonep_ws_layout(c)
+        offs = [lay[k] for k in mp.LAYOUT_FIELDS[3:]]
+        assert offs == sorted(offs)
+        assert lay["cnt"] == mp.WS_HEADER_WORDS
+        assert lay["tables_end"] == lay["base"] <= lay["words"]
+        assert lay["words"] % 4 == 0
+        T = c["R"] * c["S"]
+        assert lay["n_ranges"] == mp.moonep_num_ranges(T) == min(T, 296)
+        N = c["R"] * c["L"]
+        assert lay["words"] - lay["base"] >= N * lay["n_ranges"]
+        assert mp.moonep_plan_workspace_bytes(c) == 4 * lay["words"]
+
+
+def _memory_table():
+    rows = {}
+    with open(os.path.join(ROOT, "tests", "golden", "memory_table.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            if "=" in line:
+                setup = dict(kv.split("=") for kv in line.split())
+                continue
+            mode, B, pre, red, disp, tot = line.split()
+            rows[mode] = (int(B), float(pre), None if red == "none" else float(red), float(disp),
+                          float(tot))
+    return {k: int(v) for k, v in setup.items()}, rows
+
+
+def test_rank_bytes_match_memory_table(mp):
+    # "The Busiest Rank Sets Your Step Time", memory-cost table: per-rank
+    # prefetch, gradient-reduce and dispatch buffers for S=4096, H=7168,
+    # three projections of FFN size 2048, printed in GiB to two decimals
+    setup, rows = _memory_table()
+    S, K, H, I, P = setup["S"], setup["K"], setup["H"], setup["I"], setup["P"]
+    gib = float(1 << 30)
+    for mode, (B, pre, red, disp, tot) in rows.items():
+        c = dict(R=8, L=32, S=S, K=K, H=H, B=B, C=S * K, C_max=S * K)
+        rb = mp.moonep_rank_bytes(c, P * H * I)
+        assert round(rb["prefetch_bytes"] / gib, 2) == pytest.approx(pre, abs=0.006)
+        assert round(rb["dispatch_bytes"] / gib, 2) == pytest.approx(disp, abs=0.006)
+        total = rb["prefetch_bytes"] + rb["dispatch_bytes"]
+        if red is not None:
+            assert round(rb["reduce_bytes"] / gib, 2) == pytest.approx(red, abs=0.006)
+            total += rb["reduce_bytes"]
+        assert round(total / gib, 2) == pytest.approx(tot, abs=0.006)

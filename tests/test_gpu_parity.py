@@ -1,0 +1,436 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle
+on the same seeded inputs.  Plan tables, destinations, dispatched rows,
+prefetched weights and reduced gradients must be bit-exact; combine must be
+bit-exact against the oracle's bf16 output (same fma order) and within 4e-3
+relative of its fp32 sum.  Small cases are compared in full; the full-size
+workloads in the launch configuration the benchmark times are compared in
+full for every table and destination and on sampled rows and elements."""
+import numpy as np
+import pytest
+
+import oracle
+from load_balancing_plan_b200 import inputs
+from tests import planchecks as pc
+
+pytestmark = pytest.mark.gpu
+
+PLAN_TABLES = ["cnt", "keep", "spill", "home_off", "fb_cnt", "fb_off", "load", "deficit", "fill",
+               "slots_used", "slot_expert", "slot_cnt", "slot_off", "slot_first_j", "rep_ptr",
+               "rep_expert", "rep_recv", "rep_slot", "rep_first_j", "rep_cnt", "seg_off", "seg_len",
+               "alloc"]
+COUNTS = ["fallback_rows", "n_replicas", "migrated_rows"]
+
+
+@pytest.fixture(scope="module")
+def env():
+    import torch
+    from load_balancing_plan_b200 import build
+    build.build()
+    oracle.build()
+    from load_balancing_plan_b200 import harness
+    from load_balancing_plan_b200 import moonep as mp
+    assert torch.cuda.is_available()
+    yield torch, mp, harness
+    torch.cuda.empty_cache()
+
+
+def cfg_of(R, L, S, K, H, B, headroom=0.0):
+    C = S * K
+    return dict(R=R, L=L, S=S, K=K, H=H, B=B, C=C, C_max=int(np.floor((1 + headroom) * C)))
+
+
+def compare_plan(gpl, opl):
+    assert gpl["status"] == opl["status"], (hex(gpl["status"]), hex(opl["status"]))
+    if opl["status"] & (oracle.ST_CAPACITY | oracle.ST_EXPERT_ID):
+        return
+    for k in COUNTS:
+        assert gpl[k] == opl[k], k
+    for k in PLAN_TABLES:
+        a, b = np.asarray(gpl[k]), np.asarray(opl[k])
+        assert a.shape == b.shape, (k, a.shape, b.shape)
+        assert np.array_equal(a, b), k
+
+
+def x_host(seed, T, H):
+    return inputs.cb_bf16_np(seed, inputs.STREAM_X, np.arange(T * H, dtype=np.int64)).reshape(T, H)
+
+
+def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_seed=0):
+    """Every step on a small problem, compared element by element."""
+    torch, mp, harness = env
+    R, L, S, K, H, B, Cm = (cfg[n] for n in ("R", "L", "S", "K", "H", "B", "C_max"))
+    N, T = R * L, R * S
+    prob = harness.Problem(cfg, poison=True, w_elems=w_elems, g_elems=g_elems)
+    prob.set_routing(ids, w)
+    prob.fill_x(seed)
+    prob.fill_weights(seed)
+    prob.fill_g_rep(seed)
+    prob.plan()
+    gpl = prob.read_plan()
+    opl = oracle.plan(cfg, ids)
+    compare_plan(gpl, opl)
+    failed = bool(opl["status"] & (oracle.ST_CAPACITY | oracle.ST_EXPERT_ID))
+    if not failed:
+        pc.check_plan(cfg, ids, gpl | {"dest": opl["dest"]})
+
+    prob.dispatch()
+    torch.cuda.synchronize()
+    recv_g = harness.to_u16(prob.recv)
+    dest_g = prob.dest[:T * K].cpu().numpy()
+    if failed:
+        # a failed plan: dispatch writes nothing
+        assert np.all(recv_g == 0xFFFF)
+        assert np.all(dest_g == -7)
+        return prob, gpl, opl
+    assert np.array_equal(dest_g, opl["dest"].reshape(-1))
+    xh = x_host(seed, T, H)
+    assert np.array_equal(harness.to_u16(prob.x[:T]), xh)
+    recv_o = np.full((R * Cm, H), 0xFFFF, np.uint16)
+    oracle.dispatch(cfg, opl["dest"], xh, recv_o)
+    assert np.array_equal(recv_g, recv_o)
+
+    # stand-in expert, then combine, against the oracle's chain
+    scale = inputs.expert_scales(N, scale_seed)
+    y_g = prob.expert_scale(scale)
+    y_o = recv_o.copy()
+    oracle.expert_scale(cfg, opl, recv_o, scale, y_o)
+    assert np.array_equal(harness.to_u16(y_g), y_o)
+    prob.combine(y_g)
+    torch.cuda.synchronize()
+    out_g = harness.to_u16(prob.out[:T])
+    out_o, acc_o = oracle.combine(cfg, opl["dest"], y_o, w)
+    assert np.array_equal(out_g, out_o)
+    og = inputs.bf16_bits_to_f32_np(out_g).astype(np.float64)
+    nz = acc_o != 0
+    assert np.all(og[~nz] == 0)
+    if nz.any():
+        assert np.max(np.abs(og[nz] - acc_o[nz]) / np.abs(acc_o[nz])) <= 4e-3
+
+    # prefetch and reduce_grad
+    if w_elems:
+        w_home = harness.to_u16(prob.w_home)
+        ws_o = np.full((max(R * B, 1), w_elems), 0xFFFF, np.uint16)
+        oracle.prefetch(cfg, opl["slot_expert"], w_home, ws_o, w_elems)
+        prob.prefetch()
+        torch.cuda.synchronize()
+        assert np.array_equal(harness.to_u16(prob.w_slot), ws_o)
+    if g_elems:
+        gh = prob.g_home.cpu().numpy().copy()
+        gr = prob.g_rep.cpu().numpy().copy()
+        prob.reduce_grad()
+        torch.cuda.synchronize()
+        oracle.reduce_grad(cfg, opl, gh, gr, g_elems)
+        gh_g, gr_g = prob.g_home.cpu().numpy(), prob.g_rep.cpu().numpy()
+        assert np.array_equal(gh_g.view(np.uint32), gh.view(np.uint32))
+        assert np.array_equal(gr_g.view(np.uint32), gr.view(np.uint32))
+    return prob, gpl, opl
+
+
+# ---------------------------------------------------------------------------
+# small problems, compared in full
+# ---------------------------------------------------------------------------
+
+def test_device_generator_matches_host(env):
+    torch, mp, harness = env
+    t = torch.empty(1 << 20, dtype=torch.bfloat16, device="cuda")
+    inputs.cb_fill_torch(t, 5, inputs.STREAM_X, offset=12345)
+    h = inputs.cb_bf16_np(5, inputs.STREAM_X, np.arange(12345, 12345 + (1 << 20)))
+    assert np.array_equal(t.view(torch.int16).cpu().numpy().view(np.uint16), h)
+    f = torch.empty(1 << 20, dtype=torch.float32, device="cuda")
+    inputs.cb_fill_torch(f, 6, inputs.STREAM_G_REP)
+    assert np.array_equal(f.cpu().numpy(), inputs.cb_f32_np(6, inputs.STREAM_G_REP, np.arange(1 << 20)))
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_tiny_workload(env, seed):
+    w = inputs.WORKLOADS["tiny"]
+    r = inputs.routing(w.R, w.L, w.S, w.K, seed, alpha=1.0)
+    run_full_compare(env, w.cfg(), r.topk_idx, r.topk_w, seed=seed, w_elems=2 * 128 * 256 // 64,
+                     g_elems=128 * 256 // 32)
+
+
+def test_tiny_reduce_grad_full_size_grads(env):
+    # tiny workload with the stated gradient size H*I = 128*256 per replica
+    w = inputs.WORKLOADS["tiny"]
+    r = inputs.routing(w.R, w.L, w.S, w.K, 1, alpha=1.0)
+    run_full_compare(env, w.cfg(), r.topk_idx, r.topk_w, seed=1, w_elems=2 * 128 * 256,
+                     g_elems=128 * 256)
+
+
+@pytest.mark.parametrize("case", [
+    # R, L, S, K, H, B, headroom, routing
+    (4, 4, 64, 2, 128, 4, 0.0, "balanced"),
+    (1, 7, 500, 1, 8, 2, 0.0, "uniform"),              # single rank: stable sort
+    (3, 5, 333, 3, 296, 2, 1.0, "skew"),                # ragged sizes, headroom
+    (4, 4, 100, 2, 64, 0, 3.0, "skew"),                 # no slots: all overflow falls back
+    (16, 24, 64, 8, 64, 4, 0.25, "skew4"),              # inference-style slot limit
+    (8, 8, 40, 64, 16, 8, 0.0, "skew"),                 # K at its maximum
+    (2, 2, 300, 2, 20008, 2, 1.0, "skew"),              # rows split in several pieces
+    (64, 64, 32, 8, 32, 8, 0.0, "skew"),                # N at its maximum
+    (5, 3, 1000, 4, 40, 3, 1.0, "skew"),                # T > ranges: several tokens per range
+])
+def test_edge_cases(env, case):
+    R, L, S, K, H, B, hr, kind = case
+    cfg = cfg_of(R, L, S, K, H, B, hr)
+    rng = np.random.default_rng(R * 1000 + S)
+    if kind == "balanced":
+        r = inputs.routing(R, L, S, K, 0, balanced=True)
+        ids, w = r.topk_idx, r.topk_w
+    elif kind == "uniform":
+        ids = rng.integers(0, R * L, (R, S, K)).astype(np.int32)
+        w = rng.random((R, S, K)).astype(np.float32)
+    else:
+        target = 4.0 if kind == "skew4" else None
+        r = inputs.routing(R, L, S, K, 0, alpha=1.0 if target is None else None, maxvio=target)
+        ids, w = r.topk_idx, r.topk_w
+    run_full_compare(env, cfg, ids, w, w_elems=64, g_elems=64)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_random_histograms(env, seed):
+    rng = np.random.default_rng(seed)
+    R, L, S, K, B = 8, 4, 64, 4, 1 + seed
+    cnt = pc.random_counts(rng, R * L, R * S, K, skew=1.0 + seed)
+    ids = pc.ids_from_counts(cnt, R, S, K)
+    # shuffle tokens so the copies of an expert spread over the token ranges
+    flat = ids.reshape(R * S, K)[rng.permutation(R * S)]
+    ids = np.ascontiguousarray(flat.reshape(R, S, K))
+    w = rng.random((R, S, K)).astype(np.float32)
+    run_full_compare(env, cfg_of(R, L, S, K, 64, B, 3.0), ids, w)
+
+
+def test_empty_input(env):
+    torch, mp, harness = env
+    cfg = cfg_of(4, 2, 0, 2, 64, 2)
+    ids = np.zeros((4, 0, 2), np.int32)
+    prob = harness.Problem(cfg, w_elems=64, g_elems=64)
+    prob.plan()
+    prob.dispatch()
+    prob.combine()
+    prob.prefetch()
+    prob.reduce_grad()
+    gpl = prob.read_plan()
+    compare_plan(gpl, oracle.plan(cfg, ids))
+
+
+def test_capacity_error_writes_nothing(env):
+    R, L, S, K, B = 4, 2, 2, 2, 0
+    cfg = cfg_of(R, L, S, K, 16, B)
+    ids = pc.ids_from_counts(np.array([4, 4, 2, 2, 2, 2, 0, 0]), R, S, K)
+    w = np.full((R, S, K), 0.5, np.float32)
+    prob, gpl, opl = run_full_compare(env, cfg, ids, w)
+    assert gpl["status"] & oracle.ST_CAPACITY
+
+
+def test_bad_expert_id_writes_nothing(env):
+    torch, mp, harness = env
+    cfg = cfg_of(2, 2, 4, 2, 16, 2)
+    ids = np.array([0, 1, 2, 3, 0, 4, 1, 2, 3, 0, 1, 2, 0, 1, 2, 3], np.int32).reshape(2, 4, 2)
+    w = np.full((2, 4, 2), 0.5, np.float32)
+    prob, gpl, opl = run_full_compare(env, cfg, ids, w)
+    assert gpl["status"] & mp.ST_EXPERT_ID
+    g_home0, g_rep0 = prob.g_home.clone(), prob.g_rep.clone()
+    prob.combine()
+    prob.prefetch()
+    prob.reduce_grad()
+    torch.cuda.synchronize()
+    assert np.all(harness.to_u16(prob.out) == 0xFFFF)
+    assert np.all(harness.to_u16(prob.w_slot) == 0xFFFF)
+    assert torch.equal(prob.g_rep, g_rep0) and torch.equal(prob.g_home, g_home0)
+
+
+def test_workspace_of_other_cfg_is_refused(env):
+    torch, mp, harness = env
+    cfg = cfg_of(4, 4, 64, 2, 128, 4)
+    r = inputs.routing(4, 4, 64, 2, 0, alpha=1.0)
+    prob = harness.Problem(cfg, poison=True)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.plan()
+    other = dict(cfg, B=3)      # same workspace size class, different cfg
+    assert mp.moonep_plan_workspace_bytes(other) <= prob.ws.numel() * 4
+    mp.moonep_dispatch(other, prob.ws, prob.x, prob.ids, prob.recv, prob.dest)
+    info = mp.moonep_plan_read(cfg, prob.ws)
+    assert info["status"] & mp.ST_CFG
+    assert np.all(harness.to_u16(prob.recv) == 0xFFFF)
+
+
+def test_replan_on_same_workspace(env):
+    torch, mp, harness = env
+    cfg = cfg_of(4, 4, 64, 2, 128, 4)
+    prob = harness.Problem(cfg)
+    for seed in range(3):
+        r = inputs.routing(4, 4, 64, 2, seed, alpha=1.0 + seed)
+        prob.set_routing(r.topk_idx, r.topk_w)
+        prob.plan()
+        compare_plan(prob.read_plan(), oracle.plan(cfg, r.topk_idx))
+
+
+def test_plan_wait_timeout_sets_status(env):
+    # a wait limit of zero makes the plan's grid barrier give up; the status
+    # says so, later calls write nothing, and the next plan is clean again
+    torch, mp, harness = env
+    cfg = cfg_of(4, 4, 64, 2, 128, 4)
+    r = inputs.routing(4, 4, 64, 2, 0, alpha=1.0)
+    prob = harness.Problem(cfg, poison=True)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    try:
+        mp.moonep_set_wait_limit(0)
+        prob.plan()
+        info = prob.read_plan(tables=False)
+    finally:
+        mp.moonep_set_wait_limit(1 << 22)
+    assert info["status"] & mp.ST_TIMEOUT
+    prob.dispatch()
+    torch.cuda.synchronize()
+    assert np.all(harness.to_u16(prob.recv) == 0xFFFF)
+    prob.plan()
+    compare_plan(prob.read_plan(), oracle.plan(cfg, r.topk_idx))
+
+
+def test_dispatch_wait_timeout_is_reported_or_complete(env):
+    torch, mp, harness = env
+    cfg = cfg_of(8, 4, 512, 4, 4096, 4, headroom=1.0)
+    r = inputs.routing(8, 4, 512, 4, 0, alpha=1.0)
+    assert oracle.plan(cfg, r.topk_idx)["status"] & 0xFF == 0
+    prob = harness.Problem(cfg)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.fill_x(0)
+    prob.plan()
+    try:
+        mp.moonep_set_wait_limit(0)
+        prob.dispatch()
+        info = prob.read_plan(tables=False)
+    finally:
+        mp.moonep_set_wait_limit(1 << 22)
+    opl = oracle.plan(cfg, r.topk_idx)
+    if not info["status"] & mp.ST_TIMEOUT:
+        assert np.array_equal(prob.dest.cpu().numpy(), opl["dest"].reshape(-1))
+    # the context stays usable
+    prob.plan()
+    prob.dispatch()
+    torch.cuda.synchronize()
+    assert prob.read_plan(tables=False)["status"] & mp.ST_ERROR_MASK == 0
+    assert np.array_equal(prob.dest.cpu().numpy(), opl["dest"].reshape(-1))
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads (the benchmark's launch configuration), sampled
+# ---------------------------------------------------------------------------
+
+# (workload, target maxvio, seed); inference seed 1 needs the headroom
+FULL = [("mid", 2.0, 0), ("skew", 0.0, 0), ("skew", 8.0, 0), ("inference", 4.0, 0),
+        ("inference", 4.0, 1), ("training", 8.0, 0)]
+
+
+@pytest.mark.parametrize("name,maxvio,seed", FULL)
+def test_full_size(env, name, maxvio, seed):
+    torch, mp, harness = env
+    wl = inputs.WORKLOADS[name]
+    cfg = wl.cfg()
+    R, L, S, K, H, B, Cm = (cfg[n] for n in ("R", "L", "S", "K", "H", "B", "C_max"))
+    N, T = wl.N, wl.T
+    r = inputs.routing(R, L, S, K, seed, maxvio=maxvio)
+    assert maxvio == 0.0 or abs(r.maxvio - maxvio) <= 0.05 * maxvio
+    w_elems = wl.w_elems if name in ("mid", "training") else 0
+    g_elems = wl.g_elems if name in ("mid", "training") else 0
+    prob = harness.Problem(cfg, poison=True, w_elems=w_elems, g_elems=g_elems)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.fill_x(seed)
+    prob.fill_weights(seed)
+    prob.fill_g_rep(seed)
+    prob.plan()
+    if w_elems:
+        prob.prefetch()
+    prob.dispatch()
+    prob.combine()
+    torch.cuda.synchronize()
+    gpl = prob.read_plan()
+    opl = oracle.plan(cfg, r.topk_idx)
+    compare_plan(gpl, opl)
+    if name != "inference":
+        assert gpl["fallback_rows"] == 0
+    assert bool(gpl["status"] & mp.ST_FALLBACK) == (gpl["fallback_rows"] > 0)
+    if gpl["fallback_rows"] == 0:
+        assert np.all(gpl["alloc"].sum(0) == cfg["C"])        # exactly S*K rows per rank
+    else:
+        assert np.all(gpl["alloc"].sum(0) <= Cm)
+    if name == "inference" and seed == 1:
+        assert gpl["fallback_rows"] > 0                         # the headroom path is exercised
+    dest = prob.dest[:T * K].cpu().numpy()
+    assert np.array_equal(dest, opl["dest"].reshape(-1))
+
+    rng = np.random.default_rng(1)
+    # dispatched rows: sampled copies, against the generator by index
+    gs = rng.choice(T * K, 2048, replace=False)
+    rows = harness.to_u16(prob.recv[torch.from_numpy(dest[gs]).long().cuda()])
+    tok = gs // K
+    want = inputs.cb_bf16_np(seed, inputs.STREAM_X, (tok[:, None] * H + np.arange(H)[None, :]))
+    assert np.array_equal(rows, want)
+    # rows outside every segment stay untouched
+    used = np.zeros(R * Cm, bool)
+    used[dest] = True
+    free = np.nonzero(~used)[0]
+    if free.size:
+        pick = rng.choice(free, min(256, free.size), replace=False)
+        assert np.all(harness.to_u16(prob.recv[torch.from_numpy(pick).cuda()]) == 0xFFFF)
+    # combine with the identity expert: out[t] from K copies of x[t]
+    ts = rng.choice(T, 256, replace=False)
+    xs = inputs.cb_bf16_np(seed, inputs.STREAM_X, ts[:, None] * H + np.arange(H)[None, :])
+    mini = dict(R=1, L=1, S=len(ts), K=K, H=H, B=0, C=len(ts) * K, C_max=len(ts) * K)
+    y_mini = np.repeat(xs, K, axis=0)
+    d_mini = np.arange(len(ts) * K, dtype=np.int32).reshape(1, len(ts), K)
+    w_mini = r.topk_w.reshape(T, K)[ts]
+    out_o, acc_o = oracle.combine(mini, d_mini, y_mini, w_mini)
+    out_g = harness.to_u16(prob.out[torch.from_numpy(ts).cuda()])
+    assert np.array_equal(out_g, out_o)
+    # prefetch: every used slot, sampled elements
+    if w_elems:
+        idx = np.sort(rng.choice(w_elems, 4096, replace=False))
+        it = torch.from_numpy(idx).cuda()
+        for slot in np.nonzero(gpl["slot_expert"] >= 0)[0]:
+            e = int(gpl["slot_expert"][slot])
+            got = harness.to_u16(prob.w_slot[int(slot)][it])
+            assert np.array_equal(got, inputs.cb_bf16_np(seed, inputs.STREAM_W, e * w_elems + idx))
+        for slot in np.nonzero(gpl["slot_expert"] < 0)[0][:4]:
+            assert np.all(harness.to_u16(prob.w_slot[int(slot)][it]) == 0xFFFF)
+    # reduce_grad: sampled columns, against the oracle on those columns
+    if g_elems:
+        prob.reduce_grad()
+        torch.cuda.synchronize()
+        idx = np.sort(rng.choice(g_elems, 2048, replace=False))
+        it = torch.from_numpy(idx).cuda()
+        gh = inputs.cb_f32_np(seed, inputs.STREAM_G_HOME,
+                              np.arange(N)[:, None] * g_elems + idx[None, :]).astype(np.float32)
+        gr = inputs.cb_f32_np(seed, inputs.STREAM_G_REP,
+                              np.arange(R * B)[:, None] * g_elems + idx[None, :]).astype(np.float32)
+        gh = np.ascontiguousarray(gh)
+        gr = np.ascontiguousarray(gr)
+        oracle.reduce_grad(cfg, opl, gh, gr, len(idx))
+        got_h = prob.g_home[:, it].cpu().numpy()
+        got_r = prob.g_rep[:, it].cpu().numpy()
+        assert np.array_equal(got_h.view(np.uint32), gh.view(np.uint32))
+        assert np.array_equal(got_r.view(np.uint32), gr.view(np.uint32))
+        rel = np.abs(got_h - gh) / np.maximum(np.abs(gh), 1e-30)
+        assert rel.max() <= 1e-6
+    del prob
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("maxvio", [0.0, 1.0, 2.0, 4.0, 8.0])
+@pytest.mark.parametrize("seed", [1, 2, 3, 4])
+def test_skew_sweep_plans(env, maxvio, seed):
+    # plan tables and destinations of the skew-sweep workload for every seed
+    torch, mp, harness = env
+    wl = inputs.WORKLOADS["skew"]
+    cfg = wl.cfg()
+    r = inputs.routing(wl.R, wl.L, wl.S, wl.K, seed, maxvio=maxvio)
+    prob = harness.Problem(dict(cfg, H=8))   # H does not enter the plan or dest
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.plan()
+    prob.dispatch()
+    torch.cuda.synchronize()
+    cfg8 = dict(cfg, H=8)
+    opl = oracle.plan(cfg8, r.topk_idx)
+    compare_plan(prob.read_plan(), opl)
+    assert np.array_equal(prob.dest.cpu().numpy(), opl["dest"].reshape(-1))
+    assert opl["fallback_rows"] == 0
