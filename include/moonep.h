@@ -211,6 +211,22 @@ MOONEP_API int moonep_reduce_grad(const moonep_cfg_t *cfg, void *ws, float *g_ho
 MOONEP_API int moonep_plan_read(const moonep_cfg_t *cfg, const void *ws, moonep_plan_info_t *info,
                      int32_t *host_tables, void *stream);
 
+/* The pages have no counterpart to this entry point.  moonep_plan for
+ * callers that cannot allocate device memory themselves (a plug-in handed
+ * tensors but no allocator, or a process whose device memory belongs to a
+ * pooled allocator that must not see extra cudaMalloc calls): the workspace
+ * lives in a static 2 MiB device array inside the library (held by every
+ * GPU that loads it until exit) and the plan header and tables, words
+ * [0, layout.tables_end) of the workspace layout, are copied into
+ * tables_out (device, 16-byte aligned, caller-owned; readable with
+ * moonep_plan_read).  Same kernel and results as moonep_plan; allocates
+ * nothing.  Configurations whose workspace exceeds 2 MiB are refused with
+ * MOONEP_ERR_ARG.  The first call on a device looks up the array's device
+ * address; make that first call before any stream capture.  Every call shares
+ * the array, so calls that overlap on the GPU race: serialise them. */
+MOONEP_API int moonep_plan_noalloc(const moonep_cfg_t *cfg, const int32_t *topk_idx, int32_t *tables_out,
+                                   void *stream);
+
 /* Upper bound on polls of every bounded device wait (default 1 << 22).  A
  * wait that runs out sets MOONEP_ST_TIMEOUT and the kernel returns. */
 MOONEP_API int moonep_set_wait_limit(int64_t polls);

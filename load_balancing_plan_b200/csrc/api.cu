@@ -114,6 +114,15 @@ int check_ptr(const void *p, uintptr_t a, const char *name, bool needed) {
     return MOONEP_OK;
 }
 
+}  // namespace
+
+namespace moonep {
+// records a host error for moonep_last_error (used by other translation units)
+int set_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace moonep
+
+namespace {
+
 #define TRY(x)                        \
     do {                              \
         int _rc = (x);                \

@@ -253,4 +253,5 @@ cudaError_t launch_combine(const CombineParams &p, int grid, cudaStream_t s);
 const void *combine_kernel_ptr();
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s);
 cudaError_t launch_reduce_grad(const CopyParams &p, int grid, cudaStream_t s);
+int set_error(int code, const char *msg);
 }  // namespace moonep

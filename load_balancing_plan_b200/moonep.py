@@ -70,6 +70,7 @@ _sig = {
     "moonep_prefetch": ([_CP, _vp, _vp, _vp, _i64, _vp], ctypes.c_int),
     "moonep_reduce_grad": ([_CP, _vp, _vp, _vp, _i64, _vp], ctypes.c_int),
     "moonep_plan_read": ([_CP, _vp, ctypes.POINTER(PlanInfo), _vp, _vp], ctypes.c_int),
+    "moonep_plan_noalloc": ([_CP, _vp, _vp, _vp], ctypes.c_int),
     "moonep_set_wait_limit": ([_i64], ctypes.c_int),
     "moonep_num_ranges": ([_i64], _i64),
     "moonep_last_error": ([], ctypes.c_char_p),
@@ -154,6 +155,14 @@ def moonep_set_wait_limit(polls) -> None:
 
 def moonep_plan(cfg, topk_idx, ws, stream=None) -> None:
     _check(_lib.moonep_plan(ctypes.byref(cfg_of(cfg)), _p(topk_idx), _p(ws), _stream(stream)))
+
+
+def moonep_plan_noalloc(cfg, topk_idx, tables_out, stream=None) -> None:
+    """moonep_plan without a caller workspace: the library's static device
+    workspace is used and the header + tables are copied to tables_out
+    (at least layout["tables_end"] int32 words)."""
+    _check(_lib.moonep_plan_noalloc(ctypes.byref(cfg_of(cfg)), _p(topk_idx), _p(tables_out),
+                                    _stream(stream)))
 
 
 def moonep_dispatch(cfg, ws, x, topk_idx, recv, dest, stream=None) -> None:
