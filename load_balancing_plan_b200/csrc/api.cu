@@ -60,12 +60,7 @@ int device_info(int N, DeviceInfo **out) {
         cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
         d.ok = (major == 10 && minor == 0 && coop != 0);
         d.ready = true;
-        if (d.ok) {
-            int nb = 0;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, (const void *)combine_kernel_ptr(), 256, 0);
-            if (e != cudaSuccess) return cuda_fail(e, "occupancy(combine)");
-            d.combine_grid = d.sms * (nb > 0 ? nb : 1);
-        }
+        d.combine_grid = d.sms;  // one persistent combine CTA per SM
     }
     if (!d.ok) return fail(MOONEP_ERR_DEVICE, "device %d is not an sm_100 GPU with cooperative launch", dev);
     // plan kernel: shared memory depends on N
@@ -246,7 +241,9 @@ int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32
     p.cfg = *cfg;
     p.T = T;
     p.hv = cfg->H / 8;
-    p.upt = (p.hv + 31) / 32;  // units of 32 16-byte vectors
+    size_t smem = 0;
+    if (combine_config(cfg->K, p.hv, &p.chunk_bytes, &p.upt, &p.stages, &smem) != cudaSuccess)
+        return fail(MOONEP_ERR_ARG, "combine: no shared-memory configuration for K=%d H=%d", cfg->K, cfg->H);
     p.units = T * p.upt;
     p.rows_total = (int64_t)cfg->R * cfg->C_max;
     p.y = (const uint4 *)y;
@@ -254,11 +251,11 @@ int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32
     p.w = topk_w;
     p.out = (uint4 *)out;
     p.ws = (int32_t *)ws;
+    p.wait_limit = g_wait_limit.load();
     int64_t grid = d->combine_grid;
-    const int64_t need = (p.units + 7) / 8;  // at least one unit per warp
-    if (grid > need) grid = need;
+    if (grid > p.units) grid = p.units;
     if (grid < 1) grid = 1;
-    cudaError_t e = launch_combine(p, (int)grid, (cudaStream_t)stream);
+    cudaError_t e = launch_combine(p, (int)grid, smem, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
     return MOONEP_OK;
 }

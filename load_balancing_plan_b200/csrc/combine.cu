@@ -5,12 +5,20 @@
 // "How it works": fused unpermute).
 //
 // out[t] = bf16_rne(acc), acc = 0.0f, acc = fmaf(w[t][k], float(y[dest[t][k]]),
-// acc) for k = 0..K-1 in that order.  HBM-bound: K row reads and one row
-// write per token.  A unit of work is one token x 256 hidden values (one
-// 16-byte vector per lane of a warp); each warp takes a contiguous run of
-// units, so it reloads a token's K destinations and weights only when the
-// token changes, and keeps min(K, 8) independent 16-byte loads per lane in
-// flight.  Rows are read and written with streaming cache hints.
+// acc) for k = 0..K-1 in that order.
+//
+// HBM-bound: K row reads and one row write per token.  One persistent CTA
+// per SM runs a TMA pipeline.  A unit of work is one chunk of one token's
+// row (chunk_bytes of each of its K source rows).  Warp 0 produces: for each
+// unit it waits for a free shared-memory stage, posts the byte count on the
+// stage's "full" mbarrier, and its lanes issue the K bulk copies
+// global -> shared (lane k copies row k); it also parks the token's K
+// weights next to the stage.  Warps 1..8 consume: they wait on "full", read
+// the K chunks from shared memory (16 bytes per thread per row, conflict
+// free), accumulate in fp32 in k order, store the bf16 result with a
+// streaming hint and release the stage on its "empty" mbarrier.  Up to
+// `stages` units are in flight per SM, so the gather is never short of
+// outstanding bytes.  Every wait is bounded.  No multicast.
 #include <cuda_bf16.h>
 
 #include "moonep_internal.cuh"
@@ -19,10 +27,28 @@ namespace moonep {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kVecPerLane = 1;          // 16-byte vectors per lane per unit
-constexpr int kUnitVecs = 32 * kVecPerLane;
-constexpr int kKBatch = 8;              // rows loaded before their fmas
+#ifndef MOONEP_COMBINE_CONSUMERS
+#define MOONEP_COMBINE_CONSUMERS 8   // consumer warps per CTA
+#endif
+#ifndef MOONEP_COMBINE_CHUNK
+#define MOONEP_COMBINE_CHUNK 8192    // bytes of each source row per unit (upper bound)
+#endif
+#ifndef MOONEP_COMBINE_SMEM_KB
+#define MOONEP_COMBINE_SMEM_KB 220   // shared memory for the stages
+#endif
+
+constexpr int kConsumerWarps = MOONEP_COMBINE_CONSUMERS;
+constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kMaxStages = 8;
+constexpr int kMaxK = 64;
+
+struct StageInfo {
+    int64_t t;       // token
+    int32_t c;       // chunk of the row
+    uint32_t bytes;  // bytes of this chunk
+    int32_t valid;   // all K destinations in range
+    int32_t pad;
+};
 
 __device__ __forceinline__ void fma8(float *acc, float w, const uint4 &v) {
     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
@@ -42,84 +68,178 @@ __device__ __forceinline__ uint4 pack8(const float *acc) {
     return v;
 }
 
-__global__ void __launch_bounds__(kThreads, 2) combine_kernel(const __grid_constant__ CombineParams p) {
-    if (__ldcg(p.ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
-    const int lane = threadIdx.x & 31;
-    if (!cfg_matches(p.ws, p.cfg, num_ranges(p.T))) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.ws + HDR_STATUS, MOONEP_ST_CFG);
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// bounded wait; returns false if it gave up
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int64_t limit) {
+    int64_t n = 0;
+    while (!mbar_try_wait(bar, parity))
+        if (++n > limit) return false;
+    return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_constant__ CombineParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    int32_t *ws = p.ws;
+    if (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
+    if (!cfg_matches(ws, p.cfg, num_ranges(p.T))) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
     }
-    const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
-    const int64_t u0 = gw * p.units / nw, u1 = (gw + 1) * p.units / nw;
     const int K = p.cfg.K;
-    const int hv = p.hv;
+    const int NS = p.stages;
+    const uint32_t CH = p.chunk_bytes;
+    const size_t stage_bytes = (size_t)K * CH;
+    uint8_t *stages = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)NS * stage_bytes);
+    uint64_t *empty = full + kMaxStages;
+    StageInfo *info = reinterpret_cast<StageInfo *>(empty + kMaxStages);
+    float *sw = reinterpret_cast<float *>(info + kMaxStages);  // [kMaxStages][kMaxK]
 
-    int64_t cur = -1;
-    int dk = 0, dk2 = 0;      // dest of k = lane, lane + 32
-    float wk = 0.f, wk2 = 0.f;
-    bool tok_ok = true;
-    bool bad = false;
-    for (int64_t u = u0; u < u1; ++u) {
-        const int64_t t = u / p.upt;
-        const int sg = (int)(u - t * p.upt);
-        if (t != cur) {
-            cur = t;
-            dk = lane < K ? __ldg(p.dest + t * K + lane) : 0;
-            wk = lane < K ? __ldg(p.w + t * K + lane) : 0.f;
-            dk2 = lane + 32 < K ? __ldg(p.dest + t * K + lane + 32) : 0;
-            wk2 = lane + 32 < K ? __ldg(p.w + t * K + lane + 32) : 0.f;
-            const bool okl = (dk >= 0 && (int64_t)dk < p.rows_total) && (dk2 >= 0 && (int64_t)dk2 < p.rows_total);
-            tok_ok = __all_sync(0xffffffffu, okl);
-            bad |= !tok_ok;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
         }
-        if (!tok_ok) continue;
-        float acc[kVecPerLane][8];
-#pragma unroll
-        for (int v = 0; v < kVecPerLane; ++v)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[v][i] = 0.f;
-        const int vb = sg * kUnitVecs + lane;
-        for (int k0 = 0; k0 < K; k0 += kKBatch) {
-            uint4 ld[kKBatch][kVecPerLane];
-            float wb[kKBatch];
-#pragma unroll
-            for (int kk = 0; kk < kKBatch; ++kk) {
-                const int k = k0 + kk;
-                const int d = __shfl_sync(0xffffffffu, k < 32 ? dk : dk2, k & 31);
-                wb[kk] = __shfl_sync(0xffffffffu, k < 32 ? wk : wk2, k & 31);
-#pragma unroll
-                for (int v = 0; v < kVecPerLane; ++v) {
-                    const int vi = vb + v * 32;
-                    if (k < K && vi < hv)
-                        ld[kk][v] = __ldcs(p.y + (int64_t)d * hv + vi);
-                    else
-                        ld[kk][v] = make_uint4(0, 0, 0, 0);
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+
+    const int64_t u0 = (int64_t)blockIdx.x * p.units / gridDim.x;
+    const int64_t u1 = (int64_t)(blockIdx.x + 1) * p.units / gridDim.x;
+    const int64_t row_bytes = (int64_t)p.hv * 16;
+    const uint32_t last = (uint32_t)(row_bytes - (int64_t)(p.upt - 1) * CH);
+    const uint64_t pol = policy_evict_first();
+    const uint8_t *y = reinterpret_cast<const uint8_t *>(p.y);
+
+    if (warp == 0) {
+        // ------------------------------------------------------- producer
+        int64_t cur = -1;
+        int dk = 0, dk2 = 0;
+        float wk = 0.f, wk2 = 0.f;
+        int valid = 1;
+        bool bad = false, fail = false;
+        int64_t i = 0;
+        for (int64_t u = u0; u < u1; ++u, ++i) {
+            const int s = (int)(i % NS);
+            if (i >= NS) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait_bounded(&empty[s], (uint32_t)(((i / NS) - 1) & 1), p.wait_limit);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    fail = true;
+                    break;
                 }
             }
-#pragma unroll
-            for (int kk = 0; kk < kKBatch; ++kk) {
-                if (k0 + kk < K) {
-#pragma unroll
-                    for (int v = 0; v < kVecPerLane; ++v) fma8(acc[v], wb[kk], ld[kk][v]);
-                }
+            const int64_t t = u / p.upt;
+            const int c = (int)(u - t * p.upt);
+            if (t != cur) {
+                cur = t;
+                dk = lane < K ? __ldg(p.dest + t * K + lane) : 0;
+                wk = lane < K ? __ldg(p.w + t * K + lane) : 0.f;
+                dk2 = lane + 32 < K ? __ldg(p.dest + t * K + lane + 32) : 0;
+                wk2 = lane + 32 < K ? __ldg(p.w + t * K + lane + 32) : 0.f;
+                const bool okl = dk >= 0 && (int64_t)dk < p.rows_total && dk2 >= 0 && (int64_t)dk2 < p.rows_total;
+                valid = __all_sync(0xffffffffu, okl) ? 1 : 0;
+                bad |= !valid;
+            }
+            const uint32_t bytes = c == p.upt - 1 ? last : CH;
+            if (lane < K) sw[s * kMaxK + lane] = wk;
+            if (lane + 32 < K) sw[s * kMaxK + lane + 32] = wk2;
+            if (lane == 0) {
+                info[s].t = t;
+                info[s].c = c;
+                info[s].bytes = bytes;
+                info[s].valid = valid;
+                mbar_arrive_expect_tx(&full[s], valid ? (uint32_t)K * bytes : 0u);
+            }
+            __syncwarp();
+            if (valid) {
+                uint8_t *st = stages + (size_t)s * stage_bytes;
+                if (lane < K)
+                    bulk_g2s(st + (size_t)lane * CH, y + (int64_t)dk * row_bytes + (int64_t)c * CH, bytes, &full[s],
+                             pol);
+                if (lane + 32 < K)
+                    bulk_g2s(st + (size_t)(lane + 32) * CH, y + (int64_t)dk2 * row_bytes + (int64_t)c * CH, bytes,
+                             &full[s], pol);
             }
         }
+        // every copy issued must land before the CTA exits
+        if (lane == 0) {
+            const int64_t drain = p.wait_limit > (int64_t(1) << 20) ? p.wait_limit : (int64_t(1) << 20);
+            for (int64_t j = (i > NS ? i - NS : 0); j < i; ++j)
+                mbar_wait_bounded(&full[j % NS], (uint32_t)((j / NS) & 1), drain);
+            if (fail) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
+            if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_DEST);
+        }
+    } else {
+        // ------------------------------------------------------- consumers
+        const int ct = threadIdx.x - 32;
+        int64_t i = 0;
+        for (int64_t u = u0; u < u1; ++u, ++i) {
+            const int s = (int)(i % NS);
+            if (!mbar_wait_bounded(&full[s], (uint32_t)((i / NS) & 1), p.wait_limit)) {
+                if (ct == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
+                break;
+            }
+            const StageInfo inf = info[s];
+            if (inf.valid) {
+                const uint8_t *st = stages + (size_t)s * stage_bytes;
+                const float *wv = sw + s * kMaxK;
+                const int nv = (int)(inf.bytes >> 4);
+                uint4 *dst = p.out + inf.t * p.hv + (int64_t)inf.c * (CH >> 4);
+                for (int v = ct; v < nv; v += 32 * kConsumerWarps) {
+                    float acc[8];
 #pragma unroll
-        for (int v = 0; v < kVecPerLane; ++v) {
-            const int vi = vb + v * 32;
-            if (vi < hv) __stcs(p.out + t * hv + vi, pack8(acc[v]));
+                    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+                    for (int k = 0; k < K; ++k) {
+                        const uint4 val = *reinterpret_cast<const uint4 *>(st + (size_t)k * CH + (size_t)v * 16);
+                        fma8(acc, wv[k], val);
+                    }
+                    __stcs(dst + v, pack8(acc));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
-    if (bad && lane == 0) atomicOr(p.ws + HDR_STATUS, MOONEP_ST_DEST);
 }
 
 }  // namespace
 
 const void *combine_kernel_ptr() { return (const void *)combine_kernel; }
 
-cudaError_t launch_combine(const CombineParams &p, int grid, cudaStream_t s) {
-    combine_kernel<<<grid, kThreads, 0, s>>>(p);
+// chunk: the row split into equal pieces (multiples of 16 bytes) of at most
+// MOONEP_COMBINE_CHUNK bytes, fewer when K is large (K*chunk <= 8 chunks);
+// stages fill MOONEP_COMBINE_SMEM_KB of shared memory (at most kMaxStages).
+// Large bulk copies matter: 8 KB copies move about 1.5x the bytes per second
+// of 4 KB ones on B200.
+cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages, size_t *smem) {
+    if (K < 1 || K > kMaxK || hv < 1) return cudaErrorInvalidValue;
+    uint32_t cap = MOONEP_COMBINE_CHUNK;
+    while ((uint32_t)K * cap > 8u * MOONEP_COMBINE_CHUNK && cap > 512) cap >>= 1;
+    const uint32_t row = (uint32_t)hv * 16;
+    const int n = (int)((row + cap - 1) / cap);
+    const uint32_t ch = (((row + n - 1) / n) + 15) & ~15u;
+    const size_t stage = (size_t)K * ch;
+    const size_t fixed = 2 * kMaxStages * 8 + kMaxStages * sizeof(StageInfo) + kMaxStages * kMaxK * 4 + 128;
+    int ns = (int)((MOONEP_COMBINE_SMEM_KB * 1024 - fixed) / stage);
+    if (ns > kMaxStages) ns = kMaxStages;
+    if (ns < 2) return cudaErrorInvalidValue;
+    *chunk = ch;
+    *upt = (int)((row + ch - 1) / ch);
+    *stages = ns;
+    *smem = (size_t)ns * stage + fixed;
+    return cudaSuccess;
+}
+
+cudaError_t launch_combine(const CombineParams &p, int grid, size_t smem, cudaStream_t s) {
+    cudaError_t err = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    combine_kernel<<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 

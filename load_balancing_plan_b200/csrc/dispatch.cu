@@ -22,8 +22,17 @@ namespace moonep {
 
 namespace {
 
-constexpr int kStages = 8;      // shared-memory stages
-constexpr int kLookahead = 6;   // loads issued ahead of the stores
+#ifndef MOONEP_DISPATCH_STAGES
+#define MOONEP_DISPATCH_STAGES 8     // shared-memory stages
+#endif
+#ifndef MOONEP_DISPATCH_LOOKAHEAD
+#define MOONEP_DISPATCH_LOOKAHEAD 6  // loads issued ahead of the stores
+#endif
+#ifndef MOONEP_DISPATCH_HINTS
+#define MOONEP_DISPATCH_HINTS 1      // bit 0: evict-first on the x loads, bit 1: on the row stores
+#endif
+constexpr int kStages = MOONEP_DISPATCH_STAGES;
+constexpr int kLookahead = MOONEP_DISPATCH_LOOKAHEAD;
 constexpr int kRing = 2048;     // destination ring entries (ids)
 constexpr uint32_t kMaxPiece = 32768;
 static_assert(kStages - kLookahead - 1 >= 0, "stage reuse needs an older store group");
@@ -129,9 +138,12 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
                 const uint32_t bytes = pc == npc - 1 ? last_piece : p.piece_bytes;
                 if (it >= kStages) bulk_wait_read<kStages - kLookahead - 1>();
                 mbar_arrive_expect_tx(&sm.bars[s], bytes);
-                bulk_g2s(sm.stages + (size_t)s * p.piece_bytes,
-                         p.x + (t0 + i) * (int64_t)p.row_bytes + (int64_t)pc * p.piece_bytes, bytes, &sm.bars[s],
-                         pol);
+                uint8_t *dsm = sm.stages + (size_t)s * p.piece_bytes;
+                const uint8_t *src = p.x + (t0 + i) * (int64_t)p.row_bytes + (int64_t)pc * p.piece_bytes;
+                if (MOONEP_DISPATCH_HINTS & 1)
+                    bulk_g2s(dsm, src, bytes, &sm.bars[s], pol);
+                else
+                    bulk_g2s_plain(dsm, src, bytes, &sm.bars[s]);
             }
             issued = it + 1;
         }
@@ -153,9 +165,13 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
                     const uint8_t *src = sm.stages + (size_t)s * p.piece_bytes;
                     for (int k = 0; k < K; ++k) {
                         const int d = sm.ring[(i * K + k) % kRing];
-                        if (d >= 0)
-                            bulk_s2g(p.recv + (int64_t)d * p.row_bytes + (int64_t)pc * p.piece_bytes, src, bytes,
-                                     pol);
+                        if (d >= 0) {
+                            uint8_t *dst = p.recv + (int64_t)d * p.row_bytes + (int64_t)pc * p.piece_bytes;
+                            if (MOONEP_DISPATCH_HINTS & 2)
+                                bulk_s2g(dst, src, bytes, pol);
+                            else
+                                bulk_s2g_plain(dst, src, bytes);
+                        }
                     }
                     bulk_commit();
                 }

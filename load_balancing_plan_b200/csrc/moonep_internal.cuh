@@ -30,7 +30,10 @@ enum : int {
 // Token ranges of the dispatch grid: two per SM of a B200 (148 SMs).  The
 // plan counts copies per (expert, range) so each dispatch CTA can number its
 // copies without looking at other ranges.
-constexpr int64_t kRanges = 296;
+#ifndef MOONEP_RANGES
+#define MOONEP_RANGES 296
+#endif
+constexpr int64_t kRanges = MOONEP_RANGES;
 
 __host__ __device__ inline int64_t num_ranges(int64_t T) { return T < kRanges ? T : kRanges; }
 
@@ -122,14 +125,17 @@ struct CombineParams {
     moonep_cfg_t cfg;
     int64_t T;
     int64_t units;        // T * units_per_token
-    int32_t upt;          // units per token
+    int32_t upt;          // units (row chunks) per token
     int32_t hv;           // 16-byte vectors per row (H / 8)
     int64_t rows_total;   // R * C_max
+    uint32_t chunk_bytes; // bytes of each of the K rows per unit (last chunk may be shorter)
+    int32_t stages;       // shared-memory stages
     const uint4 *y;
     const int32_t *dest;
     const float *w;
     uint4 *out;
     int32_t *ws;
+    int64_t wait_limit;
 };
 
 struct CopyParams {
@@ -209,6 +215,21 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32
         : "memory");
 }
 
+// TMA bulk copy shared -> global, tracked by bulk async-groups (no cache hint)
+__device__ __forceinline__ void bulk_s2g_plain(void *dst, const void *src_smem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src_smem)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// TMA bulk copy global -> shared without a cache hint
+__device__ __forceinline__ void bulk_g2s_plain(void *dst_smem, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst_smem)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // TMA bulk copy shared -> global, tracked by bulk async-groups
 __device__ __forceinline__ void bulk_s2g(void *dst, const void *src_smem, uint32_t bytes, uint64_t pol) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
@@ -249,7 +270,8 @@ const void *plan_kernel_ptr();
 cudaError_t launch_dispatch(const DispatchParams &p, size_t smem, cudaStream_t s);
 cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uint32_t *piece_bytes,
                                  int *npc, size_t *smem);
-cudaError_t launch_combine(const CombineParams &p, int grid, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams &p, int grid, size_t smem, cudaStream_t s);
+cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages, size_t *smem);
 const void *combine_kernel_ptr();
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s);
 cudaError_t launch_reduce_grad(const CopyParams &p, int grid, cudaStream_t s);

@@ -34,35 +34,42 @@ namespace moonep {
 namespace {
 
 constexpr int kPlanThreads = 512;
+
+// MOONEP_PLAN_TRACE: development builds stamp %globaltimer (ns) at the phase
+// boundaries of CTA 0 into header words 32..47 of the workspace.
+#ifdef MOONEP_PLAN_TRACE
+__device__ __forceinline__ void trace(int32_t *ws, int slot) {
+    if (threadIdx.x == 0) {
+        uint64_t t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        reinterpret_cast<unsigned long long *>(ws + 32)[slot] = t;
+    }
+}
+#define TRACE(ws, slot) trace(ws, slot)
+#else
+#define TRACE(ws, slot) ((void)0)
+#endif
 constexpr int kWarps = kPlanThreads / 32;
 constexpr int kMaxR = 64;
+constexpr int kIdBatch = 8;
 
-// Exclusive scan of n ints (in and out may alias) by the whole CTA; returns
-// the total.  Each thread owns a contiguous run of ceil(n / 512) entries.
-__device__ int block_excl_scan(const int *in, int *out, int n, int *s_tmp) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = (n + kPlanThreads - 1) / kPlanThreads;
-    const int lo = min(tid * per, n), hi = min(lo + per, n);
+// Exclusive scan of n ints (in and out may alias) by one warp; returns the
+// total.  Lane l owns the contiguous run [l*per, (l+1)*per), per = ceil(n/32).
+__device__ int warp_excl_scan(const int *in, int *out, int n) {
+    const int lane = threadIdx.x & 31;
+    const int per = (n + 31) >> 5;
+    const int lo = min(lane * per, n), hi = min(lo + per, n);
     int sum = 0;
     for (int i = lo; i < hi; ++i) sum += in[i];
-    int incl = warp_incl_scan(sum);
-    if (lane == 31) s_tmp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int v = lane < kWarps ? s_tmp[lane] : 0;
-        int iv = warp_incl_scan(v);
-        if (lane < kWarps) s_tmp[lane] = iv - v;
-        if (lane == kWarps - 1) s_tmp[32] = iv;
-    }
-    __syncthreads();
-    int run = s_tmp[warp] + incl - sum;
+    const int incl = warp_incl_scan(sum);
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int run = incl - sum;
     for (int i = lo; i < hi; ++i) {
-        int v = in[i];
+        const int v = in[i];
         out[i] = run;
         run += v;
     }
-    int total = s_tmp[32];
-    __syncthreads();
+    __syncwarp();
     return total;
 }
 
@@ -134,41 +141,45 @@ __device__ void scan_column(int32_t *col, int64_t Q) {
     }
 }
 
-// The planner (one CTA).  Shared memory: six arrays of N ints + small ones.
+// The planner: one warp of CTA 0.  Every intermediate lives in shared memory
+// (seven arrays of N ints and a few of R); global memory is only written.
+// One warp needs no block-wide barriers, which dominate at these sizes.
 __device__ void plan_tables(const PlanParams &p, int *sm) {
     const moonep_cfg_t &c = p.cfg;
     const int N = p.N, R = c.R, L = c.L, B = c.B, C = c.C, Cm = c.C_max;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int SEG = 2 * L + B;
+    const int lane = threadIdx.x & 31;
     const moonep_ws_layout_t &lay = p.lay;
     int32_t *ws = p.ws;
 
-    int *s_cnt = sm;        // copies per expert
-    int *s_x = sm + N;      // scans
-    int *s_sp = sm + 2 * N; // spill per expert
-    int *s_ce = sm + 3 * N; // chunk end positions in the spill stream
-    int *s_ch = sm + 4 * N; // chunk -> expert
-    int *s_y = sm + 5 * N;  // scratch
+    int *s_cnt = sm;          // copies per expert
+    int *s_x = sm + N;        // scans: cnt prefix, then spill-stream starts, then fb_cnt
+    int *s_sp = sm + 2 * N;   // spill per expert
+    int *s_ce = sm + 3 * N;   // chunk end positions in the spill stream, then fb prefix
+    int *s_ch = sm + 4 * N;   // chunk -> expert
+    int *s_y = sm + 5 * N;    // chunk index, then pieces per expert -> rep_ptr
+    int *s_hoff = sm + 6 * N; // row of the expert's local segment
     __shared__ int s_def[kMaxR], s_rp[kMaxR], s_rt[kMaxR], s_ri0[kMaxR], s_rnp[kMaxR], s_rpb[kMaxR];
-    __shared__ int s_tmp[33];
-    __shared__ int s_misc[4];  // 0 p_end, 1 n_rx, 2 pieces, 3 capacity error
 
-    for (int e = tid; e < N; e += kPlanThreads) s_cnt[e] = __ldcg(ws + lay.cnt + e);
-    if (tid < 4) s_misc[tid] = 0;
-    __syncthreads();
-
+    TRACE(ws, 3);
     // keep/spill: each home rank keeps rows in local-expert order up to C
-    const int total = block_excl_scan(s_cnt, s_x, N, s_tmp);
-    for (int e = tid; e < N; e += kPlanThreads) {
+    const int total = warp_excl_scan(s_cnt, s_x, N);
+    for (int e = lane; e < N; e += 32) {
         const int h = e / L;
         const int hx = s_x[e] - s_x[h * L];
         const int ce = s_cnt[e];
         const int k = min(ce, max(0, C - hx));
-        ws[lay.keep + e] = k;
-        ws[lay.home_off + e] = min(hx, C);
-        ws[lay.spill + e] = ce - k;
+        const int ho = min(hx, C);
+        s_hoff[e] = ho;
         s_sp[e] = ce - k;
+        s_y[e] = ce - k > 0 ? 1 : 0;
+        ws[lay.keep + e] = k;
+        ws[lay.home_off + e] = ho;
+        ws[lay.spill + e] = ce - k;
+        ws[lay.seg_off + h * SEG + (e - h * L)] = ho;
+        ws[lay.seg_len + h * SEG + (e - h * L)] = k;
     }
-    for (int h = tid; h < R; h += kPlanThreads) {
+    for (int h = lane; h < R; h += 32) {
         const int lo = s_x[h * L];
         const int hi = h + 1 < R ? s_x[(h + 1) * L] : total;
         const int ld = hi - lo;
@@ -177,74 +188,67 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[lay.deficit + h] = d;
         s_def[h] = d;
     }
-    __syncthreads();
+    __syncwarp();
 
     // the spill stream and its chunks
-    const int total_spill = block_excl_scan(s_sp, s_x, N, s_tmp);  // s_x = A_e
-    for (int e = tid; e < N; e += kPlanThreads) s_y[e] = s_sp[e] > 0 ? 1 : 0;
-    __syncthreads();
-    const int M = block_excl_scan(s_y, s_y, N, s_tmp);  // s_y = chunk index
-    for (int e = tid; e < N; e += kPlanThreads)
+    const int total_spill = warp_excl_scan(s_sp, s_x, N);  // s_x = A_e
+    const int M = warp_excl_scan(s_y, s_y, N);             // s_y = chunk index
+    for (int e = lane; e < N; e += 32)
         if (s_sp[e] > 0) {
             s_ce[s_y[e]] = s_x[e] + s_sp[e];
             s_ch[s_y[e]] = e;
         }
-    __syncthreads();
+    __syncwarp();
+    TRACE(ws, 4);
 
     // receiver walk: receiver r takes the stream from p_r until its deficit
     // is filled or it has touched B chunks
-    if (warp == 0) {
-        int pos = 0, i0 = 0;
-        for (int r = 0; r < R; ++r) {
-            const int d = s_def[r];
-            int take = 0, np = 0, ir = i0;
-            const int pr = pos;
-            if (d > 0 && pos < total_spill && B > 0) {
-                i0 = advance_chunk(s_ce, M, i0, pos);
-                const int i1 = min(i0 + B - 1, M - 1);
-                take = min(d, s_ce[i1] - pos);
-                const int il = advance_chunk(s_ce, M, i0, pos + take - 1);
-                np = il - i0 + 1;
-                ir = i0;
-                pos += take;
-            }
-            if (lane == 0) {
-                s_rp[r] = pr;
-                s_rt[r] = take;
-                s_ri0[r] = ir;
-                s_rnp[r] = np;
-            }
+    int pos = 0, i0 = 0;
+    for (int r = 0; r < R; ++r) {
+        const int d = s_def[r];
+        int take = 0, np = 0, ir = i0;
+        const int pr = pos;
+        if (d > 0 && pos < total_spill && B > 0) {
+            i0 = advance_chunk(s_ce, M, i0, pos);
+            const int i1 = min(i0 + B - 1, M - 1);
+            take = min(d, s_ce[i1] - pos);
+            const int il = advance_chunk(s_ce, M, i0, pos + take - 1);
+            np = il - i0 + 1;
+            ir = i0;
+            pos += take;
         }
-        // pieces per receiver -> exclusive prefix (R <= 64: two per lane)
-        const int a = lane < R ? s_rnp[lane] : 0;
-        const int b = lane + 32 < R ? s_rnp[lane + 32] : 0;
-        const int ia = warp_incl_scan(a);
-        const int tot_a = __shfl_sync(0xffffffffu, ia, 31);
-        const int ib = warp_incl_scan(b);
-        if (lane < R) s_rpb[lane] = ia - a;
-        if (lane + 32 < R) s_rpb[lane + 32] = tot_a + ib - b;
-        const int P = tot_a + __shfl_sync(0xffffffffu, ib, 31);
-        // replicated experts are the chunks that start before the walk's end
-        const int nrx = pos > 0 ? advance_chunk(s_ce, M, 0, pos - 1) + 1 : 0;
         if (lane == 0) {
-            s_misc[0] = pos;
-            s_misc[1] = nrx;
-            s_misc[2] = P;
+            s_rp[r] = pr;
+            s_rt[r] = take;
+            s_ri0[r] = ir;
+            s_rnp[r] = np;
         }
     }
-    __syncthreads();
-    const int p_end = s_misc[0], nrx = s_misc[1], P = s_misc[2];
-
-    for (int r = tid; r < R; r += kPlanThreads) {
+    __syncwarp();
+    const int p_end = pos;
+    // pieces per receiver -> exclusive prefix (R <= 64: two per lane)
+    const int na = lane < R ? s_rnp[lane] : 0;
+    const int nb = lane + 32 < R ? s_rnp[lane + 32] : 0;
+    const int ia = warp_incl_scan(na);
+    const int tot_a = __shfl_sync(0xffffffffu, ia, 31);
+    const int ib = warp_incl_scan(nb);
+    if (lane < R) s_rpb[lane] = ia - na;
+    if (lane + 32 < R) s_rpb[lane + 32] = tot_a + ib - nb;
+    const int P = tot_a + __shfl_sync(0xffffffffu, ib, 31);
+    // replicated experts are the chunks that start before the walk's end
+    const int nrx = p_end > 0 ? advance_chunk(s_ce, M, 0, p_end - 1) + 1 : 0;
+    for (int e = lane; e < N; e += 32) s_y[e] = 0;  // pieces per expert
+    for (int r = lane; r < R; r += 32) {
         ws[lay.fill + r] = C - s_def[r] + s_rt[r];
         ws[lay.slots_used + r] = s_rnp[r];
     }
-    for (int e = tid; e < N; e += kPlanThreads) s_y[e] = 0;  // pieces per expert
-    __syncthreads();
+    __syncwarp();
+    TRACE(ws, 5);
 
-    // pieces and slots
-    for (int idx = tid; idx < R * B; idx += kPlanThreads) {
+    // pieces, slots and their segments, route entries and alloc entries
+    for (int idx = lane; idx < R * B; idx += 32) {
         const int r = idx / B, b = idx - r * B;
+        const int sg = r * SEG + L + b;
         if (b < s_rnp[r]) {
             const int i = s_ri0[r] + b;
             const int e = s_ch[i];
@@ -263,23 +267,26 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
             ws[lay.slot_cnt + idx] = n;
             ws[lay.slot_off + idx] = soff;
             ws[lay.slot_first_j + idx] = fj;
+            ws[lay.seg_off + sg] = soff;
+            ws[lay.seg_len + sg] = n;
             // route entry of this piece: after e's home entry and e's earlier pieces
             ws[lay.route_end + 2 * e + 1 + gp] = fj + n;
             ws[lay.route_base + 2 * e + 1 + gp] = r * Cm + soff - fj;
+            ws[lay.alloc + (int64_t)e * R + r] = n;
             atomicAdd(&s_y[e], 1);
         } else {
+            const int fill = C - s_def[r] + s_rt[r];
             ws[lay.slot_expert + idx] = -1;
             ws[lay.slot_cnt + idx] = 0;
-            ws[lay.slot_off + idx] = C - s_def[r] + s_rt[r];
+            ws[lay.slot_off + idx] = fill;
             ws[lay.slot_first_j + idx] = 0;
+            ws[lay.seg_off + sg] = fill;
+            ws[lay.seg_len + sg] = 0;
         }
     }
-    for (int x = tid; x < nrx; x += kPlanThreads) ws[lay.rx_expert + x] = s_ch[x];
-    __syncthreads();
-    block_excl_scan(s_y, s_y, N, s_tmp);  // s_y = rep_ptr
-
-    // fallback rows: the stream beyond the walk's end, per chunk
-    for (int e = tid; e < N; e += kPlanThreads) {
+    for (int x = lane; x < nrx; x += 32) ws[lay.rx_expert + x] = s_ch[x];
+    // fallback rows: the stream beyond the walk's end, per chunk (s_x: A_e -> fb_cnt)
+    for (int e = lane; e < N; e += 32) {
         int fb = 0;
         if (s_sp[e] > 0) {
             const int cs = s_x[e], ce = cs + s_sp[e];
@@ -288,61 +295,38 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         s_x[e] = fb;
         ws[lay.fb_cnt + e] = fb;
     }
-    __syncthreads();
-    block_excl_scan(s_x, s_ce, N, s_tmp);  // s_ce = exclusive prefix of fb_cnt
-    // (s_x still holds fb_cnt)
-    for (int e = tid; e < N; e += kPlanThreads) {
+    __syncwarp();
+    TRACE(ws, 6);
+    warp_excl_scan(s_y, s_y, N);   // s_y = rep_ptr
+    warp_excl_scan(s_x, s_ce, N);  // s_ce = exclusive prefix of fb_cnt
+    int cap_err = 0;
+    for (int e = lane; e < N; e += 32) {
         const int h = e / L;
         const int fbo = C + (s_ce[e] - s_ce[h * L]);
         const int fb = s_x[e];
         const int keep = s_cnt[e] - s_sp[e];
         const int rp = s_y[e];
         const int rn = (e + 1 < N ? s_y[e + 1] : P) - rp;
+        const int sg = h * SEG + L + B + (e - h * L);
         ws[lay.fb_off + e] = fbo;
         ws[lay.rep_ptr + e] = rp;
         ws[lay.route_ptr + e] = 2 * e + rp;
         ws[lay.route_end + 2 * e + rp] = keep;
-        ws[lay.route_base + 2 * e + rp] = h * Cm + ws[lay.home_off + e];
+        ws[lay.route_base + 2 * e + rp] = h * Cm + s_hoff[e];
         ws[lay.route_end + 2 * e + rp + rn + 1] = s_cnt[e];
         ws[lay.route_base + 2 * e + rp + rn + 1] = h * Cm + fbo - (s_cnt[e] - fb);
-        if ((e % L) == L - 1 && fbo + fb > Cm) s_misc[3] = 1;
+        ws[lay.seg_off + sg] = fbo;
+        ws[lay.seg_len + sg] = fb;
+        ws[lay.alloc + (int64_t)e * R + h] = keep + fb;
+        if ((e % L) == L - 1 && fbo + fb > Cm) cap_err = 1;
     }
-    if (tid == 0) {
+    cap_err = __any_sync(0xffffffffu, cap_err);
+    if (lane == 0) {
         ws[lay.rep_ptr + N] = P;
         ws[lay.route_ptr + N] = 2 * N + P;
-    }
-    // segment tables [R][2L+B]: local, slot, fallback
-    const int SEG = 2 * L + B;
-    for (int idx = tid; idx < R * SEG; idx += kPlanThreads) {
-        const int r = idx / SEG, s = idx - r * SEG;
-        int off, len;
-        if (s < L) {
-            const int e = r * L + s;
-            off = ws[lay.home_off + e];
-            len = s_cnt[e] - s_sp[e];
-        } else if (s < L + B) {
-            off = ws[lay.slot_off + r * B + (s - L)];
-            len = ws[lay.slot_cnt + r * B + (s - L)];
-        } else {
-            const int e = r * L + (s - L - B);
-            off = C + (s_ce[e] - s_ce[r * L]);
-            len = s_x[e];
-        }
-        ws[lay.seg_off + idx] = off;
-        ws[lay.seg_len + idx] = len;
-    }
-    // allocation table: zero, then home (keep + fallback) and pieces
-    for (int64_t i = tid; i < (int64_t)N * R; i += kPlanThreads) ws[lay.alloc + i] = 0;
-    __syncthreads();
-    for (int e = tid; e < N; e += kPlanThreads)
-        ws[lay.alloc + (int64_t)e * R + e / L] = s_cnt[e] - s_sp[e] + s_x[e];
-    for (int gp = tid; gp < P; gp += kPlanThreads)
-        ws[lay.alloc + (int64_t)ws[lay.rep_expert + gp] * R + ws[lay.rep_recv + gp]] = ws[lay.rep_cnt + gp];
-    __syncthreads();
-    if (tid == 0) {
         const int fallback = total_spill - p_end;
         int st = 0;
-        if (s_misc[3]) st |= MOONEP_ST_CAPACITY;
+        if (cap_err) st |= MOONEP_ST_CAPACITY;
         if (fallback > 0) st |= MOONEP_ST_FALLBACK;
         ws[HDR_FALLBACK] = fallback;
         ws[HDR_NREP] = P;
@@ -350,6 +334,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[HDR_NRX] = nrx;
         ws[HDR_TOTAL_SPILL] = total_spill;
         ws[HDR_PEND] = p_end;
+        TRACE(ws, 7);
         __threadfence();
         if (st) atomicOr(ws + HDR_STATUS, st);
     }
@@ -362,18 +347,32 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     int32_t *ws = p.ws;
     const moonep_ws_layout_t &lay = p.lay;
 
-    // phase A: per-range histograms
+    if (blockIdx.x == 0) TRACE(ws, 0);
+    // phase A: per-range histograms; each thread issues up to kIdBatch id
+    // loads before its first shared-memory atomic, so the range costs about
+    // one memory latency instead of one per loop trip
     bool bad = false;
     for (int64_t q = blockIdx.x; q < p.Q; q += gridDim.x) {
         for (int e = tid; e < N; e += kPlanThreads) sm[e] = 0;
         __syncthreads();
         const int64_t i0 = range_begin(q, p.T, p.Q) * K, i1 = range_begin(q + 1, p.T, p.Q) * K;
-        for (int64_t i = i0 + tid; i < i1; i += kPlanThreads) {
-            const int e = __ldg(p.ids + i);
-            if ((unsigned)e < (unsigned)N)
-                atomicAdd(&sm[e], 1);
-            else
-                bad = true;
+        for (int64_t b0 = i0; b0 < i1; b0 += (int64_t)kIdBatch * kPlanThreads) {
+            int v[kIdBatch];
+#pragma unroll
+            for (int u = 0; u < kIdBatch; ++u) {
+                const int64_t i = b0 + tid + (int64_t)u * kPlanThreads;
+                v[u] = i < i1 ? __ldg(p.ids + i) : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < kIdBatch; ++u) {
+                const int64_t i = b0 + tid + (int64_t)u * kPlanThreads;
+                if (i < i1) {
+                    if ((unsigned)v[u] < (unsigned)N)
+                        atomicAdd(&sm[v[u]], 1);
+                    else
+                        bad = true;
+                }
+            }
         }
         __syncthreads();
         for (int e = tid; e < N; e += kPlanThreads) {
@@ -384,6 +383,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
         __syncthreads();
     }
     if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_EXPERT_ID);
+    if (blockIdx.x == 0) TRACE(ws, 1);
     if (blockIdx.x == 0 && tid < 8) ws[HDR_CFG + tid] = (&p.cfg.R)[tid];
     if (blockIdx.x == 0 && tid == 0) ws[HDR_NRANGES] = (int32_t)p.Q;
     __threadfence();
@@ -392,27 +392,32 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
         if (tid == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
         return;
     }
+    if (blockIdx.x == 0) TRACE(ws, 2);
     const int st = __ldcg(ws + HDR_STATUS);
     if (st & MOONEP_ST_ERROR_MASK) return;
 
-    // phase B: column prefixes on CTAs 1.. (or all on CTA 0 if alone)
+    // phase B: column prefixes on CTAs 1.. (or all on CTA 0 if alone); CTA 0
+    // loads cnt and clears alloc with all its threads, then warp 0 plans
     const int warp = tid >> 5;
-    if (gridDim.x == 1) {
+    if (gridDim.x == 1)
         for (int e = warp; e < N; e += kWarps) scan_column(ws + lay.base + (int64_t)e * p.Q, p.Q);
+    if (blockIdx.x == 0) {
+        for (int e = tid; e < N; e += kPlanThreads) sm[e] = __ldcg(ws + lay.cnt + e);
+        for (int64_t i = tid; i < (int64_t)N * p.cfg.R; i += kPlanThreads) ws[lay.alloc + i] = 0;
         __syncthreads();
-        plan_tables(p, sm);
-    } else if (blockIdx.x == 0) {
-        plan_tables(p, sm);
+        if (warp == 0) plan_tables(p, sm);
     } else {
         const int gw = (blockIdx.x - 1) * kWarps + warp;
         const int nw = (gridDim.x - 1) * kWarps;
         for (int e = gw; e < N; e += nw) scan_column(ws + lay.base + (int64_t)e * p.Q, p.Q);
+        __syncthreads();
+        if (blockIdx.x == 1) TRACE(ws, 8);
     }
 }
 
 }  // namespace
 
-size_t plan_smem_bytes(int N) { return (size_t)6 * (N > 0 ? N : 1) * sizeof(int); }
+size_t plan_smem_bytes(int N) { return (size_t)7 * (N > 0 ? N : 1) * sizeof(int); }
 
 const void *plan_kernel_ptr() { return (const void *)plan_kernel; }
 

@@ -90,6 +90,9 @@ WORKLOADS = {
                           headroom=0.25, maxvio=(4.0,)),
     "training": Workload("training", R=16, L=16, S=8192, K=8, H=7168, B=16, I=2048,
                          maxvio=(8.0,)),
+    # the mid shapes at a quarter of the tokens and an eighth of the FFN size:
+    # about 3 GB on the device, still far above L2, for profiler captures
+    "profile": Workload("profile", R=8, L=8, S=1024, K=8, H=7168, B=8, I=256, maxvio=(2.0,)),
 }
 
 

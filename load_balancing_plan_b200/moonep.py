@@ -16,7 +16,9 @@ import os
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoonep.so")
+# MOONEP_LIBRARY may point at another build of the same library (development
+# builds with different tuning constants); the default is the in-tree build.
+LIB_PATH = os.environ.get("MOONEP_LIBRARY") or os.path.join(_PKG, "libmoonep.so")
 
 OK, ERR_ARG, ERR_CUDA, ERR_DEVICE = 0, 1, 2, 3
 ST_EXPERT_ID, ST_CAPACITY, ST_TIMEOUT, ST_DEST, ST_CFG = 0x1, 0x2, 0x4, 0x8, 0x10
