@@ -254,37 +254,69 @@ class Runner:
         return total_ms, per, clk.summary()
 
     def e2e(self, steps, warmup):
-        """Same calls with the step's inputs copied from pinned host memory
-        and the output copied back, all inside the timed region."""
+        """The same calls with every step's router output and hidden states
+        copied in from pinned host memory and its combined output copied back
+        to pinned host memory, all inside the timed region.  Steps are
+        pipelined: two input and two output buffer sets, host-to-device copies
+        on one stream, device-to-host copies on another, the hot path on the
+        compute stream, ordered by events (a step's kernels wait for its
+        inputs; a buffer is refilled only after the step that used it)."""
         torch = self.torch
         p = self.prob
         T, K = self.prob.T, self.cfg["K"]
+        n = T * K
         ids_h = torch.from_numpy(self.route.topk_idx.reshape(-1).copy()).pin_memory()
         w_h = torch.from_numpy(self.route.topk_w.reshape(-1).copy()).pin_memory()
         x_h = p.x.cpu().pin_memory()
-        out_h = torch.empty_like(p.out, device="cpu").pin_memory()
-        s = self.stream
+        outs_h = [torch.empty_like(p.out, device="cpu").pin_memory() for _ in range(2)]
+        dev = p.x.device
+        ids_d = [p.ids, torch.empty_like(p.ids)]
+        w_d = [p.w, torch.empty_like(p.w)]
+        x_d = [p.x, torch.empty_like(p.x)]
+        out_d = [p.out, torch.empty_like(p.out)]
+        comp = self.stream
+        h2d = torch.cuda.Stream(device=dev)
+        d2h = torch.cuda.Stream(device=dev)
+        ev = lambda: torch.cuda.Event()
+        inputs_ready = [ev(), ev()]
+        inputs_free = [ev(), ev()]
+        out_ready = [ev(), ev()]
+        out_free = [ev(), ev()]
+        for e in inputs_free + out_free:
+            e.record(comp)
 
-        def one():
-            p.ids[:T * K].copy_(ids_h, non_blocking=True)
-            p.w[:T * K].copy_(w_h, non_blocking=True)
-            p.x.copy_(x_h, non_blocking=True)
-            self.step()
-            out_h.copy_(p.out, non_blocking=True)
+        def run(nsteps):
+            for i in range(nsteps):
+                b = i & 1
+                h2d.wait_event(inputs_free[b])
+                with torch.cuda.stream(h2d):
+                    ids_d[b][:n].copy_(ids_h, non_blocking=True)
+                    w_d[b][:n].copy_(w_h, non_blocking=True)
+                    x_d[b].copy_(x_h, non_blocking=True)
+                inputs_ready[b].record(h2d)
+                comp.wait_event(inputs_ready[b])
+                comp.wait_event(out_free[b])
+                p.ids, p.w, p.x, p.out = ids_d[b], w_d[b], x_d[b], out_d[b]
+                self.step()
+                inputs_free[b].record(comp)
+                out_ready[b].record(comp)
+                d2h.wait_event(out_ready[b])
+                with torch.cuda.stream(d2h):
+                    outs_h[b].copy_(out_d[b], non_blocking=True)
+                out_free[b].record(d2h)
 
-        for _ in range(warmup):
-            one()
+        run(warmup)
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(s)
-        for _ in range(steps):
-            one()
-        b.record(s)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(h2d)
+        run(steps)
+        z.record(d2h)
         torch.cuda.synchronize()
-        h2d = ids_h.numel() * 4 + w_h.numel() * 4 + x_h.numel() * 2
-        d2h = out_h.numel() * 2
-        return a.elapsed_time(b), h2d, d2h
+        p.ids, p.w, p.x, p.out = ids_d[0], w_d[0], x_d[0], out_d[0]
+        h2d_bytes = ids_h.numel() * 4 + w_h.numel() * 4 + x_h.numel() * 2
+        d2h_bytes = outs_h[0].numel() * 2
+        return a.elapsed_time(z), h2d_bytes, d2h_bytes
 
 
 def run_gpu(args):
@@ -316,8 +348,8 @@ def run_gpu(args):
     value = dc_bytes / (max_dc_ms * 1e-3) / 1e9
     ms_per_step = max_total_ms / args.steps
 
-    e2e_ms, h2d, d2h = run.e2e(max(3, args.steps // 4), 2)
-    e2e_steps = max(3, args.steps // 4)
+    e2e_steps = max(8, args.steps // 8)
+    e2e_ms, h2d, d2h = run.e2e(e2e_steps, 3)
     max_e2e_ms, e2e_bytes = reduce_over_ranks(e2e_ms, (ab["dispatch"] + ab["combine"]) * e2e_steps, world)
 
     peak, peak_kind = measured_peak()

@@ -279,7 +279,8 @@ int moonep_prefetch(const moonep_cfg_t *cfg, void *ws, const void *w_home, void 
     p.dst = (uint4 *)w_slot;
     p.ws = (int32_t *)ws;
     compute_layout(*cfg, p.lay);
-    cudaError_t e = launch_prefetch(p, d->sms * 8, (cudaStream_t)stream);
+    p.wait_limit = g_wait_limit.load();
+    cudaError_t e = launch_prefetch(p, d->sms, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "prefetch kernel launch");
     return MOONEP_OK;
 }
@@ -303,6 +304,7 @@ int moonep_reduce_grad(const moonep_cfg_t *cfg, void *ws, float *g_home, float *
     p.dst = (uint4 *)g_rep;
     p.ws = (int32_t *)ws;
     compute_layout(*cfg, p.lay);
+    p.wait_limit = g_wait_limit.load();
     cudaError_t e = launch_reduce_grad(p, d->sms * 8, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "reduce_grad kernel launch");
     return MOONEP_OK;

@@ -140,6 +140,7 @@ struct CombineParams {
 
 struct CopyParams {
     moonep_cfg_t cfg;
+    int64_t wait_limit;
     int64_t vecs;         // 16-byte vectors per expert
     const uint4 *src;
     uint4 *dst;

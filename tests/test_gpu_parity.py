@@ -434,3 +434,27 @@ def test_skew_sweep_plans(env, maxvio, seed):
     compare_plan(prob.read_plan(), opl)
     assert np.array_equal(prob.dest.cpu().numpy(), opl["dest"].reshape(-1))
     assert opl["fallback_rows"] == 0
+
+
+def test_reduce_grad_twice_after_one_plan(env):
+    # the work counter reduce_grad hands units out with resets itself: a second
+    # call after the same plan (new replica gradients) is exact again
+    torch, mp, harness = env
+    w = inputs.WORKLOADS["tiny"]
+    cfg = w.cfg()
+    r = inputs.routing(w.R, w.L, w.S, w.K, 2, alpha=1.0)
+    E = 128 * 256
+    prob = harness.Problem(cfg, g_elems=E)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.fill_weights(2)
+    prob.plan()
+    opl = oracle.plan(cfg, r.topk_idx)
+    for seed in (2, 3):
+        prob.fill_g_rep(seed)
+        gh = prob.g_home.cpu().numpy().copy()
+        gr = prob.g_rep.cpu().numpy().copy()
+        prob.reduce_grad()
+        torch.cuda.synchronize()
+        oracle.reduce_grad(cfg, opl, gh, gr, E)
+        assert np.array_equal(prob.g_home.cpu().numpy().view(np.uint32), gh.view(np.uint32))
+        assert np.array_equal(prob.g_rep.cpu().numpy().view(np.uint32), gr.view(np.uint32))
