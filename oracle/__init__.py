@@ -14,6 +14,8 @@ the C file):
   combine       -- out = bf16(fma chain over k of w * y[dest])
   prefetch      -- w_slot[r][b] = w_home[slot_expert[r][b]]
   reduce_grad   -- g_home[e] += replicas in receiver order; zero the replicas
+  combine_backward  -- grad_y[dest] = bf16(w * grad_out); grad_w = <grad_out, y[dest]> (fp64)
+  dispatch_backward -- grad_x[t] = bf16(fp32 sum over k of grad_recv[dest[t,k]])
 """
 from __future__ import annotations
 
@@ -77,6 +79,8 @@ def _load():
         lib.or_combine.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, ctypes.c_int64]
         lib.or_prefetch.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, ctypes.c_int64]
         lib.or_reduce_grad.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, ctypes.c_int64]
+        lib.or_combine_backward.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, vp, ctypes.c_int64]
+        lib.or_dispatch_backward.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, ctypes.c_int64]
         lib.or_f32_to_bf16_export.argtypes = [ctypes.c_float]
         lib.or_f32_to_bf16_export.restype = ctypes.c_uint16
         lib.or_bf16_to_f32_export.argtypes = [ctypes.c_uint16]
@@ -194,6 +198,34 @@ def reduce_grad(cfg: dict, pl: dict, g_home: np.ndarray, g_rep: np.ndarray, elem
     lib.or_reduce_grad(ctypes.byref(_cfg(cfg)), _ptr(rp), _ptr(rr), _ptr(rs), _ptr(g_home),
                        _ptr(g_rep), int(elems))
     return g_home, g_rep
+
+
+def combine_backward(cfg: dict, dest: np.ndarray, grad_out: np.ndarray, y: np.ndarray, w: np.ndarray,
+                     grad_y: np.ndarray, n_tokens=None, with_grad_w=True):
+    """grad_out: uint16 bf16 [n, H]; y, grad_y: uint16 [R*C_max, H] (grad_y
+    written in place at the dispatched rows).  Returns grad_w fp64 [n, K]."""
+    lib = _load()
+    T = int(cfg["R"]) * int(cfg["S"])
+    n = T if n_tokens is None else int(n_tokens)
+    K = int(cfg["K"])
+    gw = np.zeros((max(n, 1), K), np.float64)
+    lib.or_combine_backward(ctypes.byref(_cfg(cfg)), _ptr(np.ascontiguousarray(dest, dtype=np.int32)),
+                            _ptr(grad_out), _ptr(y), _ptr(np.ascontiguousarray(w, dtype=np.float32)),
+                            _ptr(grad_y), _ptr(gw) if with_grad_w else None, n)
+    return gw[:n]
+
+
+def dispatch_backward(cfg: dict, dest: np.ndarray, grad_recv: np.ndarray, n_tokens=None):
+    """Returns (grad_x uint16 bf16 [n, H], acc fp32 [n, H])."""
+    lib = _load()
+    T = int(cfg["R"]) * int(cfg["S"])
+    n = T if n_tokens is None else int(n_tokens)
+    H = int(cfg["H"])
+    gx = np.zeros((max(n, 1), H), np.uint16)
+    acc = np.zeros((max(n, 1), H), np.float32)
+    lib.or_dispatch_backward(ctypes.byref(_cfg(cfg)), _ptr(np.ascontiguousarray(dest, dtype=np.int32)),
+                             _ptr(grad_recv), _ptr(gx), _ptr(acc), n)
+    return gx[:n], acc[:n]
 
 
 def f32_to_bf16(f: float) -> int:

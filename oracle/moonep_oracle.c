@@ -461,3 +461,48 @@ void or_reduce_grad(const or_cfg *c, const int32_t *rep_ptr, const int32_t *rep_
 /* exported bf16 conversions, so tests can pin them against numpy/torch */
 uint16_t or_f32_to_bf16_export(float f) { return or_f32_to_bf16(f); }
 float or_bf16_to_f32_export(uint16_t u) { return or_bf16_to_f32(u); }
+
+/* ------------------------------------------------------------------------ */
+/* Backward of the data path (training; combine's and dispatch's adjoints).  */
+/* The forward steps are linear: combine gives out[t] = sum_k w[t,k] *       */
+/* y[dest[t,k]], dispatch gives recv[dest[t,k]] = x[t].  Their gradients:    */
+/*   combine backward:  grad_y[dest[t,k]] = w[t,k] * grad_out[t]             */
+/*                      grad_w[t,k]       = sum_h grad_out[t,h] * y[dest,h]  */
+/*   dispatch backward: grad_x[t]         = sum_k grad_recv[dest[t,k]]       */
+/* grad_y is one fp32 multiply rounded to bf16; grad_w is summed in fp64     */
+/* (its order is not part of any contract); grad_x accumulates fp32 adds in  */
+/* k order and rounds once to bf16, like combine.                            */
+/* ------------------------------------------------------------------------ */
+void or_combine_backward(const or_cfg *c, const int32_t *dest, const uint16_t *grad_out, const uint16_t *y,
+                         const float *w, uint16_t *grad_y, double *grad_w, int64_t n_tokens)
+{
+    const int64_t H = c->H;
+    for (int64_t t = 0; t < n_tokens; ++t)
+        for (int k = 0; k < c->K; ++k) {
+            int64_t d = dest[t * c->K + k];
+            float wk = w[t * c->K + k];
+            double dot = 0.0;
+            for (int64_t h = 0; h < H; ++h) {
+                float g = or_bf16_to_f32(grad_out[t * H + h]);
+                grad_y[d * H + h] = or_f32_to_bf16(wk * g);
+                if (grad_w) dot += (double)g * (double)or_bf16_to_f32(y[d * H + h]);
+            }
+            if (grad_w) grad_w[t * c->K + k] = dot;
+        }
+}
+
+void or_dispatch_backward(const or_cfg *c, const int32_t *dest, const uint16_t *grad_recv, uint16_t *grad_x,
+                          float *acc_out, int64_t n_tokens)
+{
+    const int64_t H = c->H;
+    for (int64_t t = 0; t < n_tokens; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int k = 0; k < c->K; ++k) {
+                int64_t d = dest[t * c->K + k];
+                acc = acc + or_bf16_to_f32(grad_recv[d * H + h]);
+            }
+            grad_x[t * H + h] = or_f32_to_bf16(acc);
+            if (acc_out) acc_out[t * H + h] = acc;
+        }
+}
