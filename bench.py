@@ -253,6 +253,36 @@ class Runner:
         per = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)] for j, n in enumerate(names)}
         return total_ms, per, clk.summary()
 
+    def backward(self, steps, warmup):
+        """The training backward pair on the same plan: combine_backward
+        (grad_y and grad_w) and dispatch_backward, each timed alone with CUDA
+        events; the output gradient is the hidden states and the expert
+        outputs are the dispatched rows (values do not change the work)."""
+        torch = self.torch
+        from load_balancing_plan_b200 import moonep as mp
+        p, cfg, s = self.prob, self.cfg, self.stream
+        T, K, H = p.T, cfg["K"], cfg["H"]
+        grad_y = torch.empty_like(p.recv)
+        grad_w = torch.empty(T * K, dtype=torch.float32, device=p.recv.device)
+        grad_x = torch.empty_like(p.out)
+        cb = lambda: mp.moonep_combine_backward(cfg, p.ws, p.x, p.recv, p.dest, p.w, grad_y, grad_w, s)
+        db = lambda: mp.moonep_dispatch_backward(cfg, p.ws, p.recv, p.dest, grad_x, s)
+        res = {}
+        for name, fn, nbytes in (("combine_backward", cb, T * 2 * H + 2 * T * K * 2 * H + 12 * T * K),
+                                 ("dispatch_backward", db, T * K * 2 * H + T * 2 * H + 4 * T * K)):
+            for _ in range(warmup):
+                fn()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            for _ in range(steps):
+                fn()
+            b.record(s)
+            torch.cuda.synchronize()
+            us = a.elapsed_time(b) / steps * 1e3
+            res[name] = {"us": round(us, 1), "gbs": round(nbytes / us / 1e3, 1), "algorithmic_bytes": nbytes}
+        return res
+
     def e2e(self, steps, warmup):
         """The same calls with every step's router output and hidden states
         copied in from pinned host memory and its combined output copied back
@@ -359,6 +389,8 @@ def run_gpu(args):
     kernel_gbs = {k: (ab[k] / (mean[k] * 1e-3) / 1e9 if mean[k] > 0 and ab[k] else None)
                   for k in ("dispatch", "combine", "prefetch", "reduce_grad")}
 
+    bwd = run.backward(max(10, args.steps // 10), args.warmup)
+
     sweep = None
     if not args.no_sweep and world == 1:
         sweep = run_sweep(args, peak)
@@ -401,6 +433,7 @@ def run_gpu(args):
         "gpu_launches": run.launches_per_step() * args.steps,
         "clocks": clocks,
     }
+    out["backward"] = bwd
     if sweep is not None:
         out["sweep"] = sweep
     if cpu is not None:

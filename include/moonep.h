@@ -20,6 +20,8 @@
  *                       receivers' prefetch slots
  *   moonep_reduce_grad  replica gradients added to the home experts'
  *                       gradients, used slots cleared
+ *   moonep_combine_backward, moonep_dispatch_backward
+ *                       the adjoints of combine and dispatch, for training
  *
  * Notation.  R ranks; L experts per rank; N = R*L experts; expert e lives on
  * home rank home(e) = e / L at local index e % L (the contiguous blocking of
@@ -186,6 +188,28 @@ MOONEP_API int moonep_dispatch(const moonep_cfg_t *cfg, void *ws, const void *x,
  * acc = fmaf(w[t][k], float(y[dest[t][k]]), acc) for k = 0..K-1. */
 MOONEP_API int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32_t *dest,
                    const float *topk_w, void *out, void *stream);
+
+/* Combine backward, for training ("The Busiest Rank Sets Your Step Time",
+ * flowchart: the backward pass of the layer follows its forward path; combine
+ * is linear in the expert outputs and in the router weights).  grad_out:
+ * device bf16 [R*S][H], the gradient of `out`; y, dest, topk_w: as given to
+ * moonep_combine; grad_y: device bf16 [R][C_max][H], written at every
+ * dispatched row: grad_y[dest[t][k]] = bf16_rne(fp32(w[t][k] *
+ * grad_out[t])); grad_w: device fp32 [R][S][K] or NULL: grad_w[t][k] = sum
+ * over h of grad_out[t][h] * y[dest[t][k]][h], accumulated in fp32 (the
+ * order is fixed, so results repeat exactly; it is not the plain left-to-right
+ * order).  y may be NULL when grad_w is NULL.  Rows outside the plan's
+ * segments are not written. */
+MOONEP_API int moonep_combine_backward(const moonep_cfg_t *cfg, void *ws, const void *grad_out, const void *y,
+                                       const int32_t *dest, const float *topk_w, void *grad_y, float *grad_w,
+                                       void *stream);
+
+/* Dispatch backward, for training: the adjoint of the row scatter.
+ * grad_recv: device bf16 [R][C_max][H], the gradient of the dispatched rows;
+ * grad_x: device bf16 [R*S][H]: grad_x[t] = bf16_rne(acc), acc = 0.0f then
+ * acc = acc + float(grad_recv[dest[t][k]]) for k = 0..K-1 (fp32). */
+MOONEP_API int moonep_dispatch_backward(const moonep_cfg_t *cfg, void *ws, const void *grad_recv,
+                                        const int32_t *dest, void *grad_x, void *stream);
 
 /* Prefetch (twodots.gr: weights of the duplicated experts are loaded into
  * the prefetch slots [E, E+B) before the experts run).  w_home: device bf16

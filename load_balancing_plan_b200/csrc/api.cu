@@ -37,6 +37,7 @@ struct DeviceInfo {
     int sms = 0;
     int plan_grid = 0;
     int combine_grid = 0;
+    int backward_grid = 0;
     size_t plan_smem = 0;
 };
 
@@ -61,6 +62,7 @@ int device_info(int N, DeviceInfo **out) {
         d.ok = (major == 10 && minor == 0 && coop != 0);
         d.ready = true;
         d.combine_grid = d.sms;  // one persistent combine CTA per SM
+        d.backward_grid = d.sms;  // one persistent combine_backward CTA per SM
     }
     if (!d.ok) return fail(MOONEP_ERR_DEVICE, "device %d is not an sm_100 GPU with cooperative launch", dev);
     // plan kernel: shared memory depends on N
@@ -225,15 +227,17 @@ int moonep_dispatch(const moonep_cfg_t *cfg, void *ws, const void *x, const int3
     return MOONEP_OK;
 }
 
-int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32_t *dest, const float *topk_w,
-                   void *out, void *stream) {
+// combine and dispatch backward share the TMA gather kernel; the backward
+// has no weights (each one is 1)
+static int combine_impl(const moonep_cfg_t *cfg, void *ws, const void *y, const int32_t *dest, const float *topk_w,
+                        void *out, void *stream, bool weighted) {
     TRY(check_cfg(cfg));
     const int64_t T = (int64_t)cfg->R * cfg->S;
     TRY(check_ptr(ws, 16, "ws", true));
-    TRY(check_ptr(y, 16, "y", T > 0));
+    TRY(check_ptr(y, 16, weighted ? "y" : "grad_recv", T > 0));
     TRY(check_ptr(dest, 4, "dest", T > 0));
-    TRY(check_ptr(topk_w, 4, "topk_w", T > 0));
-    TRY(check_ptr(out, 16, "out", T > 0));
+    TRY(check_ptr(topk_w, 4, "topk_w", weighted && T > 0));
+    TRY(check_ptr(out, 16, weighted ? "out" : "grad_x", T > 0));
     DeviceInfo *d = nullptr;
     TRY(device_info(cfg->R * cfg->L, &d));
     if (T == 0) return MOONEP_OK;
@@ -248,7 +252,7 @@ int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32
     p.rows_total = (int64_t)cfg->R * cfg->C_max;
     p.y = (const uint4 *)y;
     p.dest = dest;
-    p.w = topk_w;
+    p.w = weighted ? topk_w : nullptr;
     p.out = (uint4 *)out;
     p.ws = (int32_t *)ws;
     p.wait_limit = g_wait_limit.load();
@@ -257,6 +261,57 @@ int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32
     if (grid < 1) grid = 1;
     cudaError_t e = launch_combine(p, (int)grid, smem, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+    return MOONEP_OK;
+}
+
+int moonep_combine(const moonep_cfg_t *cfg, void *ws, const void *y, const int32_t *dest, const float *topk_w,
+                   void *out, void *stream) {
+    return combine_impl(cfg, ws, y, dest, topk_w, out, stream, true);
+}
+
+int moonep_dispatch_backward(const moonep_cfg_t *cfg, void *ws, const void *grad_recv, const int32_t *dest,
+                             void *grad_x, void *stream) {
+    return combine_impl(cfg, ws, grad_recv, dest, nullptr, grad_x, stream, false);
+}
+
+int moonep_combine_backward(const moonep_cfg_t *cfg, void *ws, const void *grad_out, const void *y,
+                            const int32_t *dest, const float *topk_w, void *grad_y, float *grad_w, void *stream) {
+    TRY(check_cfg(cfg));
+    const int64_t T = (int64_t)cfg->R * cfg->S;
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(grad_out, 16, "grad_out", T > 0));
+    TRY(check_ptr(dest, 4, "dest", T > 0));
+    TRY(check_ptr(topk_w, 4, "topk_w", T > 0));
+    TRY(check_ptr(grad_y, 16, "grad_y", T > 0));
+    if (grad_w) {
+        TRY(check_ptr(grad_w, 4, "grad_w", true));
+        TRY(check_ptr(y, 16, "y (needed for grad_w)", T > 0));
+    }
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (T == 0) return MOONEP_OK;
+    BackwardParams p{};
+    p.cfg = *cfg;
+    p.T = T;
+    p.hv = cfg->H / 8;
+    size_t smem = 0;
+    if (combine_backward_config(cfg->K, p.hv, grad_w != nullptr, &p.chunk_bytes, &p.upt, &p.stages, &smem) !=
+        cudaSuccess)
+        return fail(MOONEP_ERR_ARG, "combine_backward: no shared-memory configuration for K=%d H=%d", cfg->K, cfg->H);
+    p.rows_total = (int64_t)cfg->R * cfg->C_max;
+    p.wait_limit = g_wait_limit.load();
+    p.grad_out = (const uint4 *)grad_out;
+    p.y = (const uint4 *)y;
+    p.dest = dest;
+    p.w = topk_w;
+    p.grad_y = (uint4 *)grad_y;
+    p.grad_w = grad_w;
+    p.ws = (int32_t *)ws;
+    int64_t grid = d->backward_grid;
+    if (grid > T) grid = T;
+    if (grid < 1) grid = 1;
+    cudaError_t e = launch_combine_backward(p, (int)grid, smem, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "combine_backward kernel launch");
     return MOONEP_OK;
 }
 

@@ -1,0 +1,272 @@
+// backward.cu -- moonep_combine_backward: the backward of the combine step
+// for training ("The Busiest Rank Sets Your Step Time: Running MoonEP's
+// Planning Code Ourselves", flowchart: in training the backward pass follows
+// the layer's data path; combine is linear in the expert outputs and in the
+// router weights, so its backward is a weighted dispatch of the output
+// gradient plus one inner product per (token, k)):
+//
+//   grad_y[dest[t][k]] = bf16_rne(fp32(w[t][k] * grad_out[t]))
+//   grad_w[t][k]       = sum_h grad_out[t][h] * y[dest[t][k]][h]   (fp32)
+//
+// HBM-bound: one read of grad_out per token, K row writes and, for grad_w,
+// K row reads.  One persistent CTA per SM owns a contiguous run of whole
+// tokens.  Warp 0 produces: per unit (one chunk of one token's row) it bulk
+// copies the grad_out chunk and, for grad_w, the K matching chunks of y into
+// a shared-memory stage (TMA, "full" mbarrier).  Warps 1..8 consume: each
+// thread takes 16-byte vectors of the chunk, stores the K scaled vectors to
+// the dispatched rows and adds the products into its own per-k partial sums
+// in shared memory.  After a token's last chunk the consumers reduce the
+// partial sums (warp butterflies, then the 8 warps in order), so grad_w does
+// not depend on timing.  Every wait is bounded; no multicast.
+#include <cuda_bf16.h>
+
+#include "moonep_internal.cuh"
+
+namespace moonep {
+
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = 32 * kConsumerWarps;
+constexpr int kThreads = 32 + kConsumers;
+constexpr int kMaxStages = 8;
+constexpr int kMaxK = 64;
+
+struct StageInfo {
+    int64_t t;       // token
+    int32_t c;       // chunk of the row
+    uint32_t bytes;  // bytes of this chunk
+    int32_t valid;   // all K destinations in range
+    int32_t pad;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __grid_constant__ BackwardParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    int32_t *ws = p.ws;
+    if (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
+    if (!cfg_matches(ws, p.cfg, num_ranges(p.T))) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
+        return;
+    }
+    const int K = p.cfg.K;
+    const bool want_w = p.grad_w != nullptr;
+    const int NS = p.stages;
+    const uint32_t CH = p.chunk_bytes;
+    const int rows_per_stage = 1 + (want_w ? K : 0);
+    const size_t stage_bytes = (size_t)rows_per_stage * CH;
+    uint8_t *stages = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)NS * stage_bytes);
+    uint64_t *empty = full + kMaxStages;
+    StageInfo *info = reinterpret_cast<StageInfo *>(empty + kMaxStages);
+    float *sw = reinterpret_cast<float *>(info + kMaxStages);        // [kMaxStages][kMaxK] weights
+    int32_t *sd = reinterpret_cast<int32_t *>(sw + kMaxStages * kMaxK);  // [kMaxStages][kMaxK] dests
+    float *s_red = reinterpret_cast<float *>(sd + kMaxStages * kMaxK);   // [kMaxK][kConsumerWarps]
+    float *s_part = s_red + kMaxK * kConsumerWarps;                       // [K][kConsumers]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (want_w)
+        for (int i = threadIdx.x; i < K * kConsumers; i += kThreads) s_part[i] = 0.f;
+    __syncthreads();
+
+    const int64_t tb = (int64_t)blockIdx.x * p.T / gridDim.x;
+    const int64_t te = (int64_t)(blockIdx.x + 1) * p.T / gridDim.x;
+    const int64_t u0 = tb * p.upt, u1 = te * p.upt;
+    const int64_t row_bytes = (int64_t)p.hv * 16;
+    const uint32_t last = (uint32_t)(row_bytes - (int64_t)(p.upt - 1) * CH);
+    const uint64_t pol = policy_evict_first();
+    const uint8_t *gsrc = reinterpret_cast<const uint8_t *>(p.grad_out);
+    const uint8_t *ysrc = reinterpret_cast<const uint8_t *>(p.y);
+
+    if (warp == 0) {
+        // ------------------------------------------------------- producer
+        int64_t cur = -1;
+        int dk = 0, dk2 = 0;
+        float wk = 0.f, wk2 = 0.f;
+        int valid = 1;
+        bool bad = false, fail = false;
+        int64_t i = 0;
+        for (int64_t u = u0; u < u1; ++u, ++i) {
+            const int s = (int)(i % NS);
+            if (i >= NS) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait_bounded(&empty[s], (uint32_t)(((i / NS) - 1) & 1), p.wait_limit);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    fail = true;
+                    break;
+                }
+            }
+            const int64_t t = u / p.upt;
+            const int c = (int)(u - t * p.upt);
+            if (t != cur) {
+                cur = t;
+                dk = lane < K ? __ldg(p.dest + t * K + lane) : 0;
+                wk = lane < K ? __ldg(p.w + t * K + lane) : 0.f;
+                dk2 = lane + 32 < K ? __ldg(p.dest + t * K + lane + 32) : 0;
+                wk2 = lane + 32 < K ? __ldg(p.w + t * K + lane + 32) : 0.f;
+                const bool okl = dk >= 0 && (int64_t)dk < p.rows_total && dk2 >= 0 && (int64_t)dk2 < p.rows_total;
+                valid = __all_sync(0xffffffffu, okl) ? 1 : 0;
+                bad |= !valid;
+            }
+            const uint32_t bytes = c == p.upt - 1 ? last : CH;
+            if (lane < K) {
+                sw[s * kMaxK + lane] = wk;
+                sd[s * kMaxK + lane] = dk;
+            }
+            if (lane + 32 < K) {
+                sw[s * kMaxK + lane + 32] = wk2;
+                sd[s * kMaxK + lane + 32] = dk2;
+            }
+            __syncwarp();  // every lane's weights and rows before lane 0's release
+            if (lane == 0) {
+                info[s].t = t;
+                info[s].c = c;
+                info[s].bytes = bytes;
+                info[s].valid = valid;
+                mbar_arrive_expect_tx(&full[s], valid ? (uint32_t)rows_per_stage * bytes : 0u);
+            }
+            __syncwarp();
+            if (valid) {
+                uint8_t *st = stages + (size_t)s * stage_bytes;
+                if (lane == 0) bulk_g2s(st, gsrc + t * row_bytes + (int64_t)c * CH, bytes, &full[s], pol);
+                if (want_w) {
+                    if (lane < K)
+                        bulk_g2s(st + (size_t)(1 + lane) * CH, ysrc + (int64_t)dk * row_bytes + (int64_t)c * CH,
+                                 bytes, &full[s], pol);
+                    if (lane + 32 < K)
+                        bulk_g2s(st + (size_t)(33 + lane) * CH, ysrc + (int64_t)dk2 * row_bytes + (int64_t)c * CH,
+                                 bytes, &full[s], pol);
+                }
+            }
+        }
+        if (lane == 0) {
+            const int64_t drain = p.wait_limit > (int64_t(1) << 20) ? p.wait_limit : (int64_t(1) << 20);
+            for (int64_t j = (i > NS ? i - NS : 0); j < i; ++j)
+                mbar_wait_bounded(&full[j % NS], (uint32_t)((j / NS) & 1), drain);
+            if (fail) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
+            if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_DEST);
+        }
+    } else {
+        // ------------------------------------------------------- consumers
+        const int ct = threadIdx.x - 32;
+        const int cw = ct >> 5;
+        int64_t i = 0;
+        bool ok = true;
+        for (int64_t u = u0; u < u1; ++u, ++i) {
+            const int s = (int)(i % NS);
+            if (ok && !mbar_wait_bounded(&full[s], (uint32_t)((i / NS) & 1), p.wait_limit)) {
+                if (ct == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
+                ok = false;  // keep joining the token-end barriers, touch nothing
+            }
+            const StageInfo inf = info[s];
+            if (ok && inf.valid) {
+                const uint8_t *st = stages + (size_t)s * stage_bytes;
+                const float *wv = sw + s * kMaxK;
+                const int32_t *dv = sd + s * kMaxK;
+                const int nv = (int)(inf.bytes >> 4);
+                const int64_t col = (int64_t)inf.c * (CH >> 4);
+                for (int v = ct; v < nv; v += kConsumers) {
+                    const uint4 gv = *reinterpret_cast<const uint4 *>(st + (size_t)v * 16);
+                    const __nv_bfloat162 *gh = reinterpret_cast<const __nv_bfloat162 *>(&gv);
+                    float gf[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 f = __bfloat1622float2(gh[q]);
+                        gf[2 * q] = f.x;
+                        gf[2 * q + 1] = f.y;
+                    }
+                    for (int k = 0; k < K; ++k) {
+                        const float w = wv[k];
+                        uint4 o;
+                        __nv_bfloat162 *oh = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            oh[q] = __floats2bfloat162_rn(__fmul_rn(w, gf[2 * q]), __fmul_rn(w, gf[2 * q + 1]));
+                        __stcs(p.grad_y + (int64_t)dv[k] * p.hv + col + v, o);
+                        if (want_w) {
+                            const uint4 yv = *reinterpret_cast<const uint4 *>(st + (size_t)(1 + k) * CH + (size_t)v * 16);
+                            const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&yv);
+                            float a = s_part[k * kConsumers + ct];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float2 f = __bfloat1622float2(yh[q]);
+                                a = __fmaf_rn(gf[2 * q], f.x, a);
+                                a = __fmaf_rn(gf[2 * q + 1], f.y, a);
+                            }
+                            s_part[k * kConsumers + ct] = a;
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            // the decision depends on u only, so all consumers join the same barriers
+            const int64_t tu = u / p.upt;
+            if (want_w && u - tu * p.upt == p.upt - 1) {
+                // the token's last chunk: reduce the partial sums in a fixed order
+                named_barrier(1, kConsumers);
+                for (int k = 0; k < K; ++k) {
+                    float a = s_part[k * kConsumers + ct];
+                    s_part[k * kConsumers + ct] = 0.f;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
+                    if (lane == 0) s_red[k * kConsumerWarps + cw] = a;
+                }
+                named_barrier(1, kConsumers);
+                if (ok && inf.valid && ct < K) {
+                    float a = 0.f;
+                    for (int q = 0; q < kConsumerWarps; ++q) a = __fadd_rn(a, s_red[ct * kConsumerWarps + q]);
+                    p.grad_w[tu * K + ct] = a;
+                }
+            }
+        }
+    }
+}
+
+}  // namespace
+
+// chunk: the row split into the fewest equal pieces (multiples of 16 bytes,
+// at most 32 KB) such that three stages of (1 + K) pieces fit in shared
+// memory beside the fixed tables; large bulk copies move the most bytes
+cudaError_t combine_backward_config(int K, int hv, bool with_grad_w, uint32_t *chunk, int *upt, int *stages,
+                                    size_t *smem) {
+    if (K < 1 || K > kMaxK || hv < 1) return cudaErrorInvalidValue;
+    const size_t rows = 1 + (with_grad_w ? (size_t)K : 0);
+    const size_t fixed = 2 * kMaxStages * 8 + kMaxStages * sizeof(StageInfo) + 2 * kMaxStages * kMaxK * 4 +
+                         kMaxK * kConsumerWarps * 4 + (with_grad_w ? (size_t)K * kConsumers * 4 : 0) + 128;
+    const size_t budget = 220 * 1024;
+    if (fixed + rows * 16 * 3 > budget) return cudaErrorInvalidValue;
+    const uint32_t row = (uint32_t)hv * 16;
+    uint32_t ch = row;
+    for (int n = 1;; ++n) {
+        ch = (((row + n - 1) / n) + 15) & ~15u;
+        if (ch <= 32768 && rows * ch * 3 <= budget - fixed) break;
+        if (ch <= 16) return cudaErrorInvalidValue;
+    }
+    const size_t stage = rows * ch;
+    int ns = (int)((budget - fixed) / stage);
+    if (ns > kMaxStages) ns = kMaxStages;
+    if (ns < 2) return cudaErrorInvalidValue;
+    *chunk = ch;
+    *upt = (int)((row + ch - 1) / ch);
+    *stages = ns;
+    *smem = (size_t)ns * stage + fixed;
+    return cudaSuccess;
+}
+
+cudaError_t launch_combine_backward(const BackwardParams &p, int grid, size_t smem, cudaStream_t s) {
+    cudaError_t err =
+        cudaFuncSetAttribute(combine_backward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    combine_backward_kernel<<<grid, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace moonep

@@ -5,7 +5,8 @@
 // "How it works": fused unpermute).
 //
 // out[t] = bf16_rne(acc), acc = 0.0f, acc = fmaf(w[t][k], float(y[dest[t][k]]),
-// acc) for k = 0..K-1 in that order.
+// acc) for k = 0..K-1 in that order.  The same kernel with no weights is the
+// dispatch backward: grad_x[t] = bf16_rne(fp32 sum over k of grad_recv[dest]).
 //
 // HBM-bound: K row reads and one row write per token.  One persistent CTA
 // per SM runs a TMA pipeline.  A unit of work is one chunk of one token's
@@ -68,18 +69,6 @@ __device__ __forceinline__ uint4 pack8(const float *acc) {
     return v;
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// bounded wait; returns false if it gave up
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int64_t limit) {
-    int64_t n = 0;
-    while (!mbar_try_wait(bar, parity))
-        if (++n > limit) return false;
-    return true;
-}
-
 __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_constant__ CombineParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     int32_t *ws = p.ws;
@@ -138,10 +127,12 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
             const int c = (int)(u - t * p.upt);
             if (t != cur) {
                 cur = t;
+                // no weights (dispatch backward): every weight is 1, and
+                // fmaf(1, v, acc) is exactly the fp32 sum acc + v
                 dk = lane < K ? __ldg(p.dest + t * K + lane) : 0;
-                wk = lane < K ? __ldg(p.w + t * K + lane) : 0.f;
+                wk = lane < K ? (p.w ? __ldg(p.w + t * K + lane) : 1.f) : 0.f;
                 dk2 = lane + 32 < K ? __ldg(p.dest + t * K + lane + 32) : 0;
-                wk2 = lane + 32 < K ? __ldg(p.w + t * K + lane + 32) : 0.f;
+                wk2 = lane + 32 < K ? (p.w ? __ldg(p.w + t * K + lane + 32) : 1.f) : 0.f;
                 const bool okl = dk >= 0 && (int64_t)dk < p.rows_total && dk2 >= 0 && (int64_t)dk2 < p.rows_total;
                 valid = __all_sync(0xffffffffu, okl) ? 1 : 0;
                 bad |= !valid;
@@ -149,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
             const uint32_t bytes = c == p.upt - 1 ? last : CH;
             if (lane < K) sw[s * kMaxK + lane] = wk;
             if (lane + 32 < K) sw[s * kMaxK + lane + 32] = wk2;
+            __syncwarp();  // every lane's weights before lane 0's release
             if (lane == 0) {
                 info[s].t = t;
                 info[s].c = c;

@@ -138,6 +138,24 @@ struct CombineParams {
     int64_t wait_limit;
 };
 
+struct BackwardParams {
+    moonep_cfg_t cfg;
+    int64_t T;
+    int32_t hv;           // 16-byte vectors per row (H / 8)
+    int32_t upt;          // row chunks per token
+    uint32_t chunk_bytes; // bytes per row chunk (the last may be shorter)
+    int32_t stages;       // shared-memory stages
+    int64_t rows_total;   // R * C_max
+    int64_t wait_limit;
+    const uint4 *grad_out;
+    const uint4 *y;       // may be NULL when grad_w is NULL
+    const int32_t *dest;
+    const float *w;
+    uint4 *grad_y;
+    float *grad_w;        // may be NULL
+    int32_t *ws;
+};
+
 struct CopyParams {
     moonep_cfg_t cfg;
     int64_t wait_limit;
@@ -198,6 +216,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// bounded mbarrier wait; returns false if it gave up after `limit` polls
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int64_t limit) {
+    int64_t n = 0;
+    while (!mbar_try_wait(bar, parity))
+        if (++n > limit) return false;
+    return true;
+}
+
+// barrier over the `count` threads of named barrier `id` (id 0 is __syncthreads)
+__device__ __forceinline__ void named_barrier(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
@@ -277,4 +312,7 @@ const void *combine_kernel_ptr();
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s);
 cudaError_t launch_reduce_grad(const CopyParams &p, int grid, cudaStream_t s);
 int set_error(int code, const char *msg);
+cudaError_t launch_combine_backward(const BackwardParams &p, int grid, size_t smem, cudaStream_t s);
+cudaError_t combine_backward_config(int K, int hv, bool with_grad_w, uint32_t *chunk, int *upt, int *stages,
+                                    size_t *smem);
 }  // namespace moonep

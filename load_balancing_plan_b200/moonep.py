@@ -73,6 +73,8 @@ _sig = {
     "moonep_reduce_grad": ([_CP, _vp, _vp, _vp, _i64, _vp], ctypes.c_int),
     "moonep_plan_read": ([_CP, _vp, ctypes.POINTER(PlanInfo), _vp, _vp], ctypes.c_int),
     "moonep_plan_noalloc": ([_CP, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_combine_backward": ([_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_dispatch_backward": ([_CP, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_set_wait_limit": ([_i64], ctypes.c_int),
     "moonep_num_ranges": ([_i64], _i64),
     "moonep_last_error": ([], ctypes.c_char_p),
@@ -175,6 +177,16 @@ def moonep_dispatch(cfg, ws, x, topk_idx, recv, dest, stream=None) -> None:
 def moonep_combine(cfg, ws, y, dest, topk_w, out, stream=None) -> None:
     _check(_lib.moonep_combine(ctypes.byref(cfg_of(cfg)), _p(ws), _p(y), _p(dest), _p(topk_w),
                                _p(out), _stream(stream)))
+
+
+def moonep_combine_backward(cfg, ws, grad_out, y, dest, topk_w, grad_y, grad_w=None, stream=None) -> None:
+    _check(_lib.moonep_combine_backward(ctypes.byref(cfg_of(cfg)), _p(ws), _p(grad_out), _p(y), _p(dest),
+                                        _p(topk_w), _p(grad_y), _p(grad_w), _stream(stream)))
+
+
+def moonep_dispatch_backward(cfg, ws, grad_recv, dest, grad_x, stream=None) -> None:
+    _check(_lib.moonep_dispatch_backward(ctypes.byref(cfg_of(cfg)), _p(ws), _p(grad_recv), _p(dest),
+                                         _p(grad_x), _stream(stream)))
 
 
 def moonep_prefetch(cfg, ws, w_home, w_slot, elems_per_expert, stream=None) -> None:
