@@ -53,7 +53,7 @@ _PLAN_FIELDS = ["cnt", "keep", "spill", "home_off", "fb_cnt", "fb_off",
                 "load", "deficit", "fill", "slots_used",
                 "slot_expert", "slot_cnt", "slot_off", "slot_first_j",
                 "rep_ptr", "rep_expert", "rep_recv", "rep_slot", "rep_first_j", "rep_cnt",
-                "seg_off", "seg_len", "alloc", "dest"]
+                "rep_off", "recv_ptr", "seg_off", "seg_len", "alloc", "dest"]
 
 
 class _Plan(ctypes.Structure):
@@ -70,12 +70,13 @@ def _load():
     if _lib is None:
         lib = ctypes.CDLL(build())
         vp = ctypes.c_void_p
-        lib.or_plan.argtypes = [ctypes.POINTER(_Cfg), vp, ctypes.POINTER(_Plan)]
-        lib.or_plan.restype = ctypes.c_int
-        lib.or_plan_unitwise.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, vp, vp]
-        lib.or_plan_unitwise.restype = ctypes.c_int
+        lib.or_plan_ex.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, vp, ctypes.POINTER(_Plan)]
+        lib.or_plan_ex.restype = ctypes.c_int
+        lib.or_plan_unitwise_ex.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, vp, vp, vp, vp, vp, vp, vp]
+        lib.or_plan_unitwise_ex.restype = ctypes.c_int
         lib.or_dispatch.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, ctypes.c_int64]
-        lib.or_expert_scale.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, vp]
+        lib.or_expert_scale.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, vp, ctypes.c_int,
+                                        vp, vp, vp, vp, vp]
         lib.or_combine.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, ctypes.c_int64]
         lib.or_prefetch.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, ctypes.c_int64]
         lib.or_reduce_grad.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, ctypes.c_int64]
@@ -98,28 +99,33 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
-def plan(cfg: dict, topk_idx: np.ndarray) -> dict:
+MODE_HEADROOM, MODE_REMOTE = 0, 1
+
+
+def plan(cfg: dict, topk_idx: np.ndarray, mode: int = MODE_HEADROOM) -> dict:
     """Run the plan on int32 topk_idx [R, S, K]; returns every table plus the
-    header counts as a dict of numpy arrays / ints."""
+    header counts as a dict of numpy arrays / ints.  mode 1: remote weights
+    (pieces beyond a receiver's B slots read their expert remotely)."""
     lib = _load()
     R, L, S, K, B = (int(cfg[n]) for n in "RLSKB")
     N = R * L
+    P = N + R
     ids = np.ascontiguousarray(topk_idx, dtype=np.int32).reshape(-1)
     assert ids.size == R * S * K
     sizes = dict(cnt=N, keep=N, spill=N, home_off=N, fb_cnt=N, fb_off=N,
                  load=R, deficit=R, fill=R, slots_used=R,
                  slot_expert=R * B, slot_cnt=R * B, slot_off=R * B, slot_first_j=R * B,
-                 rep_ptr=N + 1, rep_expert=R * B, rep_recv=R * B, rep_slot=R * B,
-                 rep_first_j=R * B, rep_cnt=R * B,
+                 rep_ptr=N + 1, rep_expert=P, rep_recv=P, rep_slot=P, rep_first_j=P, rep_cnt=P,
+                 rep_off=P, recv_ptr=R + 1,
                  seg_off=R * (2 * L + B), seg_len=R * (2 * L + B), alloc=N * R,
                  dest=R * S * K)
     arrs = {k: np.zeros(max(v, 1), np.int32) for k, v in sizes.items()}
     p = _Plan(0, 0, 0, 0, *(arrs[k].ctypes.data_as(_P) for k in _PLAN_FIELDS))
     c = _cfg(cfg)
-    lib.or_plan(ctypes.byref(c), _ptr(ids), ctypes.byref(p))
+    lib.or_plan_ex(ctypes.byref(c), int(mode), _ptr(ids), ctypes.byref(p))
     out = {k: arrs[k][:sizes[k]] for k in _PLAN_FIELDS}
     npc = p.n_replicas
-    for k in ("rep_expert", "rep_recv", "rep_slot", "rep_first_j", "rep_cnt"):
+    for k in ("rep_expert", "rep_recv", "rep_slot", "rep_first_j", "rep_cnt", "rep_off"):
         out[k] = out[k][:npc]
     out["alloc"] = out["alloc"].reshape(N, R)
     out["dest"] = out["dest"].reshape(R, S, K)
@@ -128,7 +134,7 @@ def plan(cfg: dict, topk_idx: np.ndarray) -> dict:
     return out
 
 
-def plan_unitwise(cfg: dict, topk_idx: np.ndarray) -> dict:
+def plan_unitwise(cfg: dict, topk_idx: np.ndarray, mode: int = MODE_HEADROOM) -> dict:
     lib = _load()
     R, L, S, K, B = (int(cfg[n]) for n in "RLSKB")
     N = R * L
@@ -139,8 +145,8 @@ def plan_unitwise(cfg: dict, topk_idx: np.ndarray) -> dict:
     fb = np.zeros(max(N, 1), np.int32)
     dest = np.zeros(max(ids.size, 1), np.int32)
     st = np.zeros(1, np.int32)
-    lib.or_plan_unitwise(ctypes.byref(_cfg(cfg)), _ptr(ids), _ptr(alloc), _ptr(se), _ptr(sc),
-                         _ptr(fb), _ptr(dest), _ptr(st))
+    lib.or_plan_unitwise_ex(ctypes.byref(_cfg(cfg)), int(mode), _ptr(ids), _ptr(alloc), _ptr(se),
+                            _ptr(sc), _ptr(fb), _ptr(dest), _ptr(st))
     return dict(alloc=alloc[:N * R].reshape(N, R), slot_expert=se[:R * B], slot_cnt=sc[:R * B],
                 fb_cnt=fb[:N], dest=dest[:ids.size].reshape(R, S, K), status=int(st[0]))
 
@@ -158,10 +164,14 @@ def dispatch(cfg: dict, dest: np.ndarray, x: np.ndarray, recv: np.ndarray, n_tok
 
 def expert_scale(cfg: dict, pl: dict, recv: np.ndarray, scale: np.ndarray, y: np.ndarray):
     lib = _load()
+    n = int(pl["n_replicas"])
+    reps = [np.ascontiguousarray(pl[k][:n], dtype=np.int32) if n else np.zeros(1, np.int32)
+            for k in ("rep_expert", "rep_recv", "rep_slot", "rep_off", "rep_cnt")]
     lib.or_expert_scale(ctypes.byref(_cfg(cfg)), _ptr(np.ascontiguousarray(pl["seg_off"])),
                         _ptr(np.ascontiguousarray(pl["seg_len"])),
                         _ptr(np.ascontiguousarray(pl["slot_expert"])), _ptr(recv),
-                        _ptr(np.ascontiguousarray(scale, dtype=np.float32)), _ptr(y))
+                        _ptr(np.ascontiguousarray(scale, dtype=np.float32)), _ptr(y), n,
+                        *(_ptr(a) for a in reps))
     return y
 
 

@@ -55,7 +55,9 @@ typedef struct {
     int32_t *load, *deficit, *fill, *slots_used;               /* [R]          */
     int32_t *slot_expert, *slot_cnt, *slot_off, *slot_first_j; /* [R*B]        */
     int32_t *rep_ptr;                                          /* [N+1]        */
-    int32_t *rep_expert, *rep_recv, *rep_slot, *rep_first_j, *rep_cnt; /* [R*B] */
+    int32_t *rep_expert, *rep_recv, *rep_slot, *rep_first_j, *rep_cnt; /* [N+R] */
+    int32_t *rep_off;                                          /* [N+R] row on the receiver */
+    int32_t *recv_ptr;                                         /* [R+1] pieces by receiver */
     int32_t *seg_off, *seg_len;                                /* [R*(2L+B)]   */
     int32_t *alloc;                                            /* [N*R]        */
     int32_t *dest;                                             /* [R*S*K]      */
@@ -66,7 +68,15 @@ static int64_t or_min64(int64_t a, int64_t b) { return a < b ? a : b; }
 /* ------------------------------------------------------------------------ */
 /* Plan: O1 validate, O2 histogram, O3 keep, O4 spill, O5 layout, O6 dest.  */
 /* ------------------------------------------------------------------------ */
-int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
+/* mode 0: the library's headroom rule (above).  mode 1, remote weights (the
+ * pages' inference fallback: when a rank would need more replicas than it has
+ * prefetch slots, the group GEMM reads the weights from the home rank,
+ * twodots.gr "MoonEP balances AI experts in MoE models", memory-contract
+ * paragraphs; "The Busiest Rank Sets Your Step Time", "Installation and
+ * integration"): a receiver takes spilled rows while it has room whatever its
+ * slots; its first B pieces get slots, later ones are remote (slot -1), so no
+ * row ever falls back and every rank holds exactly C rows. */
+int or_plan_ex(const or_cfg *c, int mode, const int32_t *topk_idx, or_plan_t *p)
 {
     const int R = c->R, L = c->L, B = c->B;
     const int N = R * L;
@@ -125,6 +135,7 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
         p->slot_first_j[i] = 0;
     }
     int npieces = 0;
+    int32_t *on_r = (int32_t *)calloc((size_t)(R > 0 ? R : 1), sizeof(int32_t)); /* pieces per receiver */
     for (int e = 0; e < N; ++e) {
         p->rep_ptr[e] = npieces;
         int64_t a = p->spill[e];
@@ -132,21 +143,25 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
         while (a > 0) {
             int r = -1;
             for (int q = 0; q < R; ++q)
-                if (def[q] > 0 && p->slots_used[q] < B) {
+                if (def[q] > 0 && (mode == 1 || p->slots_used[q] < B)) {
                     r = q;
                     break;
                 }
             if (r < 0) break;
             int64_t t = or_min64(a, def[r]);
-            int b = p->slots_used[r]++;
+            int b = on_r[r] < B ? on_r[r] : -1;   /* mode 0 always has a free slot here */
+            on_r[r]++;
+            if (b >= 0) p->slots_used[r]++;
             p->rep_expert[npieces] = e;
             p->rep_recv[npieces] = r;
             p->rep_slot[npieces] = b;
             p->rep_first_j[npieces] = (int32_t)(p->keep[e] + spilled);
             p->rep_cnt[npieces] = (int32_t)t;
-            p->slot_expert[r * B + b] = e;
-            p->slot_cnt[r * B + b] = (int32_t)t;
-            p->slot_first_j[r * B + b] = (int32_t)(p->keep[e] + spilled);
+            if (b >= 0) {
+                p->slot_expert[r * B + b] = e;
+                p->slot_cnt[r * B + b] = (int32_t)t;
+                p->slot_first_j[r * B + b] = (int32_t)(p->keep[e] + spilled);
+            }
             ++npieces;
             def[r] -= (int32_t)t;
             a -= t;
@@ -159,6 +174,7 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
     p->rep_ptr[N] = npieces;
     p->n_replicas = npieces;
     free(def);
+    free(on_r);
 
     /* O5: layout of rank r: kept local segments, then slots in slot order,
      * then (from row C) the fallback segments of r's own experts. */
@@ -176,6 +192,12 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
             p->seg_len[r * SEG + L + b] = p->slot_cnt[r * B + b];
             off += p->slot_cnt[r * B + b];
         }
+        /* remote pieces (mode 1) follow the slots, in piece order */
+        for (int q = 0; q < npieces; ++q)
+            if (p->rep_recv[q] == r && p->rep_slot[q] < 0) {
+                p->rep_off[q] = (int32_t)off;
+                off += p->rep_cnt[q];
+            }
         p->fill[r] = (int32_t)off;
         int64_t fo = C;
         for (int loc = 0; loc < L; ++loc) {
@@ -187,6 +209,14 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
         }
         if (fo > c->C_max) p->status |= OR_ST_CAPACITY;
     }
+    for (int q = 0; q < npieces; ++q)
+        if (p->rep_slot[q] >= 0) p->rep_off[q] = p->slot_off[p->rep_recv[q] * B + p->rep_slot[q]];
+    /* pieces grouped by receiver; pieces are created in receiver order within
+     * an expert, and receivers are filled in ascending order, so counting is
+     * enough (checked by the tests) */
+    for (int r = 0; r <= R; ++r) p->recv_ptr[r] = 0;
+    for (int q = 0; q < npieces; ++q) p->recv_ptr[p->rep_recv[q] + 1]++;
+    for (int r = 0; r < R; ++r) p->recv_ptr[r + 1] += p->recv_ptr[r];
     if (p->fallback_rows > 0) p->status |= OR_ST_FALLBACK;
     if (p->status & OR_ST_CAPACITY) return p->status;
 
@@ -215,7 +245,7 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
             for (int q = p->rep_ptr[e]; q < p->rep_ptr[e + 1]; ++q)
                 if (j >= p->rep_first_j[q] && j < p->rep_first_j[q] + p->rep_cnt[q]) {
                     rank = p->rep_recv[q];
-                    row = p->slot_off[p->rep_recv[q] * B + p->rep_slot[q]] + (j - p->rep_first_j[q]);
+                    row = p->rep_off[q] + (j - p->rep_first_j[q]);
                     break;
                 }
             if (rank < 0) {
@@ -230,6 +260,8 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
     return p->status;
 }
 
+int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p) { return or_plan_ex(c, 0, topk_idx, p); }
+
 /* ------------------------------------------------------------------------ */
 /* Independent row-at-a-time simulator of the same rule (for brute force).  */
 /* Places overflow rows one by one: a row goes home while the home rank has */
@@ -238,9 +270,9 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p)
 /* opening a new slot.  Offsets are assigned only after every row has a     */
 /* place.  Outputs: alloc, slot_expert, slot_cnt, fb_cnt, dest, status.     */
 /* ------------------------------------------------------------------------ */
-int or_plan_unitwise(const or_cfg *c, const int32_t *topk_idx, int32_t *alloc,
-                     int32_t *slot_expert, int32_t *slot_cnt, int32_t *fb_cnt,
-                     int32_t *dest, int32_t *status_out)
+int or_plan_unitwise_ex(const or_cfg *c, int mode, const int32_t *topk_idx, int32_t *alloc,
+                        int32_t *slot_expert, int32_t *slot_cnt, int32_t *fb_cnt, int32_t *dest,
+                        int32_t *status_out)
 {
     const int R = c->R, L = c->L, B = c->B, N = R * L;
     const int64_t G = (int64_t)R * c->S * c->K;
@@ -260,12 +292,17 @@ int or_plan_unitwise(const or_cfg *c, const int32_t *topk_idx, int32_t *alloc,
     for (int e = 0; e < N; ++e) fillpos[e] = count[e];
     for (int64_t g = 0; g < G; ++g) order[fillpos[topk_idx[g]]++] = g;
 
-    /* placement kind per row: 0 home, 1 slot (rank, slot), 2 fallback */
+    /* placement per row: kind 0 home, 1 piece (index in the piece list), 2 fallback */
     int *kind = (int *)malloc(sizeof(int) * (size_t)(G > 0 ? G : 1));
-    int *prank = (int *)malloc(sizeof(int) * (size_t)(G > 0 ? G : 1));
-    int *pslot = (int *)malloc(sizeof(int) * (size_t)(G > 0 ? G : 1));
-    int64_t *rows = (int64_t *)calloc((size_t)R, sizeof(int64_t));   /* rows in [0,C) */
-    int *used = (int *)calloc((size_t)R, sizeof(int));
+    int *pidx = (int *)malloc(sizeof(int) * (size_t)(G > 0 ? G : 1));
+    int64_t *rows = (int64_t *)calloc((size_t)R, sizeof(int64_t)); /* rows in [0,C) */
+    int *npc_r = (int *)calloc((size_t)R, sizeof(int));            /* pieces per receiver */
+    int maxp = (int)(N + R + 1);
+    int *pc_rank = (int *)malloc(sizeof(int) * (size_t)maxp);
+    int *pc_slot = (int *)malloc(sizeof(int) * (size_t)maxp);
+    int *pc_exp = (int *)malloc(sizeof(int) * (size_t)maxp);
+    int64_t *pc_n = (int64_t *)calloc((size_t)maxp, sizeof(int64_t));
+    int np = 0;
     for (int i = 0; i < R * B; ++i) { slot_expert[i] = -1; slot_cnt[i] = 0; }
     for (int e = 0; e < N; ++e) fb_cnt[e] = 0;
 
@@ -273,80 +310,90 @@ int or_plan_unitwise(const or_cfg *c, const int32_t *topk_idx, int32_t *alloc,
     for (int e = 0; e < N; ++e) {
         int h = e / L;
         for (int64_t q = count[e]; q < count[e + 1]; ++q) {
-            if (rows[h] < C) {
-                kind[q] = 0; prank[q] = h; pslot[q] = -1;
-                rows[h]++;
-            } else {
-                kind[q] = -1;
-            }
+            if (rows[h] < C) { kind[q] = 0; rows[h]++; }
+            else kind[q] = -1;
         }
     }
     /* pass 2: overflow rows one at a time, expert by expert */
     for (int e = 0; e < N; ++e) {
-        int h = e / L;
-        int cur = -1, curslot = -1;
+        int cur = -1;
         for (int64_t q = count[e]; q < count[e + 1]; ++q) {
             if (kind[q] == 0) continue;
-            if (cur >= 0 && rows[cur] < C) {
-                kind[q] = 1; prank[q] = cur; pslot[q] = curslot;
-                rows[cur]++;
-                slot_cnt[cur * B + curslot]++;
+            if (cur >= 0 && rows[pc_rank[cur]] < C) {
+                kind[q] = 1; pidx[q] = cur; pc_n[cur]++; rows[pc_rank[cur]]++;
                 continue;
             }
             int pick = -1;
             for (int r = 0; r < R; ++r)
-                if (rows[r] < C && used[r] < B) { pick = r; break; }
+                if (rows[r] < C && (mode == 1 || npc_r[r] < B)) { pick = r; break; }
             if (pick >= 0) {
-                cur = pick;
-                curslot = used[pick]++;
-                slot_expert[cur * B + curslot] = e;
-                kind[q] = 1; prank[q] = cur; pslot[q] = curslot;
-                rows[cur]++;
-                slot_cnt[cur * B + curslot]++;
+                cur = np++;
+                pc_rank[cur] = pick;
+                pc_slot[cur] = npc_r[pick] < B ? npc_r[pick] : -1;
+                pc_exp[cur] = e;
+                npc_r[pick]++;
+                kind[q] = 1; pidx[q] = cur; pc_n[cur] = 1; rows[pick]++;
             } else {
                 cur = -1;
-                kind[q] = 2; prank[q] = h; pslot[q] = -1;
+                kind[q] = 2;
                 fb_cnt[e]++;
             }
         }
     }
-    /* offsets: home rows per rank in expert order, then slots, fallback from C */
+    /* offsets: home rows per rank in expert order, then slotted pieces by
+     * slot, then remote pieces in creation order; fallback from C */
     int64_t *home_base = (int64_t *)calloc((size_t)N, sizeof(int64_t));
-    int64_t *slot_base = (int64_t *)calloc((size_t)R * (B > 0 ? B : 1), sizeof(int64_t));
-    int64_t *fb_base = (int64_t *)calloc((size_t)N, sizeof(int64_t));
     int64_t *home_n = (int64_t *)calloc((size_t)N, sizeof(int64_t));
+    int64_t *pc_base = (int64_t *)calloc((size_t)maxp, sizeof(int64_t));
+    int64_t *fb_base = (int64_t *)calloc((size_t)N, sizeof(int64_t));
     for (int e = 0; e < N; ++e)
         for (int64_t q = count[e]; q < count[e + 1]; ++q)
             if (kind[q] == 0) home_n[e]++;
     for (int r = 0; r < R; ++r) {
         int64_t off = 0;
         for (int loc = 0; loc < L; ++loc) { home_base[r * L + loc] = off; off += home_n[r * L + loc]; }
-        for (int b = 0; b < B; ++b) { slot_base[r * B + b] = off; off += slot_cnt[r * B + b]; }
+        for (int b = 0; b < B; ++b)
+            for (int k = 0; k < np; ++k)
+                if (pc_rank[k] == r && pc_slot[k] == b) {
+                    pc_base[k] = off; off += pc_n[k];
+                    slot_expert[r * B + b] = pc_exp[k];
+                    slot_cnt[r * B + b] = (int32_t)pc_n[k];
+                }
+        for (int k = 0; k < np; ++k)
+            if (pc_rank[k] == r && pc_slot[k] < 0) { pc_base[k] = off; off += pc_n[k]; }
         int64_t fo = C;
         for (int loc = 0; loc < L; ++loc) { fb_base[r * L + loc] = fo; fo += fb_cnt[r * L + loc]; }
         if (fo > c->C_max) status |= OR_ST_CAPACITY;
     }
     for (int64_t i = 0; i < (int64_t)N * R; ++i) alloc[i] = 0;
+    int64_t *pc_used = (int64_t *)calloc((size_t)maxp, sizeof(int64_t));
     for (int e = 0; e < N; ++e) {
+        int h = e / L;
         int64_t nh = 0, nf = 0;
-        int64_t *ns = (int64_t *)calloc((size_t)R * (B > 0 ? B : 1), sizeof(int64_t));
         for (int64_t q = count[e]; q < count[e + 1]; ++q) {
             int64_t row;
-            if (kind[q] == 0) row = home_base[e] + nh++;
-            else if (kind[q] == 1) row = slot_base[prank[q] * B + pslot[q]] + ns[prank[q] * B + pslot[q]]++;
-            else row = fb_base[e] + nf++;
-            alloc[(int64_t)e * R + prank[q]]++;
-            dest[order[q]] = (int32_t)(prank[q] * (int64_t)c->C_max + row);
+            int rank;
+            if (kind[q] == 0) { rank = h; row = home_base[e] + nh++; }
+            else if (kind[q] == 1) { rank = pc_rank[pidx[q]]; row = pc_base[pidx[q]] + pc_used[pidx[q]]++; }
+            else { rank = h; row = fb_base[e] + nf++; }
+            alloc[(int64_t)e * R + rank]++;
+            dest[order[q]] = (int32_t)(rank * (int64_t)c->C_max + row);
         }
-        free(ns);
     }
     int64_t fb_total = 0;
     for (int e = 0; e < N; ++e) fb_total += fb_cnt[e];
     if (fb_total > 0) status |= OR_ST_FALLBACK;
-    free(count); free(order); free(fillpos); free(kind); free(prank); free(pslot);
-    free(rows); free(used); free(home_base); free(slot_base); free(fb_base); free(home_n);
+    free(count); free(order); free(fillpos); free(kind); free(pidx); free(rows); free(npc_r);
+    free(pc_rank); free(pc_slot); free(pc_exp); free(pc_n); free(home_base); free(home_n);
+    free(pc_base); free(fb_base); free(pc_used);
     *status_out = status;
     return status;
+}
+
+int or_plan_unitwise(const or_cfg *c, const int32_t *topk_idx, int32_t *alloc, int32_t *slot_expert,
+                     int32_t *slot_cnt, int32_t *fb_cnt, int32_t *dest, int32_t *status_out)
+{
+    return or_plan_unitwise_ex(c, 0, topk_idx, alloc, slot_expert, slot_cnt, fb_cnt, dest, status_out);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -386,12 +433,28 @@ void or_dispatch(const or_cfg *c, const int32_t *dest, const uint16_t *x, uint16
 
 /* O8 stand-in expert: y[row] = bf16(float(recv[row]) * scale[expert(row)]),
  * one fp32 multiply; expert(row) from the segment tables. */
+static void or_scale_rows(const or_cfg *c, int64_t row0, int64_t n, int e, const uint16_t *recv,
+                          const float *scale, uint16_t *y)
+{
+    const int64_t H = c->H;
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t h = 0; h < H; ++h) {
+            float v = or_bf16_to_f32(recv[(row0 + i) * H + h]) * scale[e];
+            y[(row0 + i) * H + h] = or_f32_to_bf16(v);
+        }
+}
+
+/* remote pieces (slot -1, remote-weights mode) are not in the segment
+ * tables: rep_* describe them (n_rep pieces; may be 0) */
 void or_expert_scale(const or_cfg *c, const int32_t *seg_off, const int32_t *seg_len,
                      const int32_t *slot_expert, const uint16_t *recv, const float *scale,
-                     uint16_t *y)
+                     uint16_t *y, int n_rep, const int32_t *rep_expert, const int32_t *rep_recv,
+                     const int32_t *rep_slot, const int32_t *rep_off, const int32_t *rep_cnt)
 {
     const int R = c->R, L = c->L, B = c->B, SEG = 2 * L + B;
-    const int64_t H = c->H;
+    for (int q = 0; q < n_rep; ++q)
+        if (rep_slot[q] < 0)
+            or_scale_rows(c, (int64_t)rep_recv[q] * c->C_max + rep_off[q], rep_cnt[q], rep_expert[q], recv, scale, y);
     for (int r = 0; r < R; ++r)
         for (int s = 0; s < SEG; ++s) {
             int e;
@@ -399,13 +462,7 @@ void or_expert_scale(const or_cfg *c, const int32_t *seg_off, const int32_t *seg
             else if (s < L + B) e = slot_expert[r * B + (s - L)];
             else e = r * L + (s - L - B);
             if (seg_len[r * SEG + s] == 0 || e < 0) continue;
-            for (int64_t i = 0; i < seg_len[r * SEG + s]; ++i) {
-                int64_t row = (int64_t)r * c->C_max + seg_off[r * SEG + s] + i;
-                for (int64_t h = 0; h < H; ++h) {
-                    float v = or_bf16_to_f32(recv[row * H + h]) * scale[e];
-                    y[row * H + h] = or_f32_to_bf16(v);
-                }
-            }
+            or_scale_rows(c, (int64_t)r * c->C_max + seg_off[r * SEG + s], seg_len[r * SEG + s], e, recv, scale, y);
         }
 }
 

@@ -31,6 +31,15 @@ def row_expert_map(cfg, pl):
             lo = r * Cm + so[r, s]
             assert np.all(m[lo:lo + sl[r, s]] == -1), "overlapping segments"
             m[lo:lo + sl[r, s]] = e
+    # remote pieces (no slot) are described by the piece tables only
+    n = int(pl.get("n_replicas", 0))
+    if n and "rep_off" in pl:
+        for q in range(n):
+            if int(pl["rep_slot"][q]) < 0:
+                lo = int(pl["rep_recv"][q]) * Cm + int(pl["rep_off"][q])
+                cnt = int(pl["rep_cnt"][q])
+                assert np.all(m[lo:lo + cnt] == -1), "overlapping segments"
+                m[lo:lo + cnt] = int(pl["rep_expert"][q])
     return m
 
 
@@ -57,6 +66,10 @@ def check_plan(cfg, ids, pl):
     # replica slots per rank never exceed B
     su = np.asarray(pl["slots_used"])
     assert np.all(su <= B) and np.all(su >= 0)
+    if "rep_slot" in pl:
+        nrep = int(pl["n_replicas"])
+        slotted = np.asarray(pl["rep_slot"])[:nrep] >= 0
+        assert np.array_equal(np.bincount(np.asarray(pl["rep_recv"])[:nrep][slotted], minlength=R), su)
     if B > 0:
         assert np.array_equal((np.asarray(pl["slot_expert"]).reshape(R, B) >= 0).sum(1), su)
     # closed form: migrated rows = total home overflow - fallback

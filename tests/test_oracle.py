@@ -365,3 +365,85 @@ def test_routing_hits_maxvio(target):
     assert all(len(set(row)) == 8 for row in ids[:500].tolist())
     assert np.allclose(r.topk_w.reshape(-1, 8).sum(1), 1.0, atol=1e-6)
     assert np.all(np.diff(r.topk_w.reshape(-1, 8), axis=1) <= 0)
+
+
+# ---------------------------------------------------------------------------
+# Remote-weights mode: overflow beyond a receiver's slots is still placed on
+# it and reads its weights from the home rank, so no row falls back
+# ---------------------------------------------------------------------------
+
+def _compare_unitwise_remote(oracle, cfg, ids):
+    pl = oracle.plan(cfg, ids, mode=oracle.MODE_REMOTE)
+    un = oracle.plan_unitwise(cfg, ids, mode=oracle.MODE_REMOTE)
+    assert pl["status"] == un["status"] == 0
+    for k in ("dest", "alloc", "slot_expert", "slot_cnt", "fb_cnt"):
+        assert np.array_equal(pl[k], un[k]), k
+    info = pc.check_plan(cfg, ids, pl)
+    assert pl["fallback_rows"] == 0
+    assert np.all(info["rows"] == cfg["C"])            # the hard invariant, for any B
+    n = pl["n_replicas"]
+    # the first B pieces of a receiver have slots, the rest are remote
+    for r in range(cfg["R"]):
+        q = np.nonzero(pl["rep_recv"][:n] == r)[0]
+        slots = pl["rep_slot"][q]
+        assert np.array_equal(slots, np.where(np.arange(len(q)) < cfg["B"], np.arange(len(q)), -1))
+        assert np.array_equal(q, np.arange(pl["recv_ptr"][r], pl["recv_ptr"][r + 1]))
+    return pl
+
+
+@pytest.mark.parametrize("R,L,S,K,B", [(2, 2, 2, 2, 1), (3, 1, 2, 1, 0), (4, 1, 2, 1, 1), (2, 2, 3, 1, 0)])
+def test_bruteforce_remote_mode(oracle_lib, R, L, S, K, B):
+    N, T = R * L, R * S
+    cfg = _cfg(R, L, S, K, 8, B)
+    choices = list(itertools.permutations(range(N), K))
+    n = 0
+    for combo in itertools.product(range(len(choices)), repeat=T):
+        ids = np.array([choices[c] for c in combo], np.int32).reshape(R, S, K)
+        _compare_unitwise_remote(oracle_lib, cfg, ids)
+        n += 1
+    assert n == len(choices) ** T
+
+
+def test_remote_mode_closes_the_known_gap(oracle_lib):
+    R, L, S, K, B = 4, 2, 2, 2, 2
+    cfg = _cfg(R, L, S, K, 8, B)                       # no headroom needed
+    ids = pc.ids_from_counts(np.array([2, 3, 2, 3, 2, 3, 1, 0]), R, S, K)
+    pl = _compare_unitwise_remote(oracle_lib, cfg, ids)
+    assert pl["slots_used"].tolist() == [0, 0, 0, 2]
+    assert (pl["rep_slot"] < 0).sum() == 1              # the third piece on rank 3 is remote
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("B", [0, 1, 2])
+def test_remote_mode_random_histograms(oracle_lib, seed, B):
+    rng = np.random.default_rng(seed)
+    R, L, S, K = 8, 4, 64, 4
+    cnt = pc.random_counts(rng, R * L, R * S, K, skew=1.0 + seed)
+    ids = pc.ids_from_counts(cnt, R, S, K)
+    cfg = _cfg(R, L, S, K, 8, B)
+    pl = _compare_unitwise_remote(oracle_lib, cfg, ids)
+    # with slots for every piece the two modes agree
+    if B >= R * L:
+        assert np.array_equal(pl["dest"], oracle_lib.plan(cfg, ids)["dest"])
+
+
+def test_remote_mode_equals_headroom_mode_when_slots_suffice(oracle_lib):
+    for seed in range(5):
+        w = inputs.WORKLOADS["tiny"]
+        r = inputs.routing(w.R, w.L, w.S, w.K, seed, alpha=1.0)
+        a = oracle_lib.plan(w.cfg(), r.topk_idx)
+        b = oracle_lib.plan(w.cfg(), r.topk_idx, mode=oracle_lib.MODE_REMOTE)
+        if a["fallback_rows"] == 0:
+            assert np.array_equal(a["dest"], b["dest"]) and np.array_equal(a["alloc"], b["alloc"])
+
+
+def test_remote_mode_inference_workload(oracle_lib):
+    # the inference workload (B = 4): seed 1 falls back 887 rows under the
+    # headroom rule; with remote weights every rank holds exactly S*K rows
+    w = inputs.WORKLOADS["inference"]
+    r = inputs.routing(w.R, w.L, w.S, w.K, 1, maxvio=4.0)
+    cfg = dict(w.cfg(), C_max=w.C)
+    pl = oracle_lib.plan(cfg, r.topk_idx, mode=oracle_lib.MODE_REMOTE)
+    info = pc.check_plan(cfg, r.topk_idx, pl)
+    assert pl["fallback_rows"] == 0 and np.all(info["rows"] == w.C)
+    assert (pl["rep_slot"] < 0).sum() > 0
