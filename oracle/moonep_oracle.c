@@ -497,18 +497,22 @@ void or_prefetch(const or_cfg *c, const int32_t *slot_expert, const uint16_t *w_
 
 /* O10b reduce_grad: for each expert with replicas, in ascending receiver
  * order, g_home[e] = g_home[e] + g_rep[r][b] (fp32); then zero the used
- * replica slots. */
+ * replica slots.  The reduce buffer is [R, B, H, H'] (twodots.gr): only
+ * pieces that hold a slot have a replica gradient; a piece without one
+ * (remote weights) contributes nothing here. */
 void or_reduce_grad(const or_cfg *c, const int32_t *rep_ptr, const int32_t *rep_recv,
                     const int32_t *rep_slot, float *g_home, float *g_rep, int64_t elems)
 {
     const int N = c->R * c->L;
     for (int e = 0; e < N; ++e) {
         for (int q = rep_ptr[e]; q < rep_ptr[e + 1]; ++q) {
+            if (rep_slot[q] < 0) continue;
             const float *src = g_rep + ((int64_t)rep_recv[q] * c->B + rep_slot[q]) * elems;
             float *dst = g_home + (int64_t)e * elems;
             for (int64_t i = 0; i < elems; ++i) dst[i] = dst[i] + src[i];
         }
         for (int q = rep_ptr[e]; q < rep_ptr[e + 1]; ++q) {
+            if (rep_slot[q] < 0) continue;
             float *src = g_rep + ((int64_t)rep_recv[q] * c->B + rep_slot[q]) * elems;
             for (int64_t i = 0; i < elems; ++i) src[i] = 0.0f;
         }

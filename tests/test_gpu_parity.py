@@ -16,8 +16,8 @@ pytestmark = pytest.mark.gpu
 
 PLAN_TABLES = ["cnt", "keep", "spill", "home_off", "fb_cnt", "fb_off", "load", "deficit", "fill",
                "slots_used", "slot_expert", "slot_cnt", "slot_off", "slot_first_j", "rep_ptr",
-               "rep_expert", "rep_recv", "rep_slot", "rep_first_j", "rep_cnt", "seg_off", "seg_len",
-               "alloc"]
+               "rep_expert", "rep_recv", "rep_slot", "rep_first_j", "rep_cnt", "rep_off", "recv_ptr",
+               "seg_off", "seg_len", "alloc"]
 COUNTS = ["fallback_rows", "n_replicas", "migrated_rows"]
 
 
@@ -55,7 +55,7 @@ def x_host(seed, T, H):
     return inputs.cb_bf16_np(seed, inputs.STREAM_X, np.arange(T * H, dtype=np.int64)).reshape(T, H)
 
 
-def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_seed=0):
+def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_seed=0, remote=False):
     """Every step on a small problem, compared element by element."""
     torch, mp, harness = env
     R, L, S, K, H, B, Cm = (cfg[n] for n in ("R", "L", "S", "K", "H", "B", "C_max"))
@@ -65,9 +65,9 @@ def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_see
     prob.fill_x(seed)
     prob.fill_weights(seed)
     prob.fill_g_rep(seed)
-    prob.plan()
+    prob.plan(flags=mp.PLAN_REMOTE_WEIGHTS if remote else 0)
     gpl = prob.read_plan()
-    opl = oracle.plan(cfg, ids)
+    opl = oracle.plan(cfg, ids, mode=oracle.MODE_REMOTE if remote else oracle.MODE_HEADROOM)
     compare_plan(gpl, opl)
     failed = bool(opl["status"] & (oracle.ST_CAPACITY | oracle.ST_EXPERT_ID))
     if not failed:
@@ -458,3 +458,59 @@ def test_reduce_grad_twice_after_one_plan(env):
         oracle.reduce_grad(cfg, opl, gh, gr, E)
         assert np.array_equal(prob.g_home.cpu().numpy().view(np.uint32), gh.view(np.uint32))
         assert np.array_equal(prob.g_rep.cpu().numpy().view(np.uint32), gr.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# remote-weights plan mode (the pages' inference fallback)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", [
+    # R, L, S, K, H, B
+    (4, 2, 2, 2, 16, 2),        # the known gap: a third piece on rank 3 is remote
+    (16, 24, 64, 8, 64, 4),     # inference-style slot limit
+    (8, 4, 64, 4, 64, 0),       # no slots at all: every piece remote
+    (4, 4, 64, 2, 128, 4),
+    (64, 64, 32, 8, 32, 1),     # N at its maximum, one slot
+])
+def test_remote_weights_mode(env, case):
+    R, L, S, K, H, B = case
+    cfg = cfg_of(R, L, S, K, H, B)                       # C_max = C: no headroom needed
+    if (R, L) == (4, 2):
+        ids = pc.ids_from_counts(np.array([2, 3, 2, 3, 2, 3, 1, 0]), R, S, K)
+        w = np.full((R, S, K), 0.5, np.float32)
+    else:
+        r = inputs.routing(R, L, S, K, 1, maxvio=4.0 if R * L > 64 else None, alpha=None if R * L > 64 else 1.0)
+        ids, w = r.topk_idx, r.topk_w
+    prob, gpl, opl = run_full_compare(env, cfg, ids, w, remote=True)
+    assert gpl["fallback_rows"] == 0
+    assert np.all(gpl["alloc"].sum(0) == cfg["C"])
+    if B == 0 and gpl["n_replicas"]:
+        assert np.all(gpl["rep_slot"] == -1)
+
+
+def test_remote_weights_inference_workload(env):
+    # the inference workload at seed 1 falls back 887 rows under the headroom
+    # rule; with remote weights and C_max = C every rank holds exactly S*K rows
+    torch, mp, harness = env
+    wl = inputs.WORKLOADS["inference"]
+    cfg = dict(wl.cfg(), C_max=wl.C)
+    r = inputs.routing(wl.R, wl.L, wl.S, wl.K, 1, maxvio=4.0)
+    prob = harness.Problem(cfg, poison=True)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.fill_x(1)
+    prob.plan(flags=mp.PLAN_REMOTE_WEIGHTS)
+    prob.dispatch()
+    prob.combine()
+    torch.cuda.synchronize()
+    gpl = prob.read_plan()
+    opl = oracle.plan(cfg, r.topk_idx, mode=oracle.MODE_REMOTE)
+    compare_plan(gpl, opl)
+    assert gpl["fallback_rows"] == 0 and (gpl["rep_slot"] < 0).sum() > 0
+    dest = prob.dest.cpu().numpy()
+    assert np.array_equal(dest, opl["dest"].reshape(-1))
+    gs = np.random.default_rng(0).choice(wl.T * wl.K, 1024, replace=False)
+    rows = harness.to_u16(prob.recv[torch.from_numpy(dest[gs]).long().cuda()])
+    want = inputs.cb_bf16_np(1, inputs.STREAM_X, (gs // wl.K)[:, None] * wl.H + np.arange(wl.H)[None, :])
+    assert np.array_equal(rows, want)
+    # with C_max = C and no fallback every receive row is used
+    assert not np.any(np.all(harness.to_u16(prob.recv[::97]) == 0xFFFF, axis=1))

@@ -447,3 +447,27 @@ def test_remote_mode_inference_workload(oracle_lib):
     info = pc.check_plan(cfg, r.topk_idx, pl)
     assert pl["fallback_rows"] == 0 and np.all(info["rows"] == w.C)
     assert (pl["rep_slot"] < 0).sum() > 0
+
+
+def test_remote_pieces_carry_no_replica_gradient(oracle_lib):
+    # remote pieces have no slot, so reduce_grad adds slotted pieces only and
+    # leaves every other slot as it was
+    R, L, S, K, B = 4, 2, 2, 2, 2
+    cfg = _cfg(R, L, S, K, 8, B)
+    ids = pc.ids_from_counts(np.array([2, 3, 2, 3, 2, 3, 1, 0]), R, S, K)
+    pl = oracle_lib.plan(cfg, ids, mode=oracle_lib.MODE_REMOTE)
+    E = 16
+    gh = inputs.cb_f32_np(1, inputs.STREAM_G_HOME, np.arange(R * L * E)).reshape(R * L, E)
+    gr = inputs.cb_f32_np(1, inputs.STREAM_G_REP, np.arange(R * B * E)).reshape(R * B, E)
+    h0, r0 = gh.copy(), gr.copy()
+    oracle_lib.reduce_grad(cfg, pl, gh, gr, E)
+    slotted = pl["rep_slot"] >= 0
+    slots = pl["rep_recv"][slotted] * B + pl["rep_slot"][slotted]
+    for e in range(R * L):
+        q = [pl["rep_recv"][i] * B + pl["rep_slot"][i] for i in range(pl["rep_ptr"][e], pl["rep_ptr"][e + 1])
+             if pl["rep_slot"][i] >= 0]
+        want = h0[e].astype(np.float64) + r0[q].astype(np.float64).sum(0)
+        assert np.allclose(gh[e], want, rtol=0, atol=4 * 2.0 ** -24 * (np.abs(h0[e]) + np.abs(r0[q]).sum(0)))
+    used = np.zeros(R * B, bool)
+    used[slots] = True
+    assert np.all(gr[used] == 0) and np.array_equal(gr[~used], r0[~used])
