@@ -117,15 +117,20 @@ typedef struct {
 /* Workspace layout: offsets in int32 words from the workspace base.  The
  * header occupies words [0, MOONEP_WS_HEADER_WORDS):
  *   0 status, 1 fallback_rows, 2 n_replicas, 3 migrated_rows, 4 n_ranges,
- *   5..12 the cfg it was planned for, 13 replicated-expert count.
+ *   5..12 the cfg it was planned for, 13 replicated-expert count,
+ *   14 plan flags, 15 pieces with a slot.
  * Tables ([N] unless noted): cnt = copies per expert (tokens_per_expert);
  * keep, spill, home_off (row of e's local segment), fb_cnt, fb_off (row of
  * e's fallback segment); [R]: load (copies homed on r), deficit (C - load,
  * floored at 0), fill (rows used below C), slots_used; [R*B]: slot_expert
  * (-1 = empty), slot_cnt, slot_off, slot_first_j (first copy index j held);
  * rep_ptr [N+1] (CSR over pieces, pieces in ascending (expert, receiver)
- * order) and per piece rep_expert, rep_recv, rep_slot, rep_first_j,
- * rep_cnt; rx_expert (experts with >= 1 piece, ascending); route_ptr [N+1],
+ * order) and per piece rep_expert, rep_recv, rep_slot (-1 = no slot:
+ * remote weights), rep_first_j, rep_cnt, rep_off (first row on the
+ * receiver); recv_ptr [R+1] (the pieces of receiver r are [recv_ptr[r],
+ * recv_ptr[r+1]): piece order is receiver-major as well); slot_piece (the
+ * pieces that have a slot, in piece order); rx_expert (experts with >= 1
+ * piece, ascending); route_ptr [N+1],
  * route_end, route_base (copy j of e goes to flat row route_base[p] + j for
  * the first entry p of e with j < route_end[p]); seg_off, seg_len
  * [R][2L+B] (L local, B slot, L fallback segments per rank); alloc [N][R]
@@ -147,6 +152,7 @@ typedef struct {
     int64_t alloc;
     int64_t tables_end; /* = base                                      */
     int64_t base;
+    int64_t rep_off, recv_ptr, slot_piece; /* (between rep_cnt and rx_expert in memory) */
 } moonep_ws_layout_t;
 
 /* Per-rank buffer sizes in bytes, as a real deployment would allocate them
@@ -172,6 +178,24 @@ MOONEP_API int moonep_rank_bytes(const moonep_cfg_t *cfg, int64_t elems_per_expe
  * bytes, 16-byte aligned, owned by the caller; fully rewritten.  One memset
  * of the header and one persistent cooperative kernel; no host sync. */
 MOONEP_API int moonep_plan(const moonep_cfg_t *cfg, const int32_t *topk_idx, void *ws, void *stream);
+
+/* Plan flags for moonep_plan_ex. */
+#define MOONEP_PLAN_REMOTE_WEIGHTS 0x1
+
+/* moonep_plan with flags.  MOONEP_PLAN_REMOTE_WEIGHTS selects the pages'
+ * inference fallback instead of the headroom rule: when a receiver would need
+ * more replicas than its B prefetch slots, the group GEMM reads the expert's
+ * weights from its home rank (twodots.gr "MoonEP balances AI experts in MoE
+ * models", memory-contract paragraphs; "The Busiest Rank Sets Your Step
+ * Time", "Installation and integration"), so receivers take spilled rows while
+ * they have room whatever their slots.  Their first B pieces get slots; later
+ * pieces have rep_slot = -1 and follow the slotted ones on the receiver (rows
+ * rep_off[p] .. rep_off[p] + rep_cnt[p]).  No row falls back: every rank
+ * holds exactly C rows and C_max = C suffices.  prefetch copies slotted pieces
+ * only, reduce_grad reduces slotted pieces only (remote pieces carry no
+ * gradient slot: the mode is for inference).  flags = 0 is moonep_plan. */
+MOONEP_API int moonep_plan_ex(const moonep_cfg_t *cfg, int32_t flags, const int32_t *topk_idx, void *ws,
+                              void *stream);
 
 /* Dispatch (same flowchart: dispatch sends tokens straight to their final
  * slot on the remote rank).  x: device bf16 [R*S][H] hidden states;

@@ -167,7 +167,12 @@ const char *moonep_last_error(void) { return g_err.c_str(); }
 const char *moonep_version(void) { return "moonep-b200 0.1 (sm_100a)"; }
 
 int moonep_plan(const moonep_cfg_t *cfg, const int32_t *topk_idx, void *ws, void *stream) {
+    return moonep_plan_ex(cfg, 0, topk_idx, ws, stream);
+}
+
+int moonep_plan_ex(const moonep_cfg_t *cfg, int32_t flags, const int32_t *topk_idx, void *ws, void *stream) {
     TRY(check_cfg(cfg));
+    if (flags & ~MOONEP_PLAN_REMOTE_WEIGHTS) return fail(MOONEP_ERR_ARG, "unknown plan flags 0x%x", flags);
     const int64_t T = (int64_t)cfg->R * cfg->S;
     TRY(check_ptr(topk_idx, 4, "topk_idx", T > 0));
     TRY(check_ptr(ws, 16, "ws", true));
@@ -177,6 +182,7 @@ int moonep_plan(const moonep_cfg_t *cfg, const int32_t *topk_idx, void *ws, void
     cudaStream_t s = (cudaStream_t)stream;
     PlanParams p{};
     p.cfg = *cfg;
+    p.flags = flags;
     p.N = N;
     p.T = T;
     compute_layout(*cfg, p.lay);

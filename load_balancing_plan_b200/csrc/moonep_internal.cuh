@@ -21,6 +21,8 @@ enum : int {
     HDR_NRANGES = 4,
     HDR_CFG = 5,  // 8 words: R L S K H B C C_max
     HDR_NRX = 13,
+    HDR_FLAGS = 14,  // plan flags (MOONEP_PLAN_*)
+    HDR_NSLOT = 15,  // pieces with a prefetch slot
     HDR_BAR_COUNT = 16,
     HDR_BAR_GEN = 17,
     HDR_TOTAL_SPILL = 20,
@@ -40,11 +42,12 @@ __host__ __device__ inline int64_t num_ranges(int64_t T) { return T < kRanges ? 
 // token range q of Q: [q*T/Q, (q+1)*T/Q)
 __host__ __device__ inline int64_t range_begin(int64_t q, int64_t T, int64_t Q) { return q * T / Q; }
 
+// pieces: a receiver's range of the spill stream touches consecutive chunks,
+// so pieces <= spilled chunks + receivers - 1 < N + R (slots no longer bound
+// them once pieces may read their weights remotely)
 __host__ __device__ inline int64_t max_pieces(int R, int L, int B) {
-    int64_t N = (int64_t)R * L;
-    int64_t a = (int64_t)R * B, b = N + R;
-    int64_t p = a < b ? a : b;
-    return p > 0 ? p : 1;
+    (void)B;
+    return (int64_t)R * L + R;
 }
 
 // Fills the layout; returns false if the configuration is out of range.
@@ -77,6 +80,9 @@ __host__ __device__ inline void compute_layout(const moonep_cfg_t &c, moonep_ws_
     l.rep_slot = o; o += P;
     l.rep_first_j = o; o += P;
     l.rep_cnt = o; o += P;
+    l.rep_off = o; o += P;
+    l.recv_ptr = o; o += R + 1;
+    l.slot_piece = o; o += RB;
     l.rx_expert = o; o += N;
     l.route_ptr = o; o += N + 1;
     l.route_end = o; o += NR;
@@ -97,6 +103,7 @@ __host__ __device__ inline void compute_layout(const moonep_cfg_t &c, moonep_ws_
 // ---------------------------------------------------------------------------
 struct PlanParams {
     moonep_cfg_t cfg;
+    int32_t flags;
     int32_t N;
     int64_t T, Q;
     const int32_t *ids;

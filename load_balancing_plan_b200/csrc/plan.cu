@@ -159,7 +159,8 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     int *s_ch = sm + 4 * N;   // chunk -> expert
     int *s_y = sm + 5 * N;    // chunk index, then pieces per expert -> rep_ptr
     int *s_hoff = sm + 6 * N; // row of the expert's local segment
-    __shared__ int s_def[kMaxR], s_rp[kMaxR], s_rt[kMaxR], s_ri0[kMaxR], s_rnp[kMaxR], s_rpb[kMaxR];
+    __shared__ int s_def[kMaxR], s_rp[kMaxR], s_rt[kMaxR], s_ri0[kMaxR], s_rnp[kMaxR], s_rpb[kMaxR], s_spb[kMaxR];
+    const bool remote = (p.flags & MOONEP_PLAN_REMOTE_WEIGHTS) != 0;
 
     TRACE(ws, 3);
     // keep/spill: each home rank keeps rows in local-expert order up to C
@@ -202,15 +203,15 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     TRACE(ws, 4);
 
     // receiver walk: receiver r takes the stream from p_r until its deficit
-    // is filled or it has touched B chunks
+    // is filled or (headroom rule) it has touched B chunks
     int pos = 0, i0 = 0;
     for (int r = 0; r < R; ++r) {
         const int d = s_def[r];
         int take = 0, np = 0, ir = i0;
         const int pr = pos;
-        if (d > 0 && pos < total_spill && B > 0) {
+        if (d > 0 && pos < total_spill && (remote || B > 0)) {
             i0 = advance_chunk(s_ce, M, i0, pos);
-            const int i1 = min(i0 + B - 1, M - 1);
+            const int i1 = remote ? M - 1 : min(i0 + B - 1, M - 1);
             take = min(d, s_ce[i1] - pos);
             const int il = advance_chunk(s_ce, M, i0, pos + take - 1);
             np = il - i0 + 1;
@@ -226,7 +227,8 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     }
     __syncwarp();
     const int p_end = pos;
-    // pieces per receiver -> exclusive prefix (R <= 64: two per lane)
+    // pieces per receiver -> exclusive prefix (R <= 64: two per lane), and
+    // the same for the pieces that get a slot (the first B of each receiver)
     const int na = lane < R ? s_rnp[lane] : 0;
     const int nb = lane + 32 < R ? s_rnp[lane + 32] : 0;
     const int ia = warp_incl_scan(na);
@@ -235,54 +237,75 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     if (lane < R) s_rpb[lane] = ia - na;
     if (lane + 32 < R) s_rpb[lane + 32] = tot_a + ib - nb;
     const int P = tot_a + __shfl_sync(0xffffffffu, ib, 31);
+    const int sa = min(na, B), sb = min(nb, B);
+    const int isa = warp_incl_scan(sa);
+    const int tot_sa = __shfl_sync(0xffffffffu, isa, 31);
+    const int isb = warp_incl_scan(sb);
+    if (lane < R) s_spb[lane] = isa - sa;
+    if (lane + 32 < R) s_spb[lane + 32] = tot_sa + isb - sb;
+    const int NSLOT = tot_sa + __shfl_sync(0xffffffffu, isb, 31);
     // replicated experts are the chunks that start before the walk's end
     const int nrx = p_end > 0 ? advance_chunk(s_ce, M, 0, p_end - 1) + 1 : 0;
     for (int e = lane; e < N; e += 32) s_y[e] = 0;  // pieces per expert
     for (int r = lane; r < R; r += 32) {
         ws[lay.fill + r] = C - s_def[r] + s_rt[r];
-        ws[lay.slots_used + r] = s_rnp[r];
+        ws[lay.slots_used + r] = min(s_rnp[r], B);
+        ws[lay.recv_ptr + r] = s_rpb[r];
     }
+    if (lane == 0) ws[lay.recv_ptr + R] = P;
     __syncwarp();
     TRACE(ws, 5);
 
-    // pieces, slots and their segments, route entries and alloc entries
-    for (int idx = lane; idx < R * B; idx += 32) {
-        const int r = idx / B, b = idx - r * B;
-        const int sg = r * SEG + L + b;
-        if (b < s_rnp[r]) {
+    // pieces (receiver by receiver), their slots and slot segments, route
+    // entries and alloc entries
+    for (int r = 0; r < R; ++r) {
+        const int npr = s_rnp[r];
+        for (int b = lane; b < npr; b += 32) {
             const int i = s_ri0[r] + b;
             const int e = s_ch[i];
             const int ce = s_ce[i], cs = ce - s_sp[e];
             const int lo = max(s_rp[r], cs), hi = min(s_rp[r] + s_rt[r], ce);
             const int n = hi - lo;
             const int fj = (s_cnt[e] - s_sp[e]) + (lo - cs);
-            const int soff = (C - s_def[r]) + (lo - s_rp[r]);
+            const int off = (C - s_def[r]) + (lo - s_rp[r]);
             const int gp = s_rpb[r] + b;
+            const int slot = b < B ? b : -1;
             ws[lay.rep_expert + gp] = e;
             ws[lay.rep_recv + gp] = r;
-            ws[lay.rep_slot + gp] = b;
+            ws[lay.rep_slot + gp] = slot;
             ws[lay.rep_first_j + gp] = fj;
             ws[lay.rep_cnt + gp] = n;
-            ws[lay.slot_expert + idx] = e;
-            ws[lay.slot_cnt + idx] = n;
-            ws[lay.slot_off + idx] = soff;
-            ws[lay.slot_first_j + idx] = fj;
-            ws[lay.seg_off + sg] = soff;
-            ws[lay.seg_len + sg] = n;
+            ws[lay.rep_off + gp] = off;
+            if (slot >= 0) {
+                const int idx = r * B + slot;
+                const int sg = r * SEG + L + slot;
+                ws[lay.slot_expert + idx] = e;
+                ws[lay.slot_cnt + idx] = n;
+                ws[lay.slot_off + idx] = off;
+                ws[lay.slot_first_j + idx] = fj;
+                ws[lay.seg_off + sg] = off;
+                ws[lay.seg_len + sg] = n;
+                ws[lay.slot_piece + s_spb[r] + slot] = gp;
+            }
             // route entry of this piece: after e's home entry and e's earlier pieces
             ws[lay.route_end + 2 * e + 1 + gp] = fj + n;
-            ws[lay.route_base + 2 * e + 1 + gp] = r * Cm + soff - fj;
+            ws[lay.route_base + 2 * e + 1 + gp] = r * Cm + off - fj;
             ws[lay.alloc + (int64_t)e * R + r] = n;
             atomicAdd(&s_y[e], 1);
-        } else {
-            const int fill = C - s_def[r] + s_rt[r];
-            ws[lay.slot_expert + idx] = -1;
-            ws[lay.slot_cnt + idx] = 0;
-            ws[lay.slot_off + idx] = fill;
-            ws[lay.slot_first_j + idx] = 0;
-            ws[lay.seg_off + sg] = fill;
-            ws[lay.seg_len + sg] = 0;
         }
+    }
+    // slots no piece took
+    for (int idx = lane; idx < R * B; idx += 32) {
+        const int r = idx / B, b = idx - r * B;
+        if (b < s_rnp[r]) continue;
+        const int sg = r * SEG + L + b;
+        const int fill = C - s_def[r] + s_rt[r];
+        ws[lay.slot_expert + idx] = -1;
+        ws[lay.slot_cnt + idx] = 0;
+        ws[lay.slot_off + idx] = fill;
+        ws[lay.slot_first_j + idx] = 0;
+        ws[lay.seg_off + sg] = fill;
+        ws[lay.seg_len + sg] = 0;
     }
     for (int x = lane; x < nrx; x += 32) ws[lay.rx_expert + x] = s_ch[x];
     // fallback rows: the stream beyond the walk's end, per chunk (s_x: A_e -> fb_cnt)
@@ -332,6 +355,8 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[HDR_NREP] = P;
         ws[HDR_MIGRATED] = total_spill - fallback;
         ws[HDR_NRX] = nrx;
+        ws[HDR_FLAGS] = p.flags;
+        ws[HDR_NSLOT] = NSLOT;
         ws[HDR_TOTAL_SPILL] = total_spill;
         ws[HDR_PEND] = p_end;
         TRACE(ws, 7);

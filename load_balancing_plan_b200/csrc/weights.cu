@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
     fence_mbar_init();
     fence_proxy_async_smem();
 
-    const int64_t P = __ldcg(ws + HDR_NREP);
+    const int64_t P = __ldcg(ws + HDR_NSLOT);  // pieces with a slot (all, under the headroom rule)
     const int64_t bytes_per = p.vecs * 16;
     const int64_t cps = (bytes_per + kPfChunk - 1) / kPfChunk;
     const int64_t units = P * cps;
@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
     for (int64_t it = 0; it < n + kPfAhead; ++it) {
         if (it < n) {
             const int64_t u = u0 + it;
-            const int64_t gp = u / cps, c = u - gp * cps;
+            const int64_t sp = u / cps, c = u - sp * cps;
+            const int gp = __ldg(ws + p.lay.slot_piece + sp);
             const int e = __ldg(ws + p.lay.rep_expert + gp);
             const uint32_t bytes = (uint32_t)min((int64_t)kPfChunk, bytes_per - c * kPfChunk);
             const int s = (int)(it % kPfStages);
@@ -91,7 +92,8 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
                 }
             if (fail) break;
             const int64_t u = u0 + j;
-            const int64_t gp = u / cps, c = u - gp * cps;
+            const int64_t sp = u / cps, c = u - sp * cps;
+            const int gp = __ldg(ws + p.lay.slot_piece + sp);
             const int64_t slot = (int64_t)__ldg(ws + p.lay.rep_recv + gp) * B + __ldg(ws + p.lay.rep_slot + gp);
             const uint32_t bytes = (uint32_t)min((int64_t)kPfChunk, bytes_per - c * kPfChunk);
             bulk_s2g_plain(dst_base + slot * bytes_per + c * kPfChunk, smem + (size_t)s * kPfChunk, bytes);
@@ -144,13 +146,20 @@ __global__ void __launch_bounds__(kThreads) reduce_grad_kernel(const __grid_cons
         const int64_t x = u / cps, c = u - x * cps;
         const int e = __ldg(ws + p.lay.rx_expert + x);
         const int pb = __ldg(ws + p.lay.rep_ptr + e), pe = __ldg(ws + p.lay.rep_ptr + e + 1);
-        const int np = pe - pb;
-        __syncthreads();  // s_slot of the previous unit is no longer read
-        if (threadIdx.x < np)
-            s_slot[threadIdx.x] =
-                ((int64_t)__ldg(ws + p.lay.rep_recv + pb + threadIdx.x) * B + __ldg(ws + p.lay.rep_slot + pb + threadIdx.x)) *
-                p.vecs;
+        __shared__ int s_np;
+        __syncthreads();  // s_slot and s_np of the previous unit are no longer read
+        if (threadIdx.x == 0) {
+            // the expert's pieces in receiver order; pieces without a slot
+            // (remote weights) carry no replica gradient
+            int n = 0;
+            for (int q = pb; q < pe; ++q) {
+                const int sl = __ldg(ws + p.lay.rep_slot + q);
+                if (sl >= 0) s_slot[n++] = ((int64_t)__ldg(ws + p.lay.rep_recv + q) * B + sl) * p.vecs;
+            }
+            s_np = n;
+        }
         __syncthreads();
+        const int np = s_np;
         const int64_t n = min((int64_t)kChunkVecs, p.vecs - c * kChunkVecs);
         const int64_t off = c * kChunkVecs;
         float4 *home = g_home + (int64_t)e * p.vecs + off;

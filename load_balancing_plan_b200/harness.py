@@ -85,8 +85,11 @@ class Problem:
             inputs.cb_fill_torch(self.g_rep, seed, inputs.STREAM_G_REP)
 
     # ----------------------------------------------------------------- calls
-    def plan(self, stream=None):
-        mp.moonep_plan(self.cfg, self.ids, self.ws, stream)
+    def plan(self, stream=None, flags=0):
+        if flags:
+            mp.moonep_plan_ex(self.cfg, flags, self.ids, self.ws, stream)
+        else:
+            mp.moonep_plan(self.cfg, self.ids, self.ws, stream)
 
     def dispatch(self, stream=None):
         mp.moonep_dispatch(self.cfg, self.ws, self.x, self.ids, self.recv, self.dest, stream)
@@ -123,6 +126,11 @@ class Problem:
                     continue
                 e = r * L + s if s < L else (se[r, s - L] if s < L + B else r * L + (s - L - B))
                 m[r * Cm + so[r, s]: r * Cm + so[r, s] + sl[r, s]] = e
+        # pieces without a slot (remote weights) are in the piece tables only
+        for q in range(pl["n_replicas"]):
+            if pl["rep_slot"][q] < 0:
+                lo = pl["rep_recv"][q] * Cm + pl["rep_off"][q]
+                m[lo: lo + pl["rep_cnt"][q]] = pl["rep_expert"][q]
         return torch.from_numpy(m).to(self.device)
 
     def expert_scale(self, scale: np.ndarray, row_expert=None):

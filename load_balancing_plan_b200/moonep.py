@@ -24,6 +24,7 @@ OK, ERR_ARG, ERR_CUDA, ERR_DEVICE = 0, 1, 2, 3
 ST_EXPERT_ID, ST_CAPACITY, ST_TIMEOUT, ST_DEST, ST_CFG = 0x1, 0x2, 0x4, 0x8, 0x10
 ST_ERROR_MASK, ST_FALLBACK = 0xFF, 0x100
 WS_HEADER_WORDS = 64
+PLAN_REMOTE_WEIGHTS = 0x1
 
 
 class MoonepError(RuntimeError):
@@ -44,7 +45,8 @@ LAYOUT_FIELDS = ["words", "n_ranges", "max_pieces", "cnt", "keep", "spill", "hom
                  "fb_off", "load", "deficit", "fill", "slots_used", "slot_expert", "slot_cnt",
                  "slot_off", "slot_first_j", "rep_ptr", "rep_expert", "rep_recv", "rep_slot",
                  "rep_first_j", "rep_cnt", "rx_expert", "route_ptr", "route_end", "route_base",
-                 "seg_off", "seg_len", "alloc", "tables_end", "base"]
+                 "seg_off", "seg_len", "alloc", "tables_end", "base", "rep_off", "recv_ptr",
+                 "slot_piece"]
 
 
 class WsLayout(ctypes.Structure):
@@ -67,6 +69,7 @@ _sig = {
     "moonep_plan_workspace_bytes": ([_CP], ctypes.c_size_t),
     "moonep_rank_bytes": ([_CP, _i64, ctypes.POINTER(RankBytes)], ctypes.c_int),
     "moonep_plan": ([_CP, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_plan_ex": ([_CP, ctypes.c_int32, _vp, _vp, _vp], ctypes.c_int),
     "moonep_dispatch": ([_CP, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_combine": ([_CP, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_prefetch": ([_CP, _vp, _vp, _vp, _i64, _vp], ctypes.c_int),
@@ -161,6 +164,10 @@ def moonep_plan(cfg, topk_idx, ws, stream=None) -> None:
     _check(_lib.moonep_plan(ctypes.byref(cfg_of(cfg)), _p(topk_idx), _p(ws), _stream(stream)))
 
 
+def moonep_plan_ex(cfg, flags, topk_idx, ws, stream=None) -> None:
+    _check(_lib.moonep_plan_ex(ctypes.byref(cfg_of(cfg)), int(flags), _p(topk_idx), _p(ws), _stream(stream)))
+
+
 def moonep_plan_noalloc(cfg, topk_idx, tables_out, stream=None) -> None:
     """moonep_plan without a caller workspace: the library's static device
     workspace is used and the header + tables are copied to tables_out
@@ -219,7 +226,8 @@ def moonep_plan_read(cfg, ws, tables=False, stream=None):
         sizes = dict(cnt=N, keep=N, spill=N, home_off=N, fb_cnt=N, fb_off=N, load=R, deficit=R,
                      fill=R, slots_used=R, slot_expert=R * B, slot_cnt=R * B, slot_off=R * B,
                      slot_first_j=R * B, rep_ptr=N + 1, rep_expert=P, rep_recv=P, rep_slot=P,
-                     rep_first_j=P, rep_cnt=P, rx_expert=N, route_ptr=N + 1,
+                     rep_first_j=P, rep_cnt=P, rep_off=P, recv_ptr=R + 1, slot_piece=R * B,
+                     rx_expert=N, route_ptr=N + 1,
                      route_end=2 * N + P, route_base=2 * N + P, seg_off=R * (2 * L + B),
                      seg_len=R * (2 * L + B), alloc=N * R)
         for k, n in sizes.items():
