@@ -186,17 +186,19 @@ def barrier(world):
 # ---------------------------------------------------------------------------
 
 class Runner:
-    def __init__(self, wl, maxvio, seed, with_weights=True):
+    def __init__(self, wl, maxvio, seed, with_weights=True, plan_flags=0, seed_route=None, with_grads=True):
         import torch
         from load_balancing_plan_b200 import harness
         self.torch = torch
         self.wl = wl
         self.cfg = wl.cfg()
         t0 = time.time()
-        self.route = inputs.routing(wl.R, wl.L, wl.S, wl.K, seed, maxvio=maxvio)
+        self.route = inputs.routing(wl.R, wl.L, wl.S, wl.K, seed if seed_route is None else seed_route,
+                                    maxvio=maxvio)
+        self.plan_flags = plan_flags
         self.gen_s = time.time() - t0
         we = wl.w_elems if with_weights else 0
-        ge = wl.g_elems if with_weights else 0
+        ge = wl.g_elems if with_weights and with_grads else 0
         self.prob = harness.Problem(self.cfg, w_elems=we, g_elems=ge)
         self.prob.set_routing(self.route.topk_idx, self.route.topk_w)
         self.prob.fill_x(seed)
@@ -204,6 +206,7 @@ class Runner:
         self.prob.fill_g_rep(seed)
         self.stream = torch.cuda.current_stream()
         self.with_weights = with_weights
+        self.with_grads = with_weights and with_grads
         torch.cuda.synchronize()
 
     def step(self, ev=None):
@@ -211,7 +214,7 @@ class Runner:
         s = self.stream
         if ev is not None:
             ev[0].record(s)
-        p.plan(s)
+        p.plan(s, self.plan_flags)
         if ev is not None:
             ev[1].record(s)
         if self.with_weights:
@@ -224,13 +227,15 @@ class Runner:
         p.combine(None, s)
         if ev is not None:
             ev[4].record(s)
-        if self.with_weights:
+        if self.with_grads:
             p.reduce_grad(s)
         if ev is not None:
             ev[5].record(s)
 
     def launches_per_step(self):
-        return 5 if self.with_weights and self.cfg["B"] > 0 else 3
+        if self.cfg["B"] == 0 or not self.with_weights:
+            return 3
+        return 5 if self.with_grads else 4
 
     def timed(self, steps, warmup, world=1):
         torch = self.torch
@@ -360,15 +365,24 @@ def run_gpu(args):
                                 device_id=torch.device("cuda", local_rank))
     wl = inputs.WORKLOADS[args.workload]
     target = wl.maxvio[0] if wl.maxvio else None
-    run = Runner(wl, target, seed=args.seed)
+    flags = 1 if args.plan_mode == "remote" else 0
+    if args.plan_mode == "remote":
+        # remote weights place every row below C: no headroom is needed
+        import dataclasses
+        wl = dataclasses.replace(wl, headroom=0.0)
+    # inference (no gradients): plan -> prefetch -> dispatch -> combine
+    run = Runner(wl, target, seed=args.seed, plan_flags=flags, seed_route=args.route_seed,
+                 with_grads=wl.name != "inference")
     from load_balancing_plan_b200 import moonep as mp
     info = mp.moonep_plan_read(run.cfg, run.prob.ws)   # also checks the status
     run.step()
     info = mp.moonep_plan_read(run.cfg, run.prob.ws)
     if info["status"] & mp.ST_ERROR_MASK:
         raise RuntimeError("plan failed: status 0x%x" % info["status"])
-    n_rx = len(set(np.asarray(mp.moonep_plan_read(run.cfg, run.prob.ws, tables=True)["rep_expert"]).tolist()))
-    ab = alg_bytes(run.cfg, info["n_replicas"], n_rx, run.prob.w_elems, run.prob.g_elems)
+    tabs = mp.moonep_plan_read(run.cfg, run.prob.ws, tables=True)
+    n_rx = len(set(np.asarray(tabs["rep_expert"]).tolist()))
+    n_slot = int((np.asarray(tabs["rep_slot"]) >= 0).sum())   # pieces whose weights are prefetched
+    ab = alg_bytes(run.cfg, n_slot, n_rx, run.prob.w_elems, run.prob.g_elems)
 
     total_ms, per, clocks = run.timed(args.steps, args.warmup, world)
     mean = {k: float(np.mean(v)) for k, v in per.items()}
@@ -408,10 +422,11 @@ def run_gpu(args):
                                "router bias tuned to maxvio %.2f (achieved %.3f), seed %d"
                                % (wl.name, wl.R, wl.L, wl.N, wl.S, wl.K, wl.H, wl.B, wl.C, wl.C_max,
                                   target if target is not None else -1, run.route.maxvio, args.seed),
-                   "step": "plan -> prefetch -> dispatch -> combine -> reduce_grad",
+                   "step": "plan -> prefetch -> dispatch -> combine" + (" -> reduce_grad" if run.with_grads else ""),
                    "weights_per_expert": "bf16 [%d x %d x %d]" % (wl.P, wl.H, wl.I),
                    "grads_per_expert": "fp32 [%d x %d]" % (wl.H, wl.I),
                    "accumulate": "fp32", "parallelism": "replicas%d" % world,
+                   "plan_mode": args.plan_mode,
                    "l2": "no flush: inputs larger than L2 (x %.2f GB, recv %.2f GB)"
                          % (run.prob.x.numel() * 2 / 1e9, run.prob.recv.numel() * 2 / 1e9)},
         "plan_us": round(mean["plan"] * 1e3, 2),
@@ -420,7 +435,8 @@ def run_gpu(args):
         "rows_per_s": round(rows / (max_total_ms * 1e-3), 1),
         "dispatch_combine_frac_of_peak": round(value / world / peak, 4),
         "dispatch_combine_frac_of_8tbs": round(value / world / 8000.0, 4),
-        "plan_info": {"n_replicas": info["n_replicas"], "migrated_rows": info["migrated_rows"],
+        "plan_info": {"n_replicas": info["n_replicas"], "slotted_replicas": n_slot,
+                      "migrated_rows": info["migrated_rows"],
                       "migrated_frac": round(info["migrated_rows"] / (run.prob.T * wl.K), 4),
                       "fallback_rows": info["fallback_rows"], "replicated_experts": n_rx},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
@@ -575,6 +591,10 @@ def main(argv=None):
     ap.add_argument("--workload", default="mid", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--route-seed", type=int, default=None,
+                    help="seed of the router output (default: --seed)")
+    ap.add_argument("--plan-mode", default="headroom", choices=["headroom", "remote"],
+                    help="overflow beyond a receiver's slots: headroom rows on the home rank, or remote weights")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--sweep-steps", type=int, default=20)
     ap.add_argument("--no-cpu", action="store_true")

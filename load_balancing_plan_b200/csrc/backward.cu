@@ -43,7 +43,7 @@ struct StageInfo {
 __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __grid_constant__ BackwardParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     int32_t *ws = p.ws;
-    if (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
+    if (block_status_failed(ws)) return;
     if (!cfg_matches(ws, p.cfg, num_ranges(p.T))) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;

@@ -72,7 +72,7 @@ __device__ __forceinline__ uint4 pack8(const float *acc) {
 __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_constant__ CombineParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     int32_t *ws = p.ws;
-    if (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
+    if (block_status_failed(ws)) return;
     if (!cfg_matches(ws, p.cfg, num_ranges(p.T))) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
     const int lane = threadIdx.x;
     int32_t *ws = p.ws;
     const int64_t q = blockIdx.x;
-    if (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
+    if (block_status_failed(ws)) return;
     if (!cfg_matches(ws, p.cfg, p.Q)) {
         if (lane == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;

@@ -179,6 +179,16 @@ struct CopyParams {
 #ifdef __CUDACC__
 __device__ __forceinline__ int ld_cg(const int32_t *p) { return __ldcg(p); }
 
+// Whether the workspace status holds an error bit, read once by thread 0 and
+// shared with the whole CTA: another CTA may set a bit at any moment, and the
+// threads of one CTA must take the same early exit.
+__device__ __forceinline__ bool block_status_failed(const int32_t *ws) {
+    __shared__ int s_failed;
+    if (threadIdx.x == 0) s_failed = (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) != 0;
+    __syncthreads();
+    return s_failed != 0;
+}
+
 __device__ __forceinline__ bool cfg_matches(const int32_t *ws, const moonep_cfg_t &c, int64_t Q) {
     const int32_t *h = ws + HDR_CFG;
     return __ldcg(h + 0) == c.R && __ldcg(h + 1) == c.L && __ldcg(h + 2) == c.S &&

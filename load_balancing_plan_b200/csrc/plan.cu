@@ -52,6 +52,7 @@ __device__ __forceinline__ void trace(int32_t *ws, int slot) {
 constexpr int kWarps = kPlanThreads / 32;
 constexpr int kMaxR = 64;
 constexpr int kIdBatch = 8;
+constexpr int kWarpPlannerMaxN = 512;  // above this many experts the whole CTA plans
 
 // Exclusive scan of n ints (in and out may alias) by one warp; returns the
 // total.  Lane l owns the contiguous run [l*per, (l+1)*per), per = ceil(n/32).
@@ -70,6 +71,35 @@ __device__ int warp_excl_scan(const int *in, int *out, int n) {
         run += v;
     }
     __syncwarp();
+    return total;
+}
+
+// The same by the whole CTA (kPlanThreads threads, contiguous runs of
+// ceil(n / kPlanThreads)); s_tmp holds 33 ints.
+__device__ int block_excl_scan(const int *in, int *out, int n, int *s_tmp) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (n + kPlanThreads - 1) / kPlanThreads;
+    const int lo = min(tid * per, n), hi = min(lo + per, n);
+    int sum = 0;
+    for (int i = lo; i < hi; ++i) sum += in[i];
+    const int incl = warp_incl_scan(sum);
+    if (lane == 31) s_tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < kWarps ? s_tmp[lane] : 0;
+        const int iv = warp_incl_scan(v);
+        if (lane < kWarps) s_tmp[lane] = iv - v;
+        if (lane == kWarps - 1) s_tmp[32] = iv;
+    }
+    __syncthreads();
+    int run = s_tmp[warp] + incl - sum;
+    for (int i = lo; i < hi; ++i) {
+        const int v = in[i];
+        out[i] = run;
+        run += v;
+    }
+    const int total = s_tmp[32];
+    __syncthreads();
     return total;
 }
 
@@ -141,14 +171,18 @@ __device__ void scan_column(int32_t *col, int64_t Q) {
     }
 }
 
-// The planner: one warp of CTA 0.  Every intermediate lives in shared memory
-// (seven arrays of N ints and a few of R); global memory is only written.
-// One warp needs no block-wide barriers, which dominate at these sizes.
+// The planner, run by NT threads of CTA 0: one warp (NT = 32, no block-wide
+// barriers, which dominate at a few hundred experts) or the whole CTA (NT =
+// kPlanThreads, for thousands of experts).  Every intermediate lives in
+// shared memory (seven arrays of N ints and a few of R); global memory is
+// only written.  The receiver walk is sequential and always runs on warp 0.
+template <int NT>
 __device__ void plan_tables(const PlanParams &p, int *sm) {
     const moonep_cfg_t &c = p.cfg;
     const int N = p.N, R = c.R, L = c.L, B = c.B, C = c.C, Cm = c.C_max;
     const int SEG = 2 * L + B;
-    const int lane = threadIdx.x & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = NT / 32;
     const moonep_ws_layout_t &lay = p.lay;
     int32_t *ws = p.ws;
 
@@ -160,12 +194,24 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     int *s_y = sm + 5 * N;    // chunk index, then pieces per expert -> rep_ptr
     int *s_hoff = sm + 6 * N; // row of the expert's local segment
     __shared__ int s_def[kMaxR], s_rp[kMaxR], s_rt[kMaxR], s_ri0[kMaxR], s_rnp[kMaxR], s_rpb[kMaxR], s_spb[kMaxR];
+    __shared__ int s_tmp[33];
+    __shared__ int s_misc[6];  // 0 p_end, 1 P, 2 NSLOT, 3 nrx, 4 capacity error
     const bool remote = (p.flags & MOONEP_PLAN_REMOTE_WEIGHTS) != 0;
+    auto sync = [] {
+        if (NT == 32)
+            __syncwarp();
+        else
+            __syncthreads();
+    };
+    auto scan = [&](const int *in, int *out, int n) {
+        return NT == 32 ? warp_excl_scan(in, out, n) : block_excl_scan(in, out, n, s_tmp);
+    };
 
     TRACE(ws, 3);
+    if (tid == 0) s_misc[4] = 0;
     // keep/spill: each home rank keeps rows in local-expert order up to C
-    const int total = warp_excl_scan(s_cnt, s_x, N);
-    for (int e = lane; e < N; e += 32) {
+    const int total = scan(s_cnt, s_x, N);
+    for (int e = tid; e < N; e += NT) {
         const int h = e / L;
         const int hx = s_x[e] - s_x[h * L];
         const int ce = s_cnt[e];
@@ -180,7 +226,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[lay.seg_off + h * SEG + (e - h * L)] = ho;
         ws[lay.seg_len + h * SEG + (e - h * L)] = k;
     }
-    for (int h = lane; h < R; h += 32) {
+    for (int h = tid; h < R; h += NT) {
         const int lo = s_x[h * L];
         const int hi = h + 1 < R ? s_x[(h + 1) * L] : total;
         const int ld = hi - lo;
@@ -189,76 +235,86 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[lay.deficit + h] = d;
         s_def[h] = d;
     }
-    __syncwarp();
+    sync();
 
     // the spill stream and its chunks
-    const int total_spill = warp_excl_scan(s_sp, s_x, N);  // s_x = A_e
-    const int M = warp_excl_scan(s_y, s_y, N);             // s_y = chunk index
-    for (int e = lane; e < N; e += 32)
+    const int total_spill = scan(s_sp, s_x, N);  // s_x = A_e
+    const int M = scan(s_y, s_y, N);             // s_y = chunk index
+    for (int e = tid; e < N; e += NT)
         if (s_sp[e] > 0) {
             s_ce[s_y[e]] = s_x[e] + s_sp[e];
             s_ch[s_y[e]] = e;
         }
-    __syncwarp();
+    sync();
     TRACE(ws, 4);
 
-    // receiver walk: receiver r takes the stream from p_r until its deficit
-    // is filled or (headroom rule) it has touched B chunks
-    int pos = 0, i0 = 0;
-    for (int r = 0; r < R; ++r) {
-        const int d = s_def[r];
-        int take = 0, np = 0, ir = i0;
-        const int pr = pos;
-        if (d > 0 && pos < total_spill && (remote || B > 0)) {
-            i0 = advance_chunk(s_ce, M, i0, pos);
-            const int i1 = remote ? M - 1 : min(i0 + B - 1, M - 1);
-            take = min(d, s_ce[i1] - pos);
-            const int il = advance_chunk(s_ce, M, i0, pos + take - 1);
-            np = il - i0 + 1;
-            ir = i0;
-            pos += take;
+    if (warp == 0) {
+        // receiver walk: receiver r takes the stream from p_r until its
+        // deficit is filled or (headroom rule) it has touched B chunks
+        int pos = 0, i0 = 0;
+        for (int r = 0; r < R; ++r) {
+            const int d = s_def[r];
+            int take = 0, np = 0, ir = i0;
+            const int pr = pos;
+            if (d > 0 && pos < total_spill && (remote || B > 0)) {
+                i0 = advance_chunk(s_ce, M, i0, pos);
+                const int i1 = remote ? M - 1 : min(i0 + B - 1, M - 1);
+                take = min(d, s_ce[i1] - pos);
+                const int il = advance_chunk(s_ce, M, i0, pos + take - 1);
+                np = il - i0 + 1;
+                ir = i0;
+                pos += take;
+            }
+            if (lane == 0) {
+                s_rp[r] = pr;
+                s_rt[r] = take;
+                s_ri0[r] = ir;
+                s_rnp[r] = np;
+            }
         }
+        __syncwarp();
+        // pieces per receiver -> exclusive prefix (R <= 64: two per lane), and
+        // the same for the pieces that get a slot (the first B of each receiver)
+        const int na = lane < R ? s_rnp[lane] : 0;
+        const int nb = lane + 32 < R ? s_rnp[lane + 32] : 0;
+        const int ia = warp_incl_scan(na);
+        const int tot_a = __shfl_sync(0xffffffffu, ia, 31);
+        const int ib = warp_incl_scan(nb);
+        if (lane < R) s_rpb[lane] = ia - na;
+        if (lane + 32 < R) s_rpb[lane + 32] = tot_a + ib - nb;
+        const int sa = min(na, B), sb = min(nb, B);
+        const int isa = warp_incl_scan(sa);
+        const int tot_sa = __shfl_sync(0xffffffffu, isa, 31);
+        const int isb = warp_incl_scan(sb);
+        if (lane < R) s_spb[lane] = isa - sa;
+        if (lane + 32 < R) s_spb[lane + 32] = tot_sa + isb - sb;
+        // every lane takes part in these shuffles (a full-mask shuffle must
+        // not sit under a lane-dependent branch)
+        const int P_all = tot_a + __shfl_sync(0xffffffffu, ib, 31);
+        const int nslot_all = tot_sa + __shfl_sync(0xffffffffu, isb, 31);
+        // replicated experts are the chunks that start before the walk's end
+        const int nrx = pos > 0 ? advance_chunk(s_ce, M, 0, pos - 1) + 1 : 0;
         if (lane == 0) {
-            s_rp[r] = pr;
-            s_rt[r] = take;
-            s_ri0[r] = ir;
-            s_rnp[r] = np;
+            s_misc[0] = pos;
+            s_misc[1] = P_all;
+            s_misc[2] = nslot_all;
+            s_misc[3] = nrx;
         }
     }
-    __syncwarp();
-    const int p_end = pos;
-    // pieces per receiver -> exclusive prefix (R <= 64: two per lane), and
-    // the same for the pieces that get a slot (the first B of each receiver)
-    const int na = lane < R ? s_rnp[lane] : 0;
-    const int nb = lane + 32 < R ? s_rnp[lane + 32] : 0;
-    const int ia = warp_incl_scan(na);
-    const int tot_a = __shfl_sync(0xffffffffu, ia, 31);
-    const int ib = warp_incl_scan(nb);
-    if (lane < R) s_rpb[lane] = ia - na;
-    if (lane + 32 < R) s_rpb[lane + 32] = tot_a + ib - nb;
-    const int P = tot_a + __shfl_sync(0xffffffffu, ib, 31);
-    const int sa = min(na, B), sb = min(nb, B);
-    const int isa = warp_incl_scan(sa);
-    const int tot_sa = __shfl_sync(0xffffffffu, isa, 31);
-    const int isb = warp_incl_scan(sb);
-    if (lane < R) s_spb[lane] = isa - sa;
-    if (lane + 32 < R) s_spb[lane + 32] = tot_sa + isb - sb;
-    const int NSLOT = tot_sa + __shfl_sync(0xffffffffu, isb, 31);
-    // replicated experts are the chunks that start before the walk's end
-    const int nrx = p_end > 0 ? advance_chunk(s_ce, M, 0, p_end - 1) + 1 : 0;
-    for (int e = lane; e < N; e += 32) s_y[e] = 0;  // pieces per expert
-    for (int r = lane; r < R; r += 32) {
+    for (int e = tid; e < N; e += NT) s_y[e] = 0;  // pieces per expert
+    sync();
+    const int p_end = s_misc[0], P = s_misc[1], NSLOT = s_misc[2], nrx = s_misc[3];
+    for (int r = tid; r < R; r += NT) {
         ws[lay.fill + r] = C - s_def[r] + s_rt[r];
         ws[lay.slots_used + r] = min(s_rnp[r], B);
         ws[lay.recv_ptr + r] = s_rpb[r];
     }
-    if (lane == 0) ws[lay.recv_ptr + R] = P;
-    __syncwarp();
+    if (tid == 0) ws[lay.recv_ptr + R] = P;
     TRACE(ws, 5);
 
-    // pieces (receiver by receiver), their slots and slot segments, route
+    // pieces (a warp per receiver), their slots and slot segments, route
     // entries and alloc entries
-    for (int r = 0; r < R; ++r) {
+    for (int r = warp; r < R; r += NW) {
         const int npr = s_rnp[r];
         for (int b = lane; b < npr; b += 32) {
             const int i = s_ri0[r] + b;
@@ -295,7 +351,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         }
     }
     // slots no piece took
-    for (int idx = lane; idx < R * B; idx += 32) {
+    for (int idx = tid; idx < R * B; idx += NT) {
         const int r = idx / B, b = idx - r * B;
         if (b < s_rnp[r]) continue;
         const int sg = r * SEG + L + b;
@@ -307,9 +363,9 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[lay.seg_off + sg] = fill;
         ws[lay.seg_len + sg] = 0;
     }
-    for (int x = lane; x < nrx; x += 32) ws[lay.rx_expert + x] = s_ch[x];
+    for (int x = tid; x < nrx; x += NT) ws[lay.rx_expert + x] = s_ch[x];
     // fallback rows: the stream beyond the walk's end, per chunk (s_x: A_e -> fb_cnt)
-    for (int e = lane; e < N; e += 32) {
+    for (int e = tid; e < N; e += NT) {
         int fb = 0;
         if (s_sp[e] > 0) {
             const int cs = s_x[e], ce = cs + s_sp[e];
@@ -318,12 +374,12 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         s_x[e] = fb;
         ws[lay.fb_cnt + e] = fb;
     }
-    __syncwarp();
+    sync();
     TRACE(ws, 6);
-    warp_excl_scan(s_y, s_y, N);   // s_y = rep_ptr
-    warp_excl_scan(s_x, s_ce, N);  // s_ce = exclusive prefix of fb_cnt
+    scan(s_y, s_y, N);   // s_y = rep_ptr
+    scan(s_x, s_ce, N);  // s_ce = exclusive prefix of fb_cnt
     int cap_err = 0;
-    for (int e = lane; e < N; e += 32) {
+    for (int e = tid; e < N; e += NT) {
         const int h = e / L;
         const int fbo = C + (s_ce[e] - s_ce[h * L]);
         const int fb = s_x[e];
@@ -343,13 +399,14 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[lay.alloc + (int64_t)e * R + h] = keep + fb;
         if ((e % L) == L - 1 && fbo + fb > Cm) cap_err = 1;
     }
-    cap_err = __any_sync(0xffffffffu, cap_err);
-    if (lane == 0) {
+    if (cap_err) s_misc[4] = 1;
+    sync();
+    if (tid == 0) {
         ws[lay.rep_ptr + N] = P;
         ws[lay.route_ptr + N] = 2 * N + P;
         const int fallback = total_spill - p_end;
         int st = 0;
-        if (cap_err) st |= MOONEP_ST_CAPACITY;
+        if (s_misc[4]) st |= MOONEP_ST_CAPACITY;
         if (fallback > 0) st |= MOONEP_ST_FALLBACK;
         ws[HDR_FALLBACK] = fallback;
         ws[HDR_NREP] = P;
@@ -408,6 +465,11 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
         __syncthreads();
     }
     if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_EXPERT_ID);
+    // the allocation table is only written after the barrier: clear it now,
+    // spread over the whole grid
+    for (int64_t i = (int64_t)blockIdx.x * kPlanThreads + tid; i < (int64_t)N * p.cfg.R;
+         i += (int64_t)gridDim.x * kPlanThreads)
+        ws[lay.alloc + i] = 0;
     if (blockIdx.x == 0) TRACE(ws, 1);
     if (blockIdx.x == 0 && tid < 8) ws[HDR_CFG + tid] = (&p.cfg.R)[tid];
     if (blockIdx.x == 0 && tid == 0) ws[HDR_NRANGES] = (int32_t)p.Q;
@@ -418,19 +480,21 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
         return;
     }
     if (blockIdx.x == 0) TRACE(ws, 2);
-    const int st = __ldcg(ws + HDR_STATUS);
-    if (st & MOONEP_ST_ERROR_MASK) return;
+    if (block_status_failed(ws)) return;
 
     // phase B: column prefixes on CTAs 1.. (or all on CTA 0 if alone); CTA 0
-    // loads cnt and clears alloc with all its threads, then warp 0 plans
+    // loads cnt with all its threads, then plans (one warp, or all warps for
+    // more than kWarpPlannerMaxN experts)
     const int warp = tid >> 5;
     if (gridDim.x == 1)
         for (int e = warp; e < N; e += kWarps) scan_column(ws + lay.base + (int64_t)e * p.Q, p.Q);
     if (blockIdx.x == 0) {
         for (int e = tid; e < N; e += kPlanThreads) sm[e] = __ldcg(ws + lay.cnt + e);
-        for (int64_t i = tid; i < (int64_t)N * p.cfg.R; i += kPlanThreads) ws[lay.alloc + i] = 0;
         __syncthreads();
-        if (warp == 0) plan_tables(p, sm);
+        if (N > kWarpPlannerMaxN)
+            plan_tables<kPlanThreads>(p, sm);
+        else if (warp == 0)
+            plan_tables<32>(p, sm);
     } else {
         const int gw = (blockIdx.x - 1) * kWarps + warp;
         const int nw = (gridDim.x - 1) * kWarps;

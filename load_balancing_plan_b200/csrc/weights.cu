@@ -43,7 +43,7 @@ static_assert(kPfStages - kPfAhead - 1 >= 0, "stage reuse needs an older store g
 __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__ CopyParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     int32_t *ws = p.ws;
-    if (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
+    if (block_status_failed(ws)) return;
     if (!cfg_matches(ws, p.cfg, p.lay.n_ranges)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
@@ -128,7 +128,7 @@ __device__ __forceinline__ void add4(float4 &a, const float4 &b) {
 // expert and the experts' different replica counts even out.
 __global__ void __launch_bounds__(kThreads) reduce_grad_kernel(const __grid_constant__ CopyParams p) {
     int32_t *ws = p.ws;
-    if (__ldcg(ws + HDR_STATUS) & MOONEP_ST_ERROR_MASK) return;
+    if (block_status_failed(ws)) return;
     if (!cfg_matches(ws, p.cfg, p.lay.n_ranges)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
