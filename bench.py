@@ -237,10 +237,62 @@ class Runner:
             return 3
         return 5 if self.with_grads else 4
 
-    def timed(self, steps, warmup, world=1):
+    def timed(self, steps, warmup, world=1, graph=True):
+        """Times `steps` steps after `warmup` untimed ones.  With graph=True
+        the step is captured into a CUDA graph of G steps (timing events
+        included) and replayed: the timed region replays it steps/G times
+        back to back between two events (no host launch latency can show),
+        and a second pass of replays, each read back, gives every kernel's
+        duration from the events inside the graph.  Returns (total_ms,
+        per-kernel lists, clocks, launch mode)."""
         torch = self.torch
+        names = ["plan", "prefetch", "dispatch", "combine", "reduce_grad"]
         for _ in range(warmup):
             self.step()
+        torch.cuda.synchronize()
+        G = 10 if steps % 10 == 0 else 1
+        g = None
+        keep = self.stream
+        if graph:
+            try:
+                cap = torch.cuda.Stream()
+                cap.wait_stream(self.stream)
+                evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)] for _ in range(G)]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    self.stream = cap
+                    for i in range(G):
+                        self.step(evs[i])
+                self.stream = keep
+                torch.cuda.synchronize()
+                g.replay()
+                torch.cuda.synchronize()
+            except Exception as exc:  # capture not available: launch eagerly
+                self.stream = keep
+                g = None
+                print("bench: CUDA graph capture failed (%s); timing eager launches" % exc, file=sys.stderr)
+                torch.cuda.synchronize()
+        if g is not None:
+            barrier(world)
+            torch.cuda.synchronize()
+            with ClockSampler(torch.cuda.current_device()) as clk:
+                start = torch.cuda.Event(enable_timing=True)
+                end = torch.cuda.Event(enable_timing=True)
+                start.record(self.stream)
+                for _ in range(steps // G):
+                    g.replay()
+                end.record(self.stream)
+                torch.cuda.synchronize()
+            barrier(world)
+            total_ms = start.elapsed_time(end)
+            per = {n: [] for n in names}
+            for _ in range(steps // G):
+                g.replay()
+                torch.cuda.synchronize()
+                for i in range(G):
+                    for j, n in enumerate(names):
+                        per[n].append(evs[i][j].elapsed_time(evs[i][j + 1]))
+            return total_ms, per, clk.summary(), "cuda_graph_%d_steps" % G
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
         barrier(world)
         torch.cuda.synchronize()
@@ -254,9 +306,8 @@ class Runner:
             torch.cuda.synchronize()
         barrier(world)
         total_ms = start.elapsed_time(end)
-        names = ["plan", "prefetch", "dispatch", "combine", "reduce_grad"]
         per = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)] for j, n in enumerate(names)}
-        return total_ms, per, clk.summary()
+        return total_ms, per, clk.summary(), "eager"
 
     def backward(self, steps, warmup):
         """The training backward pair on the same plan: combine_backward
@@ -384,7 +435,7 @@ def run_gpu(args):
     n_slot = int((np.asarray(tabs["rep_slot"]) >= 0).sum())   # pieces whose weights are prefetched
     ab = alg_bytes(run.cfg, n_slot, n_rx, run.prob.w_elems, run.prob.g_elems)
 
-    total_ms, per, clocks = run.timed(args.steps, args.warmup, world)
+    total_ms, per, clocks, launch_mode = run.timed(args.steps, args.warmup, world, graph=not args.eager)
     mean = {k: float(np.mean(v)) for k, v in per.items()}
     dc_ms = sum(per["dispatch"]) + sum(per["combine"])
     max_dc_ms, dc_bytes = reduce_over_ranks(dc_ms, (ab["dispatch"] + ab["combine"]) * args.steps, world)
@@ -426,7 +477,7 @@ def run_gpu(args):
                    "weights_per_expert": "bf16 [%d x %d x %d]" % (wl.P, wl.H, wl.I),
                    "grads_per_expert": "fp32 [%d x %d]" % (wl.H, wl.I),
                    "accumulate": "fp32", "parallelism": "replicas%d" % world,
-                   "plan_mode": args.plan_mode,
+                   "plan_mode": args.plan_mode, "launch": launch_mode,
                    "l2": "no flush: inputs larger than L2 (x %.2f GB, recv %.2f GB)"
                          % (run.prob.x.numel() * 2 / 1e9, run.prob.recv.numel() * 2 / 1e9)},
         "plan_us": round(mean["plan"] * 1e3, 2),
@@ -469,7 +520,7 @@ def run_sweep(args, peak):
     res = {}
     for mv in wl.maxvio:
         run = Runner(wl, mv, seed=0, with_weights=False)
-        total_ms, per, _ = run.timed(args.sweep_steps, 3)
+        total_ms, per, _, _ = run.timed(args.sweep_steps, 3, graph=not args.eager)
         from load_balancing_plan_b200 import moonep as mp
         info = mp.moonep_plan_read(run.cfg, run.prob.ws)
         ab = alg_bytes(run.cfg)
@@ -596,6 +647,7 @@ def main(argv=None):
     ap.add_argument("--plan-mode", default="headroom", choices=["headroom", "remote"],
                     help="overflow beyond a receiver's slots: headroom rows on the home rank, or remote weights")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="launch every step from the host (no CUDA graph)")
     ap.add_argument("--sweep-steps", type=int, default=20)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,

@@ -68,7 +68,8 @@ int device_info(int N, DeviceInfo **out) {
     // plan kernel: shared memory depends on N
     const size_t smem = plan_smem_bytes(N);
     if (smem != d.plan_smem) {
-        e = cudaFuncSetAttribute(plan_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        static std::atomic<size_t> plan_smem_set[64];
+        e = set_smem_limit(plan_kernel_ptr(), smem, plan_smem_set);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(plan)");
         int nb = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, plan_kernel_ptr(), 512, smem);

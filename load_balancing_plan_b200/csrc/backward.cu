@@ -262,8 +262,8 @@ cudaError_t combine_backward_config(int K, int hv, bool with_grad_w, uint32_t *c
 }
 
 cudaError_t launch_combine_backward(const BackwardParams &p, int grid, size_t smem, cudaStream_t s) {
-    cudaError_t err =
-        cudaFuncSetAttribute(combine_backward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<size_t> smem_set[64];
+    cudaError_t err = set_smem_limit((const void *)combine_backward_kernel, smem, smem_set);
     if (err != cudaSuccess) return err;
     combine_backward_kernel<<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();

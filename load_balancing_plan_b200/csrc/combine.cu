@@ -229,7 +229,8 @@ cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages
 }
 
 cudaError_t launch_combine(const CombineParams &p, int grid, size_t smem, cudaStream_t s) {
-    cudaError_t err = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<size_t> smem_set[64];
+    cudaError_t err = set_smem_limit((const void *)combine_kernel, smem, smem_set);
     if (err != cudaSuccess) return err;
     combine_kernel<<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();

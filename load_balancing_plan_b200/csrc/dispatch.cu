@@ -225,7 +225,8 @@ cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uin
 }
 
 cudaError_t launch_dispatch(const DispatchParams &p, size_t smem, cudaStream_t s) {
-    cudaError_t err = cudaFuncSetAttribute(dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<size_t> smem_set[64];
+    cudaError_t err = set_smem_limit((const void *)dispatch_kernel, smem, smem_set);
     if (err != cudaSuccess) return err;
     dispatch_kernel<<<(unsigned)p.Q, 32, smem, s>>>(p);
     return cudaGetLastError();

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "moonep.h"
 
 namespace moonep {
@@ -313,6 +315,34 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 }
 #endif
 
+}  // namespace moonep
+
+namespace moonep {
+// Raises a kernel's dynamic shared-memory limit on the current device only
+// when a launch needs more than was set before, so steady-state launches make
+// no attribute call (`cache` holds one entry per device).
+//
+// MOONEP_CARVEOUT (percent of the unified L1/shared storage given to shared
+// memory, -1 = the driver's choice) is requested for every kernel alike, so
+// consecutive kernels of a step never make the SM change its split.
+#ifndef MOONEP_CARVEOUT
+#define MOONEP_CARVEOUT -1
+#endif
+inline cudaError_t set_smem_limit(const void *func, size_t smem, std::atomic<size_t> *cache) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const size_t want = smem > 0 ? smem : 1;
+    if (cache[dev].load(std::memory_order_relaxed) >= want) return cudaSuccess;
+    if (MOONEP_CARVEOUT >= 0) {
+        e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, MOONEP_CARVEOUT);
+        if (e != cudaSuccess) return e;
+    }
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) cache[dev].store(want, std::memory_order_relaxed);
+    return e;
+}
 }  // namespace moonep
 
 // launchers (defined in the kernel files, called by the C ABI layer)

@@ -200,13 +200,17 @@ __global__ void __launch_bounds__(kThreads) reduce_grad_kernel(const __grid_cons
 
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s) {
     const size_t smem = (size_t)kPfStages * kPfChunk + kPfStages * 8;
-    cudaError_t err = cudaFuncSetAttribute(prefetch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<size_t> smem_set[64];
+    cudaError_t err = set_smem_limit((const void *)prefetch_kernel, smem, smem_set);
     if (err != cudaSuccess) return err;
     prefetch_kernel<<<grid, 32, smem, s>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_grad(const CopyParams &p, int grid, cudaStream_t s) {
+    static std::atomic<size_t> smem_set[64];
+    cudaError_t err = set_smem_limit((const void *)reduce_grad_kernel, 0, smem_set);
+    if (err != cudaSuccess) return err;
     reduce_grad_kernel<<<grid, kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
