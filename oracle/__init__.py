@@ -99,13 +99,14 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
-MODE_HEADROOM, MODE_REMOTE = 0, 1
+MODE_HEADROOM, MODE_REMOTE, MODE_ONE_GROUP = 0, 1, 2
 
 
 def plan(cfg: dict, topk_idx: np.ndarray, mode: int = MODE_HEADROOM) -> dict:
     """Run the plan on int32 topk_idx [R, S, K]; returns every table plus the
     header counts as a dict of numpy arrays / ints.  mode 1: remote weights
-    (pieces beyond a receiver's B slots read their expert remotely)."""
+    (pieces beyond a receiver's B slots read their expert remotely); mode 2:
+    a receiver takes replicas of one home group only."""
     lib = _load()
     R, L, S, K, B = (int(cfg[n]) for n in "RLSKB")
     N = R * L

@@ -75,7 +75,13 @@ static int64_t or_min64(int64_t a, int64_t b) { return a < b ? a : b; }
  * paragraphs; "The Busiest Rank Sets Your Step Time", "Installation and
  * integration"): a receiver takes spilled rows while it has room whatever its
  * slots; its first B pieces get slots, later ones are remote (slot -1), so no
- * row ever falls back and every rank holds exactly C rows. */
+ * row ever falls back and every rank holds exactly C rows.
+ * mode 2, one home group per receiver ("The Busiest Rank Sets Your Step
+ * Time", section "Installation and integration", the paragraph on B after
+ * the weight-tensor figure: a rank duplicates experts of at most one remote
+ * home group, which is why B = E/R slots always suffice): the headroom rule
+ * with one more condition on the receiver -- once it holds a piece of an
+ * expert of home group h, it takes rows of group h only. */
 int or_plan_ex(const or_cfg *c, int mode, const int32_t *topk_idx, or_plan_t *p)
 {
     const int R = c->R, L = c->L, B = c->B;
@@ -136,6 +142,8 @@ int or_plan_ex(const or_cfg *c, int mode, const int32_t *topk_idx, or_plan_t *p)
     }
     int npieces = 0;
     int32_t *on_r = (int32_t *)calloc((size_t)(R > 0 ? R : 1), sizeof(int32_t)); /* pieces per receiver */
+    int32_t *lock = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R > 0 ? R : 1)); /* mode 2: home group */
+    for (int r = 0; r < R; ++r) lock[r] = -1;
     for (int e = 0; e < N; ++e) {
         p->rep_ptr[e] = npieces;
         int64_t a = p->spill[e];
@@ -143,14 +151,16 @@ int or_plan_ex(const or_cfg *c, int mode, const int32_t *topk_idx, or_plan_t *p)
         while (a > 0) {
             int r = -1;
             for (int q = 0; q < R; ++q)
-                if (def[q] > 0 && (mode == 1 || p->slots_used[q] < B)) {
+                if (def[q] > 0 && (mode == 1 || p->slots_used[q] < B) &&
+                    (mode != 2 || lock[q] < 0 || lock[q] == e / L)) {
                     r = q;
                     break;
                 }
             if (r < 0) break;
             int64_t t = or_min64(a, def[r]);
-            int b = on_r[r] < B ? on_r[r] : -1;   /* mode 0 always has a free slot here */
+            int b = on_r[r] < B ? on_r[r] : -1;   /* modes 0 and 2 always have a free slot here */
             on_r[r]++;
+            lock[r] = e / L;
             if (b >= 0) p->slots_used[r]++;
             p->rep_expert[npieces] = e;
             p->rep_recv[npieces] = r;
@@ -175,6 +185,7 @@ int or_plan_ex(const or_cfg *c, int mode, const int32_t *topk_idx, or_plan_t *p)
     p->n_replicas = npieces;
     free(def);
     free(on_r);
+    free(lock);
 
     /* O5: layout of rank r: kept local segments, then slots in slot order,
      * then (from row C) the fallback segments of r's own experts. */
@@ -267,8 +278,10 @@ int or_plan(const or_cfg *c, const int32_t *topk_idx, or_plan_t *p) { return or_
 /* Places overflow rows one by one: a row goes home while the home rank has */
 /* room; else to the receiver of the expert's current piece while that      */
 /* receiver has room; else to the lowest rank with room and a free slot,    */
-/* opening a new slot.  Offsets are assigned only after every row has a     */
-/* place.  Outputs: alloc, slot_expert, slot_cnt, fb_cnt, dest, status.     */
+/* opening a new slot (mode 2: and, once it holds a piece, whose pieces are */
+/* all of this row's home group).  Offsets are assigned only after every row */
+/* has a place.  Outputs: alloc, slot_expert, slot_cnt, fb_cnt, dest,       */
+/* status.                                                                   */
 /* ------------------------------------------------------------------------ */
 int or_plan_unitwise_ex(const or_cfg *c, int mode, const int32_t *topk_idx, int32_t *alloc,
                         int32_t *slot_expert, int32_t *slot_cnt, int32_t *fb_cnt, int32_t *dest,
@@ -297,6 +310,8 @@ int or_plan_unitwise_ex(const or_cfg *c, int mode, const int32_t *topk_idx, int3
     int *pidx = (int *)malloc(sizeof(int) * (size_t)(G > 0 ? G : 1));
     int64_t *rows = (int64_t *)calloc((size_t)R, sizeof(int64_t)); /* rows in [0,C) */
     int *npc_r = (int *)calloc((size_t)R, sizeof(int));            /* pieces per receiver */
+    int *grp_r = (int *)malloc(sizeof(int) * (size_t)(R > 0 ? R : 1)); /* home group of its pieces */
+    for (int r = 0; r < R; ++r) grp_r[r] = -1;
     int maxp = (int)(N + R + 1);
     int *pc_rank = (int *)malloc(sizeof(int) * (size_t)maxp);
     int *pc_slot = (int *)malloc(sizeof(int) * (size_t)maxp);
@@ -325,13 +340,15 @@ int or_plan_unitwise_ex(const or_cfg *c, int mode, const int32_t *topk_idx, int3
             }
             int pick = -1;
             for (int r = 0; r < R; ++r)
-                if (rows[r] < C && (mode == 1 || npc_r[r] < B)) { pick = r; break; }
+                if (rows[r] < C && (mode == 1 || npc_r[r] < B) &&
+                    (mode != 2 || grp_r[r] < 0 || grp_r[r] == e / L)) { pick = r; break; }
             if (pick >= 0) {
                 cur = np++;
                 pc_rank[cur] = pick;
                 pc_slot[cur] = npc_r[pick] < B ? npc_r[pick] : -1;
                 pc_exp[cur] = e;
                 npc_r[pick]++;
+                grp_r[pick] = e / L;
                 kind[q] = 1; pidx[q] = cur; pc_n[cur] = 1; rows[pick]++;
             } else {
                 cur = -1;
@@ -383,7 +400,7 @@ int or_plan_unitwise_ex(const or_cfg *c, int mode, const int32_t *topk_idx, int3
     int64_t fb_total = 0;
     for (int e = 0; e < N; ++e) fb_total += fb_cnt[e];
     if (fb_total > 0) status |= OR_ST_FALLBACK;
-    free(count); free(order); free(fillpos); free(kind); free(pidx); free(rows); free(npc_r);
+    free(count); free(order); free(fillpos); free(kind); free(pidx); free(rows); free(npc_r); free(grp_r);
     free(pc_rank); free(pc_slot); free(pc_exp); free(pc_n); free(home_base); free(home_n);
     free(pc_base); free(fb_base); free(pc_used);
     *status_out = status;
