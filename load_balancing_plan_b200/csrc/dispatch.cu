@@ -28,6 +28,9 @@ namespace {
 #ifndef MOONEP_DISPATCH_LOOKAHEAD
 #define MOONEP_DISPATCH_LOOKAHEAD 6  // loads issued ahead of the stores
 #endif
+#ifndef MOONEP_DISPATCH_LOADER
+#define MOONEP_DISPATCH_LOADER 0     // 1: loader warps fetch x with plain loads; TMA only stores
+#endif
 #ifndef MOONEP_DISPATCH_HINTS
 #define MOONEP_DISPATCH_HINTS 1      // bit 0: evict-first on the x loads, bit 1: on the row stores
 #endif
@@ -198,6 +201,127 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
     }
 }
 
+// The same dispatch with the x rows fetched by kLoaderWarps loader warps
+// with ordinary 16-byte loads (registers, then shared memory, a proxy fence
+// and an mbarrier arrive), so the SM's TMA unit carries only the row stores.
+// Warp 0 numbers the copies and issues the K bulk stores of each unit; once
+// the store group of unit j - kRelease has read its stage, it hands that stage
+// back on the stage's "empty" mbarrier.  Shared memory: stages, kStages "full"
+// then kStages "empty" barriers, ring, counters.
+#ifndef MOONEP_DISPATCH_LOADER_WARPS
+#define MOONEP_DISPATCH_LOADER_WARPS 2
+#endif
+constexpr int kLoaderWarps = MOONEP_DISPATCH_LOADER_WARPS;
+constexpr int kVec = 16;       // 16-byte vectors per lane per pass (8 KB per warp)
+constexpr int kRelease = 2;    // store groups left reading their stages
+static_assert(kRelease >= 1 && kRelease < kStages, "a stage is handed back before its next load needs it");
+
+__global__ void __launch_bounds__(32 * (1 + kLoaderWarps), 1)
+    dispatch_loader_kernel(const __grid_constant__ DispatchParams p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int32_t *ws = p.ws;
+    const int64_t q = blockIdx.x;
+    if (block_status_failed(ws)) return;
+    if (!cfg_matches(ws, p.cfg, p.Q)) {
+        if (threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
+        return;
+    }
+    Smem sm;
+    sm.stages = smem_raw;
+    sm.bars = reinterpret_cast<uint64_t *>(smem_raw + (size_t)kStages * p.piece_bytes);
+    uint64_t *empty = sm.bars + kStages;
+    sm.ring = reinterpret_cast<int32_t *>(empty + kStages);
+    sm.ctr = sm.ring + kRing;
+    const int K = p.cfg.K, npc = p.npc;
+    for (int e = threadIdx.x; e < p.N; e += blockDim.x) sm.ctr[e] = __ldg(ws + p.lay.base + (int64_t)e * p.Q + q);
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kStages; ++st) {
+            mbar_init(&sm.bars[st], 1);
+            mbar_init(&empty[st], 1);
+        }
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+
+    const int64_t t0 = range_begin(q, p.T, p.Q), t1 = range_begin(q + 1, p.T, p.Q);
+    const int64_t ntok = t1 - t0;
+    const int64_t g0 = t0 * K, nids = ntok * K;
+    const int64_t nunits = ntok * npc;
+    const uint32_t last_piece = p.row_bytes - (uint32_t)(npc - 1) * p.piece_bytes;
+
+    if (warp > 0) {
+        // ------------------------------------------------------ loaders
+        for (int64_t u = warp - 1; u < nunits; u += kLoaderWarps) {
+            const int st = (int)(u % kStages);
+            int ok = 1;
+            if (lane == 0 && u >= kStages)
+                ok = mbar_wait_bounded(&empty[st], (uint32_t)(((u / kStages) - 1) & 1), p.wait_limit);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                if (lane == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
+                break;
+            }
+            const int64_t i = u / npc;
+            const int pc = (int)(u - i * npc);
+            const uint32_t bytes = pc == npc - 1 ? last_piece : p.piece_bytes;
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (t0 + i) * (int64_t)p.row_bytes +
+                                                               (int64_t)pc * p.piece_bytes);
+            uint4 *dst = reinterpret_cast<uint4 *>(sm.stages + (size_t)st * p.piece_bytes);
+            const int nv = (int)(bytes >> 4);
+            for (int v0 = 0; v0 < nv; v0 += 32 * kVec) {
+                uint4 v[kVec];
+#pragma unroll
+                for (int k = 0; k < kVec; ++k)
+                    if (v0 + lane + 32 * k < nv) v[k] = __ldcs(src + v0 + lane + 32 * k);
+#pragma unroll
+                for (int k = 0; k < kVec; ++k)
+                    if (v0 + lane + 32 * k < nv) dst[v0 + lane + 32 * k] = v[k];
+            }
+            fence_proxy_async_smem();  // these generic-proxy writes before the bulk stores read them
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.bars[st]);
+        }
+        return;
+    }
+    // ---------------------------------------------------------- warp 0
+    int64_t nranked = 0;
+    bool bad = false, fail = false;
+    for (int64_t j = 0; j < nunits; ++j) {
+        const int64_t i = j / npc;
+        while (nranked < (i + 1) * K) {
+            bad |= rank_group(p, sm, g0, nranked, nids);
+            nranked = min(nranked + 32, nids);
+        }
+        if (lane == 0) {
+            const int st = (int)(j % kStages);
+            if (!mbar_wait_bounded(&sm.bars[st], (uint32_t)((j / kStages) & 1), p.wait_limit)) {
+                fail = true;
+            } else {
+                const int pc = (int)(j - i * npc);
+                const uint32_t bytes = pc == npc - 1 ? last_piece : p.piece_bytes;
+                const uint8_t *src = sm.stages + (size_t)st * p.piece_bytes;
+                for (int k = 0; k < K; ++k) {
+                    const int d = sm.ring[(i * K + k) % kRing];
+                    if (d >= 0)
+                        bulk_s2g_plain(p.recv + (int64_t)d * p.row_bytes + (int64_t)pc * p.piece_bytes, src, bytes);
+                }
+                bulk_commit();
+                bulk_wait_read<kRelease>();
+                if (j >= kRelease) mbar_arrive(&empty[(j - kRelease) % kStages]);
+            }
+        }
+        fail = __shfl_sync(0xffffffffu, (int)fail, 0) != 0;
+        if (fail) break;
+    }
+    if (lane == 0) {
+        bulk_wait_all<0>();
+        if (fail) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
+        if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_DEST);
+    }
+}
+
 }  // namespace
 
 // Shared memory: kStages pieces + barriers + ring + N counters, sized so that
@@ -225,6 +349,14 @@ cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uin
 }
 
 cudaError_t launch_dispatch(const DispatchParams &p, size_t smem, cudaStream_t s) {
+    if (MOONEP_DISPATCH_LOADER) {
+        static std::atomic<size_t> smem_set2[64];
+        const size_t smem2 = smem + (size_t)kStages * 8;  // the "empty" barriers
+        cudaError_t err = set_smem_limit((const void *)dispatch_loader_kernel, smem2, smem_set2);
+        if (err != cudaSuccess) return err;
+        dispatch_loader_kernel<<<(unsigned)p.Q, 32 * (1 + kLoaderWarps), smem2, s>>>(p);
+        return cudaGetLastError();
+    }
     static std::atomic<size_t> smem_set[64];
     cudaError_t err = set_smem_limit((const void *)dispatch_kernel, smem, smem_set);
     if (err != cudaSuccess) return err;
