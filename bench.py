@@ -416,11 +416,16 @@ def run_gpu(args):
                                 device_id=torch.device("cuda", local_rank))
     wl = inputs.WORKLOADS[args.workload]
     target = wl.maxvio[0] if wl.maxvio else None
-    flags = 1 if args.plan_mode == "remote" else 0
+    from load_balancing_plan_b200 import moonep as mp
+    flags = {"headroom": 0, "remote": mp.PLAN_REMOTE_WEIGHTS, "one_group": mp.PLAN_ONE_GROUP}[args.plan_mode]
     if args.plan_mode == "remote":
         # remote weights place every row below C: no headroom is needed
         import dataclasses
         wl = dataclasses.replace(wl, headroom=0.0)
+    elif args.plan_mode == "one_group":
+        # receivers locked to one home group leave rows on their home ranks
+        import dataclasses
+        wl = dataclasses.replace(wl, headroom=max(wl.headroom, 1.0))
     # inference (no gradients): plan -> prefetch -> dispatch -> combine
     run = Runner(wl, target, seed=args.seed, plan_flags=flags, seed_route=args.route_seed,
                  with_grads=wl.name != "inference")
@@ -644,8 +649,9 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--route-seed", type=int, default=None,
                     help="seed of the router output (default: --seed)")
-    ap.add_argument("--plan-mode", default="headroom", choices=["headroom", "remote"],
-                    help="overflow beyond a receiver's slots: headroom rows on the home rank, or remote weights")
+    ap.add_argument("--plan-mode", default="headroom", choices=["headroom", "remote", "one_group"],
+                    help="overflow beyond a receiver's slots: headroom rows on the home rank, or remote "
+                         "weights; one_group: receivers take replicas of one home group only")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every step from the host (no CUDA graph)")
     ap.add_argument("--sweep-steps", type=int, default=20)

@@ -181,6 +181,7 @@ MOONEP_API int moonep_plan(const moonep_cfg_t *cfg, const int32_t *topk_idx, voi
 
 /* Plan flags for moonep_plan_ex. */
 #define MOONEP_PLAN_REMOTE_WEIGHTS 0x1
+#define MOONEP_PLAN_ONE_GROUP 0x2
 
 /* moonep_plan with flags.  MOONEP_PLAN_REMOTE_WEIGHTS selects the pages'
  * inference fallback instead of the headroom rule: when a receiver would need
@@ -193,7 +194,16 @@ MOONEP_API int moonep_plan(const moonep_cfg_t *cfg, const int32_t *topk_idx, voi
  * rep_off[p] .. rep_off[p] + rep_cnt[p]).  No row falls back: every rank
  * holds exactly C rows and C_max = C suffices.  prefetch copies slotted pieces
  * only, reduce_grad reduces slotted pieces only (remote pieces carry no
- * gradient slot: the mode is for inference).  flags = 0 is moonep_plan. */
+ * gradient slot: the mode is for inference).
+ * MOONEP_PLAN_ONE_GROUP keeps the headroom rule and adds the pages' planner
+ * variant in which a rank duplicates experts of at most one remote home group
+ * ("The Busiest Rank Sets Your Step Time", "Installation and integration",
+ * the paragraph on B after the weight-tensor figure): a receiver stops at the
+ * end of the home group its first piece comes from, so it never holds pieces
+ * of more than L = E/R experts and B = L slots always suffice.  The price is
+ * balance: rows that no receiver may take fall back to their home rank's
+ * headroom (rows from C), so C_max must leave room for them.  The two flags
+ * exclude each other (MOONEP_ERR_ARG).  flags = 0 is moonep_plan. */
 MOONEP_API int moonep_plan_ex(const moonep_cfg_t *cfg, int32_t flags, const int32_t *topk_idx, void *ws,
                               void *stream);
 

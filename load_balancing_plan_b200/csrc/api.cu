@@ -173,7 +173,10 @@ int moonep_plan(const moonep_cfg_t *cfg, const int32_t *topk_idx, void *ws, void
 
 int moonep_plan_ex(const moonep_cfg_t *cfg, int32_t flags, const int32_t *topk_idx, void *ws, void *stream) {
     TRY(check_cfg(cfg));
-    if (flags & ~MOONEP_PLAN_REMOTE_WEIGHTS) return fail(MOONEP_ERR_ARG, "unknown plan flags 0x%x", flags);
+    if (flags & ~(MOONEP_PLAN_REMOTE_WEIGHTS | MOONEP_PLAN_ONE_GROUP))
+        return fail(MOONEP_ERR_ARG, "unknown plan flags 0x%x", flags);
+    if ((flags & MOONEP_PLAN_REMOTE_WEIGHTS) && (flags & MOONEP_PLAN_ONE_GROUP))
+        return fail(MOONEP_ERR_ARG, "plan flags 0x%x: remote weights and one group exclude each other", flags);
     const int64_t T = (int64_t)cfg->R * cfg->S;
     TRY(check_ptr(topk_idx, 4, "topk_idx", T > 0));
     TRY(check_ptr(ws, 16, "ws", true));

@@ -26,7 +26,10 @@
 // (one slot per chunk it touches).  That is exactly "each chunk goes to the
 // lowest-index rank that still has room and a free slot", computed as a walk
 // over at most R receivers instead of over the chunks.  Rows past the last
-// receiver's stop fall back to their home rank's headroom.
+// receiver's stop fall back to their home rank's headroom.  Plan flags: with
+// MOONEP_PLAN_REMOTE_WEIGHTS the B limit is dropped (pieces past a receiver's
+// B-th read their weights remotely); with MOONEP_PLAN_ONE_GROUP a receiver
+// also stops where the stream leaves its first chunk's home group.
 #include "moonep_internal.cuh"
 
 namespace moonep {
@@ -197,6 +200,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     __shared__ int s_tmp[33];
     __shared__ int s_misc[6];  // 0 p_end, 1 P, 2 NSLOT, 3 nrx, 4 capacity error
     const bool remote = (p.flags & MOONEP_PLAN_REMOTE_WEIGHTS) != 0;
+    const bool one_group = (p.flags & MOONEP_PLAN_ONE_GROUP) != 0;
     auto sync = [] {
         if (NT == 32)
             __syncwarp();
@@ -250,7 +254,8 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
 
     if (warp == 0) {
         // receiver walk: receiver r takes the stream from p_r until its
-        // deficit is filled or (headroom rule) it has touched B chunks
+        // deficit is filled or (headroom rule) it has touched B chunks or
+        // (one-group rule) the stream leaves its first chunk's home group
         int pos = 0, i0 = 0;
         for (int r = 0; r < R; ++r) {
             const int d = s_def[r];
@@ -258,7 +263,14 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
             const int pr = pos;
             if (d > 0 && pos < total_spill && (remote || B > 0)) {
                 i0 = advance_chunk(s_ce, M, i0, pos);
-                const int i1 = remote ? M - 1 : min(i0 + B - 1, M - 1);
+                int i1 = remote ? M - 1 : min(i0 + B - 1, M - 1);
+                if (one_group) {
+                    // stop at the last chunk of the first chunk's home group
+                    // (chunk experts ascend, so it is one before the first
+                    // chunk of an expert of a later group)
+                    const int h = s_ch[i0] / L;
+                    i1 = min(i1, advance_chunk(s_ch, M, i0, (h + 1) * L - 1) - 1);
+                }
                 take = min(d, s_ce[i1] - pos);
                 const int il = advance_chunk(s_ce, M, i0, pos + take - 1);
                 np = il - i0 + 1;

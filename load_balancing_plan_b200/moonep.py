@@ -25,6 +25,7 @@ ST_EXPERT_ID, ST_CAPACITY, ST_TIMEOUT, ST_DEST, ST_CFG = 0x1, 0x2, 0x4, 0x8, 0x1
 ST_ERROR_MASK, ST_FALLBACK = 0xFF, 0x100
 WS_HEADER_WORDS = 64
 PLAN_REMOTE_WEIGHTS = 0x1
+PLAN_ONE_GROUP = 0x2
 
 
 class MoonepError(RuntimeError):

@@ -129,3 +129,11 @@ def test_rank_bytes_match_memory_table(mp):
             assert round(rb["reduce_bytes"] / gib, 2) == pytest.approx(red, abs=0.006)
             total += rb["reduce_bytes"]
         assert round(total / gib, 2) == pytest.approx(tot, abs=0.006)
+
+
+def test_plan_flags_checked_before_any_cuda_call(mp):
+    c = _cfg()
+    for flags in (0x4, -1, mp.PLAN_REMOTE_WEIGHTS | mp.PLAN_ONE_GROUP):
+        with pytest.raises(mp.MoonepError) as ei:
+            mp.moonep_plan_ex(c, flags, 16, 256, stream=0)
+        assert ei.value.code == mp.ERR_ARG

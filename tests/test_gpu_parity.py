@@ -55,7 +55,8 @@ def x_host(seed, T, H):
     return inputs.cb_bf16_np(seed, inputs.STREAM_X, np.arange(T * H, dtype=np.int64)).reshape(T, H)
 
 
-def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_seed=0, remote=False):
+def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_seed=0, remote=False,
+                     one_group=False):
     """Every step on a small problem, compared element by element."""
     torch, mp, harness = env
     R, L, S, K, H, B, Cm = (cfg[n] for n in ("R", "L", "S", "K", "H", "B", "C_max"))
@@ -65,9 +66,10 @@ def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_see
     prob.fill_x(seed)
     prob.fill_weights(seed)
     prob.fill_g_rep(seed)
-    prob.plan(flags=mp.PLAN_REMOTE_WEIGHTS if remote else 0)
+    prob.plan(flags=mp.PLAN_REMOTE_WEIGHTS if remote else mp.PLAN_ONE_GROUP if one_group else 0)
     gpl = prob.read_plan()
-    opl = oracle.plan(cfg, ids, mode=oracle.MODE_REMOTE if remote else oracle.MODE_HEADROOM)
+    mode = oracle.MODE_REMOTE if remote else oracle.MODE_ONE_GROUP if one_group else oracle.MODE_HEADROOM
+    opl = oracle.plan(cfg, ids, mode=mode)
     compare_plan(gpl, opl)
     failed = bool(opl["status"] & (oracle.ST_CAPACITY | oracle.ST_EXPERT_ID))
     if not failed:
@@ -514,3 +516,131 @@ def test_remote_weights_inference_workload(env):
     assert np.array_equal(rows, want)
     # with C_max = C and no fallback every receive row is used
     assert not np.any(np.all(harness.to_u16(prob.recv[::97]) == 0xFFFF, axis=1))
+
+
+# ---------------------------------------------------------------------------
+# several layers through one set of buffers
+# ---------------------------------------------------------------------------
+
+def test_layers_share_buffers(env):
+    # a model runs its MoE layers one after another through the same per-rank
+    # buffers (workspace, receive rows, replica weight slots, replica
+    # gradients); the slots a layer fills differ from the last layer's, and
+    # the plan mode may change between layers.  Every layer matches the
+    # oracle run on the oracle's own carried-over buffers.
+    torch, mp, harness = env
+    cfg = cfg_of(8, 6, 96, 4, 64, 3, headroom=0.25)
+    R, L, S, K, H, B, Cm = (cfg[n] for n in ("R", "L", "S", "K", "H", "B", "C_max"))
+    N, T, E = R * L, R * S, 512
+    prob = harness.Problem(cfg, poison=True, w_elems=E, g_elems=E)
+    recv_o = np.full((R * Cm, H), 0xFFFF, np.uint16)
+    wslot_o = np.full((R * B, E), 0xFFFF, np.uint16)
+    layers = [(11, 1.5, False), (12, 6.0, True), (13, 3.0, False), (14, 0.0, False)]
+    seen_slots = []
+    for layer, (seed, maxvio, remote) in enumerate(layers):
+        r = inputs.routing(R, L, S, K, seed, maxvio=maxvio)
+        prob.set_routing(r.topk_idx, r.topk_w)
+        prob.fill_x(seed)
+        prob.fill_weights(seed)
+        prob.fill_g_rep(seed)
+        mode = oracle.MODE_REMOTE if remote else oracle.MODE_HEADROOM
+        prob.plan(flags=mp.PLAN_REMOTE_WEIGHTS if remote else 0)
+        opl = oracle.plan(cfg, r.topk_idx, mode=mode)
+        assert opl["status"] & 0xFF == 0
+        compare_plan(prob.read_plan(), opl)
+        seen_slots.append(tuple(opl["slot_expert"].tolist()))
+        # forward: prefetch, dispatch, stand-in expert, combine
+        prob.prefetch()
+        prob.dispatch()
+        torch.cuda.synchronize()
+        oracle.prefetch(cfg, opl["slot_expert"], harness.to_u16(prob.w_home), wslot_o, E)
+        assert np.array_equal(harness.to_u16(prob.w_slot), wslot_o), layer
+        oracle.dispatch(cfg, opl["dest"], x_host(seed, T, H), recv_o)
+        assert np.array_equal(harness.to_u16(prob.recv), recv_o), layer
+        scale = inputs.expert_scales(N, seed)
+        y_g = prob.expert_scale(scale)
+        y_o = recv_o.copy()
+        oracle.expert_scale(cfg, opl, recv_o, scale, y_o)
+        prob.combine(y_g)
+        torch.cuda.synchronize()
+        out_o, _ = oracle.combine(cfg, opl["dest"], y_o, r.topk_w)
+        assert np.array_equal(harness.to_u16(prob.out[:T]), out_o), layer
+        # backward: replica gradients back to their home experts
+        gh = prob.g_home.cpu().numpy().copy()
+        gr = prob.g_rep.cpu().numpy().copy()
+        prob.reduce_grad()
+        torch.cuda.synchronize()
+        oracle.reduce_grad(cfg, opl, gh, gr, E)
+        assert np.array_equal(prob.g_home.cpu().numpy().view(np.uint32), gh.view(np.uint32)), layer
+        assert np.array_equal(prob.g_rep.cpu().numpy().view(np.uint32), gr.view(np.uint32)), layer
+    # the layers really used different slot assignments
+    assert len(set(seen_slots)) == len(layers)
+
+
+# ---------------------------------------------------------------------------
+# one-home-group plan mode (the pages' planner variant)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", [
+    # R, L, S, K, H, B, headroom
+    (3, 1, 2, 1, 16, 2, 1.0),       # two senders, one receiver: a row falls back
+    (8, 4, 64, 4, 64, 4, 1.0),      # B = E/R
+    (8, 8, 128, 8, 64, 2, 1.0),     # fewer slots than L: both limits bind
+    (16, 24, 64, 8, 32, 24, 1.0),   # many groups, long spill stream
+])
+def test_one_group_mode(env, case):
+    R, L, S, K, H, B, hr = case
+    cfg = cfg_of(R, L, S, K, H, B, headroom=hr)
+    for seed in range(3):
+        r = inputs.routing(R, L, S, K, seed, maxvio=min(4.0, R - 1.0))
+        prob, gpl, opl = run_full_compare(env, cfg, r.topk_idx, r.topk_w, seed=seed, one_group=True)
+        n = opl["n_replicas"]
+        groups = [set((opl["rep_expert"][:n][opl["rep_recv"][:n] == q] // L).tolist()) for q in range(R)]
+        assert all(len(g) <= 1 for g in groups)
+
+
+def test_one_group_worked_example(env):
+    # experts 0 and 1 three rows each, expert 2 none (R=3, L=1, C=2): the
+    # receiver takes expert 0's spilled row; expert 1's stays on rank 1 at row C
+    torch, mp, harness = env
+    cfg = cfg_of(3, 1, 2, 1, 16, 2, headroom=1.0)
+    ids = pc.ids_from_counts(np.array([3, 3, 0]), 3, 2, 1)
+    w = np.ones((3, 2, 1), np.float32)
+    prob, gpl, opl = run_full_compare(env, cfg, ids, w, one_group=True)
+    assert prob.dest[:6].cpu().tolist() == [0, 1, 8, 4, 5, 6]
+    assert gpl["fallback_rows"] == 1
+
+
+def test_one_group_mid_workload(env):
+    # the mid workload's routing under the one-group rule: the plan, every
+    # destination and sampled rows against the oracle
+    torch, mp, harness = env
+    wl = inputs.WORKLOADS["mid"]
+    cfg = dict(wl.cfg(), C_max=2 * wl.C)
+    r = inputs.routing(wl.R, wl.L, wl.S, wl.K, 1, maxvio=wl.maxvio[0])
+    prob = harness.Problem(cfg)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.fill_x(1)
+    prob.plan(flags=mp.PLAN_ONE_GROUP)
+    prob.dispatch()
+    torch.cuda.synchronize()
+    opl = oracle.plan(cfg, r.topk_idx, mode=oracle.MODE_ONE_GROUP)
+    compare_plan(prob.read_plan(), opl)
+    assert opl["fallback_rows"] > 0
+    dest = prob.dest[:wl.T * wl.K].cpu().numpy()
+    assert np.array_equal(dest, opl["dest"].reshape(-1))
+    rng = np.random.default_rng(3)
+    g = np.sort(rng.choice(wl.T * wl.K, 256, replace=False))
+    t = g // wl.K
+    xs = inputs.cb_bf16_np(1, inputs.STREAM_X, t[:, None] * wl.H + np.arange(wl.H)[None, :])
+    got = harness.to_u16(prob.recv[torch.from_numpy(dest[g]).long().cuda()])
+    assert np.array_equal(got, xs)
+
+
+def test_plan_flags_exclude_each_other(env):
+    torch, mp, harness = env
+    w = inputs.WORKLOADS["tiny"]
+    prob = harness.Problem(w.cfg())
+    with pytest.raises(mp.MoonepError) as ei:
+        prob.plan(flags=mp.PLAN_REMOTE_WEIGHTS | mp.PLAN_ONE_GROUP)
+    assert ei.value.code == mp.ERR_ARG
