@@ -75,6 +75,8 @@ def _load():
         lib.or_plan_unitwise_ex.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, vp, vp, vp, vp, vp, vp, vp]
         lib.or_plan_unitwise_ex.restype = ctypes.c_int
         lib.or_dispatch.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, ctypes.c_int64]
+        lib.or_copy_out.argtypes = [ctypes.POINTER(_Cfg), vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, vp]
+        lib.or_copy_out.restype = ctypes.c_int64
         lib.or_expert_scale.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, vp, ctypes.c_int,
                                         vp, vp, vp, vp, vp]
         lib.or_combine.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp, ctypes.c_int64]
@@ -161,6 +163,19 @@ def dispatch(cfg: dict, dest: np.ndarray, x: np.ndarray, recv: np.ndarray, n_tok
     assert x.dtype == np.uint16 and recv.dtype == np.uint16
     lib.or_dispatch(ctypes.byref(_cfg(cfg)), _ptr(d), _ptr(x), _ptr(recv), n)
     return recv
+
+
+def copy_out(cfg: dict, pl: dict, recv: np.ndarray, out: np.ndarray) -> int:
+    """Copy the rows the plan uses from recv to out (both uint16 [R*C_max, H]);
+    returns the number of rows copied."""
+    lib = _load()
+    assert recv.dtype == np.uint16 and out.dtype == np.uint16
+    n = int(pl["n_replicas"])
+    reps = [np.ascontiguousarray(pl[k][:n], dtype=np.int32) if n else np.zeros(1, np.int32)
+            for k in ("rep_recv", "rep_slot", "rep_off", "rep_cnt")]
+    return int(lib.or_copy_out(ctypes.byref(_cfg(cfg)), _ptr(np.ascontiguousarray(pl["seg_off"], np.int32)),
+                               _ptr(np.ascontiguousarray(pl["seg_len"], np.int32)), n,
+                               *(_ptr(a) for a in reps), _ptr(recv), _ptr(out)))
 
 
 def expert_scale(cfg: dict, pl: dict, recv: np.ndarray, scale: np.ndarray, y: np.ndarray):

@@ -448,6 +448,40 @@ void or_dispatch(const or_cfg *c, const int32_t *dest, const uint16_t *x, uint16
         }
 }
 
+/* O7b copy-out (zero_copy = false): the rows the plan put in the receive
+ * buffer -- every segment of every rank (local, slot, fallback) and every
+ * remote piece -- copied bitwise to the same rows of a buffer of the
+ * caller's; other rows of `out` are left alone.  The application normally
+ * works on views of the communication buffer, which the next dispatch or
+ * combine overwrites; a caller that keeps rows beyond that (autograd, for
+ * one) asks for zero_copy = false and gets its own copy ("MoonEP balances AI
+ * experts in MoE models", twodots.gr: the paragraph on zero-copy
+ * communication and static shapes, and the one on the lifetime of zero-copy
+ * views).  Returns the number of rows copied. */
+int64_t or_copy_out(const or_cfg *c, const int32_t *seg_off, const int32_t *seg_len, int n_rep,
+                    const int32_t *rep_recv, const int32_t *rep_slot, const int32_t *rep_off,
+                    const int32_t *rep_cnt, const uint16_t *recv, uint16_t *out)
+{
+    const int64_t H = c->H, Cm = c->C_max;
+    const int SEG = 2 * c->L + c->B;
+    int64_t rows = 0;
+    for (int r = 0; r < c->R; ++r) {
+        for (int s = 0; s < SEG; ++s) {
+            int64_t row0 = (int64_t)r * Cm + seg_off[r * SEG + s];
+            int64_t n = seg_len[r * SEG + s];
+            memcpy(out + row0 * H, recv + row0 * H, (size_t)(n * H * 2));
+            rows += n;
+        }
+    }
+    for (int q = 0; q < n_rep; ++q)
+        if (rep_slot[q] < 0) {
+            int64_t row0 = (int64_t)rep_recv[q] * Cm + rep_off[q];
+            memcpy(out + row0 * H, recv + row0 * H, (size_t)((int64_t)rep_cnt[q] * H * 2));
+            rows += rep_cnt[q];
+        }
+    return rows;
+}
+
 /* O8 stand-in expert: y[row] = bf16(float(recv[row]) * scale[expert(row)]),
  * one fp32 multiply; expert(row) from the segment tables. */
 static void or_scale_rows(const or_cfg *c, int64_t row0, int64_t n, int e, const uint16_t *recv,

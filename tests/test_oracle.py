@@ -471,3 +471,29 @@ def test_remote_pieces_carry_no_replica_gradient(oracle_lib):
     used = np.zeros(R * B, bool)
     used[slots] = True
     assert np.all(gr[used] == 0) and np.array_equal(gr[~used], r0[~used])
+
+
+# ---------------------------------------------------------------------------
+# copy-out (zero_copy = false): the rows in use, and only those
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode_name,seed", [("MODE_HEADROOM", 0), ("MODE_HEADROOM", 3), ("MODE_REMOTE", 1),
+                                            ("MODE_ONE_GROUP", 2)])
+def test_copy_out_copies_exactly_the_rows_in_use(oracle_lib, mode_name, seed):
+    # against the row -> expert map built from the plan's segment and piece
+    # tables with numpy: rows with an expert are copied, the rest untouched
+    R, L, S, K, H, B = 6, 3, 40, 4, 24, 2
+    cfg = _cfg(R, L, S, K, H, B, C_max=2 * S * K)
+    rng = np.random.default_rng(seed)
+    cnt = pc.random_counts(rng, R * L, R * S, K, skew=1.5)
+    ids = pc.ids_from_counts(cnt, R, S, K)
+    pl = oracle_lib.plan(cfg, ids, mode=getattr(oracle_lib, mode_name))
+    assert pl["status"] & 0xFF == 0
+    rows = R * cfg["C_max"]
+    recv = inputs.cb_bf16_np(seed, inputs.STREAM_X, np.arange(rows * H)).reshape(rows, H)
+    out = np.full((rows, H), 0xBEEF, np.uint16)
+    n = oracle_lib.copy_out(cfg, pl, recv, out)
+    used = pc.row_expert_map(cfg, pl) >= 0
+    assert n == used.sum() == R * S * K
+    assert np.array_equal(out[used], recv[used])
+    assert np.all(out[~used] == 0xBEEF)
