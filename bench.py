@@ -313,7 +313,10 @@ class Runner:
         """The training backward pair on the same plan: combine_backward
         (grad_y and grad_w) and dispatch_backward, each timed alone with CUDA
         events; the output gradient is the hidden states and the expert
-        outputs are the dispatched rows (values do not change the work)."""
+        outputs are the dispatched rows (values do not change the work).
+        Also times copy_out (zero_copy = false) of the dispatched rows.  The
+        gradient buffer doubles as copy_out's target (it is rewritten by each
+        combine_backward anyway)."""
         torch = self.torch
         from load_balancing_plan_b200 import moonep as mp
         p, cfg, s = self.prob, self.cfg, self.stream
@@ -323,9 +326,13 @@ class Runner:
         grad_x = torch.empty_like(p.out)
         cb = lambda: mp.moonep_combine_backward(cfg, p.ws, p.x, p.recv, p.dest, p.w, grad_y, grad_w, s)
         db = lambda: mp.moonep_dispatch_backward(cfg, p.ws, p.recv, p.dest, grad_x, s)
+        # zero_copy = false: the dispatched rows (T*K of them) copied out
+        kept = grad_y
+        co = lambda: mp.moonep_copy_out(cfg, p.ws, p.recv, kept, s)
         res = {}
         for name, fn, nbytes in (("combine_backward", cb, T * 2 * H + 2 * T * K * 2 * H + 12 * T * K),
-                                 ("dispatch_backward", db, T * K * 2 * H + T * 2 * H + 4 * T * K)):
+                                 ("dispatch_backward", db, T * K * 2 * H + T * 2 * H + 4 * T * K),
+                                 ("copy_out", co, 2 * T * K * 2 * H)):
             for _ in range(warmup):
                 fn()
             a = torch.cuda.Event(enable_timing=True)
@@ -505,6 +512,7 @@ def run_gpu(args):
         "gpu_launches": run.launches_per_step() * args.steps,
         "clocks": clocks,
     }
+    out["copy_out"] = bwd.pop("copy_out")
     out["backward"] = bwd
     if sweep is not None:
         out["sweep"] = sweep

@@ -215,6 +215,26 @@ MOONEP_API int moonep_plan_ex(const moonep_cfg_t *cfg, int32_t flags, const int3
 MOONEP_API int moonep_dispatch(const moonep_cfg_t *cfg, void *ws, const void *x, const int32_t *topk_idx,
                     void *recv, int32_t *dest, void *stream);
 
+/* Copy-out, the zero_copy = false path (twodots.gr "MoonEP balances AI
+ * experts in MoE models": the application works on views of the
+ * communication buffer, which the next dispatch or combine overwrites, so a
+ * caller that keeps the rows longer -- autograd saving them for the backward
+ * pass, for one -- needs zero_copy = false, i.e. a copy of its own).
+ * recv: device bf16 [R][C_max][H] after moonep_dispatch with this plan; out:
+ * device bf16 [R][C_max][H] owned by the caller, not overlapping recv
+ * (MOONEP_ERR_ARG).  Copies every row the plan uses -- on rank r the rows
+ * [0, fill[r]) and the fallback segments of r's experts from row C -- to the
+ * same row of out, bitwise; other rows of out are not written, so the plan's
+ * segment tables index out as they index recv.  Both pointers 16-byte
+ * aligned.  Status bits as for dispatch (a failed plan: nothing written). */
+MOONEP_API int moonep_copy_out(const moonep_cfg_t *cfg, void *ws, const void *recv, void *out, void *stream);
+
+/* Generation of the zero-copy views tied to a workspace: the number of
+ * moonep_dispatch and moonep_combine calls launched with `ws` so far in this
+ * process (host-side count; no GPU work, never fails; 0 for an unknown ws).
+ * A view taken at generation g is stale once the generation moves past g. */
+MOONEP_API int64_t moonep_view_generation(const void *ws);
+
 /* Combine (same flowchart: combine gathers results back into token order).
  * y: device bf16 [R][C_max][H] expert outputs in the dispatched layout;
  * dest: from moonep_dispatch; topk_w: device fp32 [R][S][K] router weights;

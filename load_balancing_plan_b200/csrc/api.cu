@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <unordered_map>
 
 #include "moonep_internal.cuh"
 
@@ -43,6 +44,15 @@ struct DeviceInfo {
 
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
+
+// zero-copy view generations: dispatch and combine launches per workspace
+std::mutex g_gen_mu;
+std::unordered_map<const void *, int64_t> g_gen;
+
+void bump_generation(const void *ws) {
+    std::lock_guard<std::mutex> lk(g_gen_mu);
+    ++g_gen[ws];
+}
 
 // Checks the current device once (sm_100, cooperative launch) and caches
 // launch sizes that depend on it.
@@ -234,6 +244,7 @@ int moonep_dispatch(const moonep_cfg_t *cfg, void *ws, const void *x, const int3
     p.wait_limit = g_wait_limit.load();
     e = launch_dispatch(p, smem, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "dispatch kernel launch");
+    bump_generation(ws);
     return MOONEP_OK;
 }
 
@@ -271,6 +282,7 @@ static int combine_impl(const moonep_cfg_t *cfg, void *ws, const void *y, const 
     if (grid < 1) grid = 1;
     cudaError_t e = launch_combine(p, (int)grid, smem, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+    if (weighted) bump_generation(ws);
     return MOONEP_OK;
 }
 
@@ -323,6 +335,40 @@ int moonep_combine_backward(const moonep_cfg_t *cfg, void *ws, const void *grad_
     cudaError_t e = launch_combine_backward(p, (int)grid, smem, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "combine_backward kernel launch");
     return MOONEP_OK;
+}
+
+int moonep_copy_out(const moonep_cfg_t *cfg, void *ws, const void *recv, void *out, void *stream) {
+    TRY(check_cfg(cfg));
+    const int64_t rows = (int64_t)cfg->R * cfg->C_max;
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(recv, 16, "recv", rows > 0));
+    TRY(check_ptr(out, 16, "out", rows > 0));
+    const int64_t bytes = rows * cfg->H * 2;
+    const char *a = (const char *)recv, *b = (const char *)out;
+    if (rows > 0 && a < b + bytes && b < a + bytes) return fail(MOONEP_ERR_ARG, "copy_out: recv and out overlap");
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (rows == 0 || (int64_t)cfg->R * cfg->S == 0) return MOONEP_OK;
+    CopyOutParams p{};
+    p.cfg = *cfg;
+    compute_layout(*cfg, p.lay);
+    p.Q = p.lay.n_ranges;
+    p.row_vecs = cfg->H / 8;
+    p.src = (const uint4 *)recv;
+    p.dst = (uint4 *)out;
+    p.ws = (int32_t *)ws;
+    // the CTAs one wave holds (6 of 256 threads per SM), shared by the R fill runs
+    int per_rank = (int)((6 * (int64_t)d->sms + cfg->R - 1) / cfg->R);
+    if (per_rank < 1) per_rank = 1;
+    cudaError_t e = launch_copy_out(p, per_rank, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "copy_out kernel launch");
+    return MOONEP_OK;
+}
+
+int64_t moonep_view_generation(const void *ws) {
+    std::lock_guard<std::mutex> lk(g_gen_mu);
+    auto it = g_gen.find(ws);
+    return it == g_gen.end() ? 0 : it->second;
 }
 
 int moonep_prefetch(const moonep_cfg_t *cfg, void *ws, const void *w_home, void *w_slot, int64_t elems_per_expert,

@@ -5,16 +5,20 @@
 // writes there, so no receive-buffer-to-compute-buffer copy exists;
 // agentlenshq "MoonshotAI/MoonEP", "How it works": fused permute).
 //
-// One CTA of one warp per token range (the ranges the plan counted).  The
-// warp numbers the range's copies in ascending g: for each group of 32 ids it
+// One CTA per token range (the ranges the plan counted; two per SM).  Warp 0
+// numbers the range's copies in ascending g: for each group of 32 ids it
 // finds equal experts with __match_any_sync, ranks lanes within a group by
 // popcount, and adds a per-expert running counter kept in shared memory
 // (initialised from the plan's per-range prefix), which gives the copy index
 // j of every (token, k); j maps to a flat row through the expert's route
-// entries.  Lane 0 then moves the data with TMA bulk copies: each row piece
-// of x is loaded once into a shared-memory stage (mbarrier completion) and
-// stored K times straight to its destination rows (bulk async-groups), with
-// kLookahead loads in flight ahead of the stores.  Numbering runs just ahead
+// entries.  The data moves through shared-memory stages, one row piece each:
+// a loader warp fills a stage from x with 16-byte loads (then a proxy fence
+// and an mbarrier arrive), and lane 0 of warp 0 stores the piece K times
+// straight to its destination rows with TMA bulk copies (bulk async-groups),
+// handing the stage back on an mbarrier once the group has read it.  Keeping
+// the x loads off the TMA unit lets them overlap the row stores instead of
+// queueing behind them (about 4% faster than the same pipeline with TMA
+// loads, which MOONEP_DISPATCH_LOADER=0 builds).  Numbering runs just ahead
 // of the copies, so its cost hides under them.  No multicast.
 #include "moonep_internal.cuh"
 
@@ -29,7 +33,7 @@ namespace {
 #define MOONEP_DISPATCH_LOOKAHEAD 6  // loads issued ahead of the stores
 #endif
 #ifndef MOONEP_DISPATCH_LOADER
-#define MOONEP_DISPATCH_LOADER 0     // 1: loader warps fetch x with plain loads; TMA only stores
+#define MOONEP_DISPATCH_LOADER 1     // 1: a loader warp fetches x with plain loads, TMA only stores; 0: TMA loads too
 #endif
 #ifndef MOONEP_DISPATCH_HINTS
 #define MOONEP_DISPATCH_HINTS 1      // bit 0: evict-first on the x loads, bit 1: on the row stores
@@ -209,11 +213,14 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
 // back on the stage's "empty" mbarrier.  Shared memory: stages, kStages "full"
 // then kStages "empty" barriers, ring, counters.
 #ifndef MOONEP_DISPATCH_LOADER_WARPS
-#define MOONEP_DISPATCH_LOADER_WARPS 2
+#define MOONEP_DISPATCH_LOADER_WARPS 1
 #endif
 constexpr int kLoaderWarps = MOONEP_DISPATCH_LOADER_WARPS;
 constexpr int kVec = 16;       // 16-byte vectors per lane per pass (8 KB per warp)
-constexpr int kRelease = 2;    // store groups left reading their stages
+#ifndef MOONEP_DISPATCH_RELEASE
+#define MOONEP_DISPATCH_RELEASE 2
+#endif
+constexpr int kRelease = MOONEP_DISPATCH_RELEASE;  // store groups left reading their stages
 static_assert(kRelease >= 1 && kRelease < kStages, "a stage is handed back before its next load needs it");
 
 __global__ void __launch_bounds__(32 * (1 + kLoaderWarps), 1)
@@ -304,8 +311,12 @@ __global__ void __launch_bounds__(32 * (1 + kLoaderWarps), 1)
                 const uint8_t *src = sm.stages + (size_t)st * p.piece_bytes;
                 for (int k = 0; k < K; ++k) {
                     const int d = sm.ring[(i * K + k) % kRing];
-                    if (d >= 0)
-                        bulk_s2g_plain(p.recv + (int64_t)d * p.row_bytes + (int64_t)pc * p.piece_bytes, src, bytes);
+                    if (d < 0) continue;
+                    uint8_t *dst = p.recv + (int64_t)d * p.row_bytes + (int64_t)pc * p.piece_bytes;
+                    if (MOONEP_DISPATCH_HINTS & 2)
+                        bulk_s2g(dst, src, bytes, policy_evict_first());
+                    else
+                        bulk_s2g_plain(dst, src, bytes);
                 }
                 bulk_commit();
                 bulk_wait_read<kRelease>();

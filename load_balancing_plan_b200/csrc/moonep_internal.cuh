@@ -175,6 +175,17 @@ struct CopyParams {
     moonep_ws_layout_t lay;
 };
 
+struct CopyOutParams {
+    moonep_cfg_t cfg;
+    int64_t Q;            // token ranges of the plan (workspace check)
+    int64_t row_vecs;     // 16-byte vectors per row
+    const uint4 *src;     // receive buffer [R, C_max, H]
+    uint4 *dst;           // the caller's copy, same shape
+    int32_t *ws;
+    moonep_ws_layout_t lay;
+};
+constexpr int kCopyOutThreads = 256;
+
 // ---------------------------------------------------------------------------
 // device helpers
 // ---------------------------------------------------------------------------
@@ -359,6 +370,7 @@ const void *combine_kernel_ptr();
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s);
 cudaError_t launch_reduce_grad(const CopyParams &p, int grid, cudaStream_t s);
 int set_error(int code, const char *msg);
+cudaError_t launch_copy_out(const CopyOutParams &p, int blocks_per_rank, cudaStream_t s);
 cudaError_t launch_combine_backward(const BackwardParams &p, int grid, size_t smem, cudaStream_t s);
 cudaError_t combine_backward_config(int K, int hv, bool with_grad_w, uint32_t *chunk, int *upt, int *stages,
                                     size_t *smem);

@@ -79,6 +79,8 @@ _sig = {
     "moonep_plan_noalloc": ([_CP, _vp, _vp, _vp], ctypes.c_int),
     "moonep_combine_backward": ([_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_dispatch_backward": ([_CP, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_copy_out": ([_CP, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_view_generation": ([_vp], _i64),
     "moonep_set_wait_limit": ([_i64], ctypes.c_int),
     "moonep_num_ranges": ([_i64], _i64),
     "moonep_last_error": ([], ctypes.c_char_p),
@@ -180,6 +182,14 @@ def moonep_plan_noalloc(cfg, topk_idx, tables_out, stream=None) -> None:
 def moonep_dispatch(cfg, ws, x, topk_idx, recv, dest, stream=None) -> None:
     _check(_lib.moonep_dispatch(ctypes.byref(cfg_of(cfg)), _p(ws), _p(x), _p(topk_idx), _p(recv),
                                 _p(dest), _stream(stream)))
+
+
+def moonep_copy_out(cfg, ws, recv, out, stream=None) -> None:
+    _check(_lib.moonep_copy_out(ctypes.byref(cfg_of(cfg)), _p(ws), _p(recv), _p(out), _stream(stream)))
+
+
+def moonep_view_generation(ws) -> int:
+    return int(_lib.moonep_view_generation(_p(ws)))
 
 
 def moonep_combine(cfg, ws, y, dest, topk_w, out, stream=None) -> None:

@@ -137,3 +137,18 @@ def test_plan_flags_checked_before_any_cuda_call(mp):
         with pytest.raises(mp.MoonepError) as ei:
             mp.moonep_plan_ex(c, flags, 16, 256, stream=0)
         assert ei.value.code == mp.ERR_ARG
+
+
+def test_copy_out_arguments_checked_before_any_cuda_call(mp):
+    c = _cfg()
+    rows_bytes = c["R"] * c["C_max"] * c["H"] * 2
+    for args in [(None, 256, 1 << 40), (256, 264, 1 << 40), (256, 1 << 40, 8),
+                 (256, 4096, 4096 + rows_bytes - 16), (256, 4096 + 16, 4096)]:   # misaligned, overlapping
+        with pytest.raises(mp.MoonepError) as ei:
+            mp.moonep_copy_out(c, *args, stream=0)
+        assert ei.value.code == mp.ERR_ARG
+
+
+def test_view_generation_of_unknown_workspace_is_zero(mp):
+    assert mp.moonep_view_generation(0x1000) == 0
+    assert mp.moonep_view_generation(None) == 0

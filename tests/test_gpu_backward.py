@@ -79,6 +79,7 @@ def test_tiny(env, seed):
     (8, 8, 40, 64, 16, 8, 0.0),      # K at its maximum: several k batches
     (2, 2, 300, 2, 20008, 2, 1.0),   # long rows
     (1, 7, 500, 1, 8, 2, 0.0),
+    (2, 2, 4, 2, 1 << 20, 2, 1.0),   # H at its maximum (2 MB rows)
 ])
 def test_edge_cases(env, case):
     R, L, S, K, H, B, hr = case

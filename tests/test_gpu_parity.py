@@ -80,9 +80,13 @@ def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_see
     recv_g = harness.to_u16(prob.recv)
     dest_g = prob.dest[:T * K].cpu().numpy()
     if failed:
-        # a failed plan: dispatch writes nothing
+        # a failed plan: dispatch and copy-out write nothing
         assert np.all(recv_g == 0xFFFF)
         assert np.all(dest_g == -7)
+        out_c = torch.full_like(prob.recv, 0x1357)
+        mp.moonep_copy_out(cfg, prob.ws, prob.recv, out_c)
+        torch.cuda.synchronize()
+        assert np.all(harness.to_u16(out_c) == 0x1357)
         return prob, gpl, opl
     assert np.array_equal(dest_g, opl["dest"].reshape(-1))
     xh = x_host(seed, T, H)
@@ -90,6 +94,14 @@ def run_full_compare(env, cfg, ids, w, seed=0, w_elems=64, g_elems=64, scale_see
     recv_o = np.full((R * Cm, H), 0xFFFF, np.uint16)
     oracle.dispatch(cfg, opl["dest"], xh, recv_o)
     assert np.array_equal(recv_g, recv_o)
+
+    # zero_copy = false: the rows in use copied out, the rest untouched
+    out_c = torch.full_like(prob.recv, 0x1357)
+    mp.moonep_copy_out(cfg, prob.ws, prob.recv, out_c)
+    torch.cuda.synchronize()
+    out_co = np.full((R * Cm, H), 0x1357, np.uint16)
+    assert oracle.copy_out(cfg, opl, recv_o, out_co) == T * K
+    assert np.array_equal(harness.to_u16(out_c), out_co)
 
     # stand-in expert, then combine, against the oracle's chain
     scale = inputs.expert_scales(N, scale_seed)
@@ -170,6 +182,7 @@ def test_tiny_reduce_grad_full_size_grads(env):
     (2, 2, 300, 2, 20008, 2, 1.0, "skew"),              # rows split in several pieces
     (64, 64, 32, 8, 32, 8, 0.0, "skew"),                # N at its maximum
     (5, 3, 1000, 4, 40, 3, 1.0, "skew"),                # T > ranges: several tokens per range
+    (2, 2, 4, 2, 1 << 20, 2, 1.0, "skew"),              # H at its maximum (2 MB rows)
 ])
 def test_edge_cases(env, case):
     R, L, S, K, H, B, hr, kind = case
@@ -644,3 +657,70 @@ def test_plan_flags_exclude_each_other(env):
     with pytest.raises(mp.MoonepError) as ei:
         prob.plan(flags=mp.PLAN_REMOTE_WEIGHTS | mp.PLAN_ONE_GROUP)
     assert ei.value.code == mp.ERR_ARG
+
+
+# ---------------------------------------------------------------------------
+# zero_copy = false and the lifetime of zero-copy views
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,mode", [("mid", 0), ("inference", 0), ("inference", 2)])
+def test_copy_out_full_size(env, name, mode):
+    # every row the plan uses is copied, no other row is written (a property
+    # that holds at any size, checked on the device over all rows)
+    torch, mp, harness = env
+    wl = inputs.WORKLOADS[name]
+    cfg = dict(wl.cfg(), C_max=2 * wl.C) if mode == 2 else wl.cfg()
+    r = inputs.routing(wl.R, wl.L, wl.S, wl.K, 1, maxvio=wl.maxvio[0])
+    prob = harness.Problem(cfg)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.fill_x(1)
+    prob.plan(flags=mp.PLAN_ONE_GROUP if mode == 2 else 0)
+    prob.dispatch()
+    out = torch.full_like(prob.recv, 0x1357)
+    mp.moonep_copy_out(cfg, prob.ws, prob.recv, out)
+    torch.cuda.synchronize()
+    assert mp.moonep_plan_read(cfg, prob.ws)["status"] & mp.ST_ERROR_MASK == 0
+    used = prob.row_expert() >= 0
+    assert int(used.sum()) == wl.T * wl.K
+    assert torch.equal(out[used], prob.recv[used])
+    assert bool((out[~used] == 0x1357).all())
+    del out
+
+
+def test_views_go_stale_after_the_next_dispatch(env):
+    torch, mp, harness = env
+    from load_balancing_plan_b200 import views
+    w = inputs.WORKLOADS["tiny"]
+    cfg = w.cfg()
+    r = inputs.routing(w.R, w.L, w.S, w.K, 0, alpha=1.0)
+    prob = harness.Problem(cfg)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.fill_x(0)
+    prob.plan()
+    prob.dispatch()
+    used1 = (prob.row_expert() >= 0).view(w.R, w.C_max)[1]
+    v = views.RecvView(cfg, prob.ws, prob.recv, rank=1)
+    first = v.tensor.clone()
+    kept = v.copy()                       # zero_copy = false
+    assert v.valid()
+    assert torch.equal(kept[used1], first[used1])
+    # a second step writes other rows into the same buffer
+    r2 = inputs.routing(w.R, w.L, w.S, w.K, 5, alpha=1.0)
+    prob.set_routing(r2.topk_idx, r2.topk_w)
+    prob.fill_x(5)
+    prob.plan()
+    prob.dispatch()
+    torch.cuda.synchronize()
+    assert not v.valid()
+    with pytest.raises(views.StaleViewError):
+        v.tensor
+    with pytest.raises(views.StaleViewError):
+        v.copy()
+    # the buffer now holds the second step's rows; the copy taken before
+    # still holds the first step's
+    assert not torch.equal(prob.recv.view(w.R, w.C_max, w.H)[1][used1], first[used1])
+    assert torch.equal(kept[used1], first[used1])
+    # combine moves the generation too
+    v2 = views.RecvView(cfg, prob.ws, prob.recv)
+    prob.combine()
+    assert not v2.valid()
