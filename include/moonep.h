@@ -135,8 +135,11 @@ typedef struct {
  * the first entry p of e with j < route_end[p]); seg_off, seg_len
  * [R][2L+B] (L local, B slot, L fallback segments per rank); alloc [N][R]
  * (rows of expert e on rank r, fallback included: the allocation table);
- * base [N][n_ranges] (copies of e in earlier token ranges; dispatch scratch).
- * Tables from `cnt` up to, not including, `base` are contiguous. */
+ * base [N][n_ranges] (copies of e in the earlier token ranges of the range's
+ * block) and blk [N][n_blocks] (copies of e in earlier blocks; a block is
+ * n_ranges / n_blocks consecutive ranges): dispatch scratch, copy numbers
+ * start at base + blk.  Tables from `cnt` up to, not including, `base` are
+ * contiguous. */
 #define MOONEP_WS_HEADER_WORDS 64
 typedef struct {
     int64_t words;      /* total size in int32 words                  */
@@ -153,6 +156,8 @@ typedef struct {
     int64_t tables_end; /* = base                                      */
     int64_t base;
     int64_t rep_off, recv_ptr, slot_piece; /* (between rep_cnt and rx_expert in memory) */
+    int64_t n_blocks;   /* blocks of consecutive token ranges          */
+    int64_t blk;
 } moonep_ws_layout_t;
 
 /* Per-rank buffer sizes in bytes, as a real deployment would allocate them
@@ -309,8 +314,11 @@ MOONEP_API int moonep_plan_noalloc(const moonep_cfg_t *cfg, const int32_t *topk_
  * wait that runs out sets MOONEP_ST_TIMEOUT and the kernel returns. */
 MOONEP_API int moonep_set_wait_limit(int64_t polls);
 
-/* Token ranges (dispatch CTAs) used for T tokens. */
-MOONEP_API int64_t moonep_num_ranges(int64_t T);
+/* Token ranges (dispatch CTAs) used for T tokens and N experts: a whole
+ * number w >= 1 of waves of 296 ranges (two per SM of a B200), w = T / 4736
+ * rounded to the nearest (about 16 tokens per range) and at most
+ * 2^20 / (296 N); T itself if T is smaller. */
+MOONEP_API int64_t moonep_num_ranges(int64_t T, int64_t N);
 
 /* Description of the last host error on this thread ("" if none). */
 MOONEP_API const char *moonep_last_error(void);

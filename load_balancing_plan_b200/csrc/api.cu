@@ -165,7 +165,7 @@ int moonep_rank_bytes(const moonep_cfg_t *cfg, int64_t elems_per_expert, moonep_
     return MOONEP_OK;
 }
 
-int64_t moonep_num_ranges(int64_t T) { return T < 0 ? 0 : num_ranges(T); }
+int64_t moonep_num_ranges(int64_t T, int64_t N) { return T < 0 || N < 0 ? 0 : num_ranges(T, N); }
 
 int moonep_set_wait_limit(int64_t polls) {
     if (polls < 0) return fail(MOONEP_ERR_ARG, "wait limit < 0");
@@ -201,6 +201,13 @@ int moonep_plan_ex(const moonep_cfg_t *cfg, int32_t flags, const int32_t *topk_i
     p.T = T;
     compute_layout(*cfg, p.lay);
     p.Q = p.lay.n_ranges;
+    {
+        // phase A holds one block's (range, expert) histogram in shared memory
+        const int64_t rpb = p.lay.n_blocks > 0 ? (p.Q + p.lay.n_blocks - 1) / p.lay.n_blocks : 0;
+        if ((size_t)(rpb * N) * sizeof(int) > d->plan_smem)
+            return fail(MOONEP_ERR_ARG, "plan: %lld ranges per block of %d experts exceed shared memory",
+                        (long long)rpb, N);
+    }
     p.ids = topk_idx;
     p.ws = (int32_t *)ws;
     p.wait_limit = g_wait_limit.load();
@@ -232,7 +239,9 @@ int moonep_dispatch(const moonep_cfg_t *cfg, void *ws, const void *x, const int3
     p.Q = p.lay.n_ranges;
     p.row_bytes = (uint32_t)cfg->H * 2;
     size_t smem = 0;
-    const int ctas_per_sm = (int)((p.Q + d->sms - 1) / d->sms);
+    // two resident CTAs per SM; ranges beyond those run in later waves
+    int ctas_per_sm = (int)((p.Q + d->sms - 1) / d->sms);
+    if (ctas_per_sm > 2) ctas_per_sm = 2;
     cudaError_t e = dispatch_smem_config(N, p.row_bytes, ctas_per_sm < 1 ? 1 : ctas_per_sm, &p.piece_bytes, &p.npc,
                                          &smem);
     if (e != cudaSuccess) return fail(MOONEP_ERR_ARG, "dispatch: no shared-memory configuration for H=%d", cfg->H);
@@ -416,7 +425,7 @@ int moonep_reduce_grad(const moonep_cfg_t *cfg, void *ws, float *g_home, float *
     p.ws = (int32_t *)ws;
     compute_layout(*cfg, p.lay);
     p.wait_limit = g_wait_limit.load();
-    cudaError_t e = launch_reduce_grad(p, d->sms * 8, (cudaStream_t)stream);
+    cudaError_t e = launch_reduce_grad(p, d->sms, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "reduce_grad kernel launch");
     return MOONEP_OK;
 }

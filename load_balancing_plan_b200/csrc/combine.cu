@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
     extern __shared__ __align__(1024) uint8_t smem[];
     int32_t *ws = p.ws;
     if (block_status_failed(ws)) return;
-    if (!cfg_matches(ws, p.cfg, num_ranges(p.T))) {
+    if (!cfg_matches(ws, p.cfg, num_ranges(p.T, (int64_t)p.cfg.R * p.cfg.L))) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
     }

@@ -5,21 +5,25 @@
 // writes there, so no receive-buffer-to-compute-buffer copy exists;
 // agentlenshq "MoonshotAI/MoonEP", "How it works": fused permute).
 //
-// One CTA per token range (the ranges the plan counted; two per SM).  Warp 0
+// One CTA per token range (the ranges the plan counted: about 16 tokens each,
+// run in waves of two resident CTAs per SM, so that at any moment the stores
+// of all CTAs go to neighbouring rows of each expert's segment).  Warp 0
 // numbers the range's copies in ascending g: for each group of 32 ids it
 // finds equal experts with __match_any_sync, ranks lanes within a group by
 // popcount, and adds a per-expert running counter kept in shared memory
-// (initialised from the plan's per-range prefix), which gives the copy index
+// (initialised from the plan's base + blk prefixes), which gives the copy index
 // j of every (token, k); j maps to a flat row through the expert's route
-// entries.  The data moves through shared-memory stages, one row piece each:
-// a loader warp fills a stage from x with 16-byte loads (then a proxy fence
-// and an mbarrier arrive), and lane 0 of warp 0 stores the piece K times
-// straight to its destination rows with TMA bulk copies (bulk async-groups),
-// handing the stage back on an mbarrier once the group has read it.  Keeping
-// the x loads off the TMA unit lets them overlap the row stores instead of
-// queueing behind them (about 4% faster than the same pipeline with TMA
-// loads, which MOONEP_DISPATCH_LOADER=0 builds).  Numbering runs just ahead
+// entries.  Lane 0 then moves the data with TMA bulk copies: each row piece
+// of x is loaded once into a shared-memory stage (mbarrier completion) and
+// stored K times straight to its destination rows (bulk async-groups), with
+// kLookahead loads in flight ahead of the stores.  Numbering runs just ahead
 // of the copies, so its cost hides under them.  No multicast.
+//
+// MOONEP_DISPATCH_LOADER=1 builds a variant in which a loader warp fills the
+// stages with 16-byte loads and the TMA unit only stores.  With one long
+// token range per resident CTA it was 4% faster (the x loads no longer queued
+// behind the stores); with the short ranges the plan makes, the plain
+// TMA pipeline is about 1% ahead, so it is the default.
 #include "moonep_internal.cuh"
 
 namespace moonep {
@@ -33,7 +37,7 @@ namespace {
 #define MOONEP_DISPATCH_LOOKAHEAD 6  // loads issued ahead of the stores
 #endif
 #ifndef MOONEP_DISPATCH_LOADER
-#define MOONEP_DISPATCH_LOADER 1     // 1: a loader warp fetches x with plain loads, TMA only stores; 0: TMA loads too
+#define MOONEP_DISPATCH_LOADER 0     // 1: a loader warp fetches x with plain loads, TMA only stores; 0: TMA loads too
 #endif
 #ifndef MOONEP_DISPATCH_HINTS
 #define MOONEP_DISPATCH_HINTS 1      // bit 0: evict-first on the x loads, bit 1: on the row stores
@@ -113,7 +117,13 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
     }
     const Smem sm = carve(smem_raw, p.piece_bytes);
     const int K = p.cfg.K, npc = p.npc;
-    for (int e = lane; e < p.N; e += 32) sm.ctr[e] = __ldg(ws + p.lay.base + (int64_t)e * p.Q + q);
+    {
+        // copy numbers of this range start after the earlier ranges of its
+        // block and the earlier blocks
+        const int64_t NB = p.lay.n_blocks, b = block_of_range(q, p.Q, NB);
+        for (int e = lane; e < p.N; e += 32)
+            sm.ctr[e] = __ldg(ws + p.lay.base + (int64_t)e * p.Q + q) + __ldg(ws + p.lay.blk + (int64_t)e * NB + b);
+    }
     if (lane == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.bars[s], 1);
         fence_mbar_init();
@@ -241,7 +251,13 @@ __global__ void __launch_bounds__(32 * (1 + kLoaderWarps), 1)
     sm.ring = reinterpret_cast<int32_t *>(empty + kStages);
     sm.ctr = sm.ring + kRing;
     const int K = p.cfg.K, npc = p.npc;
-    for (int e = threadIdx.x; e < p.N; e += blockDim.x) sm.ctr[e] = __ldg(ws + p.lay.base + (int64_t)e * p.Q + q);
+    {
+        // copy numbers of this range start after the earlier ranges of its
+        // block and the earlier blocks
+        const int64_t NB = p.lay.n_blocks, b = block_of_range(q, p.Q, NB);
+        for (int e = threadIdx.x; e < p.N; e += blockDim.x)
+            sm.ctr[e] = __ldg(ws + p.lay.base + (int64_t)e * p.Q + q) + __ldg(ws + p.lay.blk + (int64_t)e * NB + b);
+    }
     if (threadIdx.x == 0) {
         for (int st = 0; st < kStages; ++st) {
             mbar_init(&sm.bars[st], 1);

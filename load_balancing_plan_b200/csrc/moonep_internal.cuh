@@ -31,15 +31,52 @@ enum : int {
     HDR_PEND = 21,
 };
 
-// Token ranges of the dispatch grid: two per SM of a B200 (148 SMs).  The
-// plan counts copies per (expert, range) so each dispatch CTA can number its
-// copies without looking at other ranges.
-#ifndef MOONEP_RANGES
-#define MOONEP_RANGES 296
+// Token ranges of the dispatch grid.  The plan counts copies per (expert,
+// range) so each dispatch CTA can number its copies without looking at other
+// ranges.  Ranges are short (about kRangeTokens tokens) and far more numerous
+// than the CTAs the GPU holds at once (kMinRanges: two per SM of a B200), so
+// the resident CTAs always work on neighbouring token ranges and their row
+// stores land close together in every expert's segment (DRAM pages stay
+// open; with one long range per resident CTA the stores of dispatch spread
+// over the whole receive buffer at once and ran 6% slower).  Q is a whole
+// number of such waves, so the last wave is full, and at most about
+// kBaseWords / N so that the per-(expert, range) table stays small.
+constexpr int64_t kMinRanges = 296;
+#ifndef MOONEP_RANGE_TOKENS
+#define MOONEP_RANGE_TOKENS 16
 #endif
-constexpr int64_t kRanges = MOONEP_RANGES;
+constexpr int64_t kRangeTokens = MOONEP_RANGE_TOKENS;
+constexpr int64_t kBaseWords = int64_t(1) << 20;
+// The plan counts ranges in blocks of consecutive ranges (one CTA walks a
+// block and keeps a running count per expert); kBlocks blocks at most.
+constexpr int64_t kBlocks = 296;
 
-__host__ __device__ inline int64_t num_ranges(int64_t T) { return T < kRanges ? T : kRanges; }
+#ifndef MOONEP_RANGE_WAVES
+#define MOONEP_RANGE_WAVES 1
+#endif
+__host__ __device__ inline int64_t num_ranges(int64_t T, int64_t N) {
+    if (!MOONEP_RANGE_WAVES) {
+        int64_t q = T / kRangeTokens;
+        const int64_t cap = kBaseWords / (N > 0 ? N : 1);
+        if (q > cap) q = cap;
+        if (q < kMinRanges) q = kMinRanges;
+        return q < T ? q : (T > 0 ? T : 0);
+    }
+    const int64_t wave_tokens = kRangeTokens * kMinRanges;
+    int64_t w = (T + wave_tokens / 2) / wave_tokens;  // waves, rounded to the nearest
+    const int64_t wcap = kBaseWords / ((N > 0 ? N : 1) * kMinRanges);
+    if (w > wcap) w = wcap;
+    if (w < 1) w = 1;
+    const int64_t q = w * kMinRanges;
+    return q < T ? q : (T > 0 ? T : 0);
+}
+
+__host__ __device__ inline int64_t num_blocks(int64_t Q) { return Q < kBlocks ? Q : kBlocks; }
+
+// block b of NB holds ranges [b*Q/NB, (b+1)*Q/NB); range q is in block
+// floor(((q+1)*NB - 1) / Q) (the last b with b*Q/NB <= q)
+__host__ __device__ inline int64_t block_first_range(int64_t b, int64_t Q, int64_t NB) { return b * Q / NB; }
+__host__ __device__ inline int64_t block_of_range(int64_t q, int64_t Q, int64_t NB) { return ((q + 1) * NB - 1) / Q; }
 
 // token range q of Q: [q*T/Q, (q+1)*T/Q)
 __host__ __device__ inline int64_t range_begin(int64_t q, int64_t T, int64_t Q) { return q * T / Q; }
@@ -60,7 +97,8 @@ __host__ __device__ inline void compute_layout(const moonep_cfg_t &c, moonep_ws_
     const int64_t NR = 2 * N + P;
     const int64_t SEG = R * (2 * (int64_t)c.L + c.B);
     int64_t o = MOONEP_WS_HEADER_WORDS;
-    l.n_ranges = num_ranges(T);
+    l.n_ranges = num_ranges(T, N);
+    l.n_blocks = num_blocks(l.n_ranges);
     l.max_pieces = P;
     l.cnt = o; o += N;
     l.keep = o; o += N;
@@ -96,6 +134,8 @@ __host__ __device__ inline void compute_layout(const moonep_cfg_t &c, moonep_ws_
     l.tables_end = o;
     l.base = o;
     o += N * (l.n_ranges > 0 ? l.n_ranges : 1);
+    l.blk = o;
+    o += N * (l.n_blocks > 0 ? l.n_blocks : 1);
     o = (o + 3) & ~(int64_t)3;
     l.words = o;
 }
@@ -368,7 +408,7 @@ cudaError_t launch_combine(const CombineParams &p, int grid, size_t smem, cudaSt
 cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages, size_t *smem);
 const void *combine_kernel_ptr();
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s);
-cudaError_t launch_reduce_grad(const CopyParams &p, int grid, cudaStream_t s);
+cudaError_t launch_reduce_grad(const CopyParams &p, int sms, cudaStream_t s);
 int set_error(int code, const char *msg);
 cudaError_t launch_copy_out(const CopyOutParams &p, int blocks_per_rank, cudaStream_t s);
 cudaError_t launch_combine_backward(const BackwardParams &p, int grid, size_t smem, cudaStream_t s);

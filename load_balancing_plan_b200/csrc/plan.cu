@@ -7,16 +7,18 @@
 // experts in MoE models" (the GPU planner; the planner emits cu_seqlens).
 //
 // One persistent cooperative kernel, 512 threads per CTA, one CTA per SM:
-//   phase A  every CTA counts the top-K ids of its token ranges into a
-//            shared-memory histogram, writes the per-(expert, range) counts
-//            and adds them to the global tokens_per_expert (cnt);
+//   phase A  every CTA walks blocks of consecutive token ranges, counting
+//            the top-K ids into a running shared-memory histogram; it
+//            stores the running count before each range (base: copies of e
+//            in the block's earlier ranges) and the block total (blk), and
+//            adds the totals to the global tokens_per_expert (cnt);
 //   barrier  one bounded grid barrier (gives up after wait_limit polls and
 //            records MOONEP_ST_TIMEOUT; all CTAs are co-resident by the
 //            cooperative launch, so it normally completes at once);
 //   phase B  CTA 0 runs the planner on cnt (keep/spill split, spill stream,
 //            receiver walk, pieces, slots, fallback, route/segment/alloc
-//            tables) while CTAs 1.. turn the per-range counts into
-//            exclusive prefixes (one warp per expert column).
+//            tables) while CTAs 1.. turn the block totals into exclusive
+//            prefixes (one warp per expert column).
 //
 // The spill planner.  Spilled rows form one stream, expert by expert in
 // ascending order (chunk m of expert e spans stream positions [A_e, A_e +
@@ -442,14 +444,22 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     const moonep_ws_layout_t &lay = p.lay;
 
     if (blockIdx.x == 0) TRACE(ws, 0);
-    // phase A: per-range histograms; each thread issues up to kIdBatch id
-    // loads before its first shared-memory atomic, so the range costs about
-    // one memory latency instead of one per loop trip
+    // phase A: each CTA takes blocks of consecutive token ranges and counts
+    // the block's ids into a shared-memory histogram per (range, expert) --
+    // all of a block's ids are loaded in one batch of up to kIdBatch per
+    // thread, so a block costs about one memory latency however many ranges
+    // it holds.  Then one thread per expert walks the block's ranges in
+    // order: base[e][q] = copies of e in the block's earlier ranges, blk[e][b]
+    // = the block's total, which also goes into the global
+    // tokens_per_expert (cnt).
     bool bad = false;
-    for (int64_t q = blockIdx.x; q < p.Q; q += gridDim.x) {
-        for (int e = tid; e < N; e += kPlanThreads) sm[e] = 0;
+    const int64_t NB = lay.n_blocks;
+    for (int64_t b = blockIdx.x; b < NB; b += gridDim.x) {
+        const int64_t qa = block_first_range(b, p.Q, NB), qb = block_first_range(b + 1, p.Q, NB);
+        const int nr = (int)(qb - qa);
+        for (int i = tid; i < nr * N; i += kPlanThreads) sm[i] = 0;
         __syncthreads();
-        const int64_t i0 = range_begin(q, p.T, p.Q) * K, i1 = range_begin(q + 1, p.T, p.Q) * K;
+        const int64_t i0 = range_begin(qa, p.T, p.Q) * K, i1 = range_begin(qb, p.T, p.Q) * K;
         for (int64_t b0 = i0; b0 < i1; b0 += (int64_t)kIdBatch * kPlanThreads) {
             int v[kIdBatch];
 #pragma unroll
@@ -461,18 +471,26 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
             for (int u = 0; u < kIdBatch; ++u) {
                 const int64_t i = b0 + tid + (int64_t)u * kPlanThreads;
                 if (i < i1) {
-                    if ((unsigned)v[u] < (unsigned)N)
-                        atomicAdd(&sm[v[u]], 1);
-                    else
+                    if ((unsigned)v[u] < (unsigned)N) {
+                        // the range of token i / K: the last q with q*T/Q <= t
+                        const int64_t t = i / K;
+                        const int64_t q = ((t + 1) * p.Q - 1) / p.T;
+                        atomicAdd(&sm[(q - qa) * N + v[u]], 1);
+                    } else {
                         bad = true;
+                    }
                 }
             }
         }
         __syncthreads();
         for (int e = tid; e < N; e += kPlanThreads) {
-            const int v = sm[e];
-            ws[lay.base + (int64_t)e * p.Q + q] = v;
-            if (v) atomicAdd(ws + lay.cnt + e, v);
+            int run = 0;
+            for (int r = 0; r < nr; ++r) {
+                ws[lay.base + (int64_t)e * p.Q + qa + r] = run;
+                run += sm[r * N + e];
+            }
+            ws[lay.blk + (int64_t)e * NB + b] = run;
+            if (run) atomicAdd(ws + lay.cnt + e, run);
         }
         __syncthreads();
     }
@@ -494,12 +512,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     if (blockIdx.x == 0) TRACE(ws, 2);
     if (block_status_failed(ws)) return;
 
-    // phase B: column prefixes on CTAs 1.. (or all on CTA 0 if alone); CTA 0
-    // loads cnt with all its threads, then plans (one warp, or all warps for
-    // more than kWarpPlannerMaxN experts)
+    // phase B: exclusive prefixes of the block totals per expert on CTAs 1..
+    // (or all on CTA 0 if alone); CTA 0 loads cnt with all its threads, then
+    // plans (one warp, or all warps for more than kWarpPlannerMaxN experts)
     const int warp = tid >> 5;
     if (gridDim.x == 1)
-        for (int e = warp; e < N; e += kWarps) scan_column(ws + lay.base + (int64_t)e * p.Q, p.Q);
+        for (int e = warp; e < N; e += kWarps) scan_column(ws + lay.blk + (int64_t)e * NB, NB);
     if (blockIdx.x == 0) {
         for (int e = tid; e < N; e += kPlanThreads) sm[e] = __ldcg(ws + lay.cnt + e);
         __syncthreads();
@@ -510,7 +528,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     } else {
         const int gw = (blockIdx.x - 1) * kWarps + warp;
         const int nw = (gridDim.x - 1) * kWarps;
-        for (int e = gw; e < N; e += nw) scan_column(ws + lay.base + (int64_t)e * p.Q, p.Q);
+        for (int e = gw; e < N; e += nw) scan_column(ws + lay.blk + (int64_t)e * NB, NB);
         __syncthreads();
         if (blockIdx.x == 1) TRACE(ws, 8);
     }
@@ -518,7 +536,15 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
 
 }  // namespace
 
-size_t plan_smem_bytes(int N) { return (size_t)7 * (N > 0 ? N : 1) * sizeof(int); }
+// Dynamic shared memory of the plan: 7 arrays of N ints for the planner, or
+// phase A's (range, expert) histogram of a block, ceil(Q / NB) * N ints,
+// whichever is larger.  With Q <= max(kMinRanges, kBaseWords / N) and NB =
+// min(Q, kBlocks), ceil(Q / NB) * N <= kBaseWords / kBlocks + N.
+size_t plan_smem_bytes(int N) {
+    const int64_t n = N > 0 ? N : 1;
+    const int64_t a = 7 * n, b = kBaseWords / kBlocks + n + 1;
+    return (size_t)(a > b ? a : b) * sizeof(int);
+}
 
 const void *plan_kernel_ptr() { return (const void *)plan_kernel; }
 

@@ -47,7 +47,7 @@ LAYOUT_FIELDS = ["words", "n_ranges", "max_pieces", "cnt", "keep", "spill", "hom
                  "slot_off", "slot_first_j", "rep_ptr", "rep_expert", "rep_recv", "rep_slot",
                  "rep_first_j", "rep_cnt", "rx_expert", "route_ptr", "route_end", "route_base",
                  "seg_off", "seg_len", "alloc", "tables_end", "base", "rep_off", "recv_ptr",
-                 "slot_piece"]
+                 "slot_piece", "n_blocks", "blk"]
 
 
 class WsLayout(ctypes.Structure):
@@ -82,7 +82,7 @@ _sig = {
     "moonep_copy_out": ([_CP, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_view_generation": ([_vp], _i64),
     "moonep_set_wait_limit": ([_i64], ctypes.c_int),
-    "moonep_num_ranges": ([_i64], _i64),
+    "moonep_num_ranges": ([_i64, _i64], _i64),
     "moonep_last_error": ([], ctypes.c_char_p),
     "moonep_version": ([], ctypes.c_char_p),
 }
@@ -155,8 +155,8 @@ def moonep_rank_bytes(cfg, elems_per_expert) -> dict:
                 reduce_bytes=out.reduce_bytes)
 
 
-def moonep_num_ranges(T) -> int:
-    return int(_lib.moonep_num_ranges(int(T)))
+def moonep_num_ranges(T, N) -> int:
+    return int(_lib.moonep_num_ranges(int(T), int(N)))
 
 
 def moonep_set_wait_limit(polls) -> None:

@@ -84,16 +84,23 @@ def test_layout_is_consistent(mp):
               dict(R=16, L=24, S=2048, K=8, H=7168, B=4, C=16384, C_max=20480),
               _cfg(S=0, C=0, C_max=0), _cfg(B=0)]:
         lay = mp.moonep_ws_layout(c)
-        tables = [k for k in mp.LAYOUT_FIELDS[3:] if k not in ("tables_end", "base")]
+        tables = [k for k in mp.LAYOUT_FIELDS[3:] if k not in ("tables_end", "base", "n_blocks", "blk")]
         offs = sorted(lay[k] for k in tables)
         assert len(set(offs)) == len(offs)                      # every table has its own place
         assert offs[0] == lay["cnt"] == mp.WS_HEADER_WORDS and offs[-1] < lay["tables_end"]
         assert lay["tables_end"] == lay["base"] <= lay["words"]
         assert lay["words"] % 4 == 0
         T = c["R"] * c["S"]
-        assert lay["n_ranges"] == mp.moonep_num_ranges(T) == min(T, 296)
         N = c["R"] * c["L"]
-        assert lay["words"] - lay["base"] >= N * lay["n_ranges"]
+        # whole waves of 296 ranges of about 16 tokens, at most 2^20 / N
+        # entries per expert (T itself if fewer); blocks of consecutive
+        # ranges, at most 296
+        w = max(1, min((T + 2368) // 4736, (1 << 20) // (N * 296)))
+        Q = min(T, 296 * w)
+        assert lay["n_ranges"] == mp.moonep_num_ranges(T, N) == Q
+        assert lay["n_blocks"] == min(Q, 296)
+        assert lay["blk"] == lay["base"] + N * max(Q, 1)
+        assert lay["words"] >= lay["blk"] + N * max(lay["n_blocks"], 1)
         assert mp.moonep_plan_workspace_bytes(c) == 4 * lay["words"]
 
 
