@@ -136,9 +136,9 @@ typedef struct {
  * [R][2L+B] (L local, B slot, L fallback segments per rank); alloc [N][R]
  * (rows of expert e on rank r, fallback included: the allocation table);
  * base [N][n_ranges] (copies of e in the earlier token ranges of the range's
- * block) and blk [N][n_blocks] (copies of e in earlier blocks; a block is
- * n_ranges / n_blocks consecutive ranges): dispatch scratch, copy numbers
- * start at base + blk.  Tables from `cnt` up to, not including, `base` are
+ * block; written only where the range has a copy of e) and blk [N][n_blocks]
+ * (copies of e in earlier blocks; a block is n_ranges / n_blocks consecutive
+ * ranges): dispatch scratch, copy numbers start at base + blk.  Tables from `cnt` up to, not including, `base` are
  * contiguous. */
 #define MOONEP_WS_HEADER_WORDS 64
 typedef struct {
@@ -315,9 +315,9 @@ MOONEP_API int moonep_plan_noalloc(const moonep_cfg_t *cfg, const int32_t *topk_
 MOONEP_API int moonep_set_wait_limit(int64_t polls);
 
 /* Token ranges (dispatch CTAs) used for T tokens and N experts: a whole
- * number w >= 1 of waves of 296 ranges (two per SM of a B200), w = T / 4736
- * rounded to the nearest (about 16 tokens per range) and at most
- * 2^20 / (296 N); T itself if T is smaller. */
+ * number w >= 1 of waves of 296 ranges (two per SM of a B200), w = T / 1184
+ * rounded to the nearest (about 4 tokens per range) and at most
+ * 2^22 / (296 N); T itself if T is smaller. */
 MOONEP_API int64_t moonep_num_ranges(int64_t T, int64_t N);
 
 /* Description of the last host error on this thread ("" if none). */

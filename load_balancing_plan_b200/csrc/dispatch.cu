@@ -105,6 +105,35 @@ __device__ __forceinline__ bool rank_group(const DispatchParams &p, const Smem &
     return __any_sync(0xffffffffu, bad);
 }
 
+// Copy numbers of range q start after the earlier ranges of its block and
+// the earlier blocks (base + blk).  Only the counters of the experts the
+// range routes to are read: each thread loads those of the ids it covers,
+// kInitBatch ids at a time with all their loads in flight (equal ids store
+// equal values), so the cost follows the range's ids, not the expert count.
+constexpr int kInitBatch = 4;
+__device__ __forceinline__ void init_counters(const DispatchParams &p, int32_t *ctr, int64_t q, int64_t g0,
+                                              int64_t nids, int tid, int nthreads) {
+    const int32_t *ws = p.ws;
+    const int64_t NB = p.lay.n_blocks;
+    const int32_t *base = ws + p.lay.base + q;                          // base[e][q] = base[e * Q]
+    const int32_t *blk = ws + p.lay.blk + block_of_range(q, p.Q, NB);   // blk[e][b] = blk[e * NB]
+    for (int64_t l0 = 0; l0 < nids; l0 += (int64_t)kInitBatch * nthreads) {
+        int e[kInitBatch], v[kInitBatch];
+#pragma unroll
+        for (int u = 0; u < kInitBatch; ++u) {
+            const int64_t l = l0 + tid + (int64_t)u * nthreads;
+            e[u] = l < nids ? __ldg(p.ids + g0 + l) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kInitBatch; ++u)
+            if ((unsigned)e[u] < (unsigned)p.N)
+                v[u] = __ldg(base + (int64_t)e[u] * p.Q) + __ldg(blk + (int64_t)e[u] * NB);
+#pragma unroll
+        for (int u = 0; u < kInitBatch; ++u)
+            if ((unsigned)e[u] < (unsigned)p.N) ctr[e[u]] = v[u];
+    }
+}
+
 __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__ DispatchParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int lane = threadIdx.x;
@@ -117,13 +146,10 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
     }
     const Smem sm = carve(smem_raw, p.piece_bytes);
     const int K = p.cfg.K, npc = p.npc;
-    {
-        // copy numbers of this range start after the earlier ranges of its
-        // block and the earlier blocks
-        const int64_t NB = p.lay.n_blocks, b = block_of_range(q, p.Q, NB);
-        for (int e = lane; e < p.N; e += 32)
-            sm.ctr[e] = __ldg(ws + p.lay.base + (int64_t)e * p.Q + q) + __ldg(ws + p.lay.blk + (int64_t)e * NB + b);
-    }
+    const int64_t t0 = range_begin(q, p.T, p.Q), t1 = range_begin(q + 1, p.T, p.Q);
+    const int64_t ntok = t1 - t0;
+    const int64_t g0 = t0 * K, nids = ntok * K;
+    init_counters(p, sm.ctr, q, g0, nids, lane, 32);
     if (lane == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.bars[s], 1);
         fence_mbar_init();
@@ -131,9 +157,6 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
     }
     __syncwarp();
 
-    const int64_t t0 = range_begin(q, p.T, p.Q), t1 = range_begin(q + 1, p.T, p.Q);
-    const int64_t ntok = t1 - t0;
-    const int64_t g0 = t0 * K, nids = ntok * K;
     const int64_t nunits = ntok * npc;
     const uint32_t last_piece = p.row_bytes - (uint32_t)(npc - 1) * p.piece_bytes;
     const uint64_t pol = policy_evict_first();
@@ -252,11 +275,8 @@ __global__ void __launch_bounds__(32 * (1 + kLoaderWarps), 1)
     sm.ctr = sm.ring + kRing;
     const int K = p.cfg.K, npc = p.npc;
     {
-        // copy numbers of this range start after the earlier ranges of its
-        // block and the earlier blocks
-        const int64_t NB = p.lay.n_blocks, b = block_of_range(q, p.Q, NB);
-        for (int e = threadIdx.x; e < p.N; e += blockDim.x)
-            sm.ctr[e] = __ldg(ws + p.lay.base + (int64_t)e * p.Q + q) + __ldg(ws + p.lay.blk + (int64_t)e * NB + b);
+        const int64_t t0 = range_begin(q, p.T, p.Q), t1 = range_begin(q + 1, p.T, p.Q);
+        init_counters(p, sm.ctr, q, t0 * K, (t1 - t0) * K, threadIdx.x, blockDim.x);
     }
     if (threadIdx.x == 0) {
         for (int st = 0; st < kStages; ++st) {

@@ -37,16 +37,19 @@ enum : int {
 // than the CTAs the GPU holds at once (kMinRanges: two per SM of a B200), so
 // the resident CTAs always work on neighbouring token ranges and their row
 // stores land close together in every expert's segment (DRAM pages stay
-// open; with one long range per resident CTA the stores of dispatch spread
-// over the whole receive buffer at once and ran 6% slower).  Q is a whole
-// number of such waves, so the last wave is full, and at most about
+// open): on the mid workload dispatch takes 666 us with 4-token ranges, 689
+// with 16-token ranges and 734 with one 110-token range per resident CTA.  Q
+// is a whole number of such waves, so the last wave is full, and at most
 // kBaseWords / N so that the per-(expert, range) table stays small.
 constexpr int64_t kMinRanges = 296;
 #ifndef MOONEP_RANGE_TOKENS
-#define MOONEP_RANGE_TOKENS 16
+#define MOONEP_RANGE_TOKENS 4
 #endif
 constexpr int64_t kRangeTokens = MOONEP_RANGE_TOKENS;
-constexpr int64_t kBaseWords = int64_t(1) << 20;
+#ifndef MOONEP_BASE_WORDS_LOG2
+#define MOONEP_BASE_WORDS_LOG2 22
+#endif
+constexpr int64_t kBaseWords = int64_t(1) << MOONEP_BASE_WORDS_LOG2;
 // The plan counts ranges in blocks of consecutive ranges (one CTA walks a
 // block and keeps a running count per expert); kBlocks blocks at most.
 constexpr int64_t kBlocks = 296;

@@ -449,9 +449,11 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     // all of a block's ids are loaded in one batch of up to kIdBatch per
     // thread, so a block costs about one memory latency however many ranges
     // it holds.  Then one thread per expert walks the block's ranges in
-    // order: base[e][q] = copies of e in the block's earlier ranges, blk[e][b]
-    // = the block's total, which also goes into the global
-    // tokens_per_expert (cnt).
+    // order: base[e][q] = copies of e in the block's earlier ranges (stored
+    // only where range q has a copy of e: a range of a few tokens routes to
+    // few experts, and dispatch reads no other entry), blk[e][b] = the
+    // block's total, which also goes into the global tokens_per_expert
+    // (cnt).
     bool bad = false;
     const int64_t NB = lay.n_blocks;
     for (int64_t b = blockIdx.x; b < NB; b += gridDim.x) {
@@ -486,8 +488,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
         for (int e = tid; e < N; e += kPlanThreads) {
             int run = 0;
             for (int r = 0; r < nr; ++r) {
-                ws[lay.base + (int64_t)e * p.Q + qa + r] = run;
-                run += sm[r * N + e];
+                // dispatch reads base[e][q] only where range q routes to e
+                const int c = sm[r * N + e];
+                if (c) ws[lay.base + (int64_t)e * p.Q + qa + r] = run;
+                run += c;
             }
             ws[lay.blk + (int64_t)e * NB + b] = run;
             if (run) atomicAdd(ws + lay.cnt + e, run);

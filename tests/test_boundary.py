@@ -92,10 +92,10 @@ def test_layout_is_consistent(mp):
         assert lay["words"] % 4 == 0
         T = c["R"] * c["S"]
         N = c["R"] * c["L"]
-        # whole waves of 296 ranges of about 16 tokens, at most 2^20 / N
+        # whole waves of 296 ranges of about 4 tokens, at most 2^22 / N
         # entries per expert (T itself if fewer); blocks of consecutive
         # ranges, at most 296
-        w = max(1, min((T + 2368) // 4736, (1 << 20) // (N * 296)))
+        w = max(1, min((T + 592) // 1184, (1 << 22) // (N * 296)))
         Q = min(T, 296 * w)
         assert lay["n_ranges"] == mp.moonep_num_ranges(T, N) == Q
         assert lay["n_blocks"] == min(Q, 296)

@@ -71,7 +71,7 @@ def test_two_calls_in_a_row_match_moonep_plan(mp):
     # two consecutive calls on the shared static workspace, different router
     # outputs and a different configuration the second time, so a stale value
     # left by the first call would show
-    wl = inputs.WORKLOADS["mid"]
+    wl = inputs.WORKLOADS["profile"]
     r1 = inputs.routing(wl.R, wl.L, wl.S, wl.K, 0, maxvio=2.0)
     ref1, got1 = _plan_both(mp, torch, wl.cfg(), r1)
     t = inputs.WORKLOADS["tiny"]
