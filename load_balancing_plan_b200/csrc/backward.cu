@@ -76,9 +76,16 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
         for (int i = threadIdx.x; i < K * kConsumers; i += kThreads) s_part[i] = 0.f;
     __syncthreads();
 
-    const int64_t tb = (int64_t)blockIdx.x * p.T / gridDim.x;
-    const int64_t te = (int64_t)(blockIdx.x + 1) * p.T / gridDim.x;
-    const int64_t u0 = tb * p.upt, u1 = te * p.upt;
+    // the CTA's tokens (whole tokens, so grad_w needs no cross-CTA sum): a
+    // contiguous share, or (MOONEP_INTERLEAVE) every gridDim.x-th token, so
+    // that the CTAs work on neighbouring tokens; unit i of the CTA is chunk
+    // i % upt of its (i / upt)-th token
+    const int64_t tb = MOONEP_INTERLEAVE ? blockIdx.x : (int64_t)blockIdx.x * p.T / gridDim.x;
+    const int64_t tstep = MOONEP_INTERLEAVE ? gridDim.x : 1;
+    const int64_t ntk = MOONEP_INTERLEAVE ? (blockIdx.x < p.T ? (p.T - 1 - blockIdx.x) / gridDim.x + 1 : 0)
+                                          : (int64_t)(blockIdx.x + 1) * p.T / gridDim.x - tb;
+    const int64_t nun = ntk * p.upt;
+    auto unit_of = [&](int64_t i) { return (tb + (i / p.upt) * tstep) * p.upt + i % p.upt; };
     const int64_t row_bytes = (int64_t)p.hv * 16;
     const uint32_t last = (uint32_t)(row_bytes - (int64_t)(p.upt - 1) * CH);
     const uint64_t pol = policy_evict_first();
@@ -93,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
         int valid = 1;
         bool bad = false, fail = false;
         int64_t i = 0;
-        for (int64_t u = u0; u < u1; ++u, ++i) {
+        for (int64_t u = unit_of(0); i < nun; ++i, u = unit_of(i)) {
             const int s = (int)(i % NS);
             if (i >= NS) {
                 int ok = 1;
@@ -159,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
         const int cw = ct >> 5;
         int64_t i = 0;
         bool ok = true;
-        for (int64_t u = u0; u < u1; ++u, ++i) {
+        for (int64_t u = unit_of(0); i < nun; ++i, u = unit_of(i)) {
             const int s = (int)(i % NS);
             if (ok && !mbar_wait_bounded(&full[s], (uint32_t)((i / NS) & 1), p.wait_limit)) {
                 if (ct == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);

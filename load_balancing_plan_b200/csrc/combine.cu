@@ -98,8 +98,12 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
     }
     __syncthreads();
 
-    const int64_t u0 = (int64_t)blockIdx.x * p.units / gridDim.x;
-    const int64_t u1 = (int64_t)(blockIdx.x + 1) * p.units / gridDim.x;
+    // the CTA's units: a contiguous share, or (MOONEP_INTERLEAVE) every
+    // gridDim.x-th unit, so that the CTAs work on neighbouring tokens
+    const int64_t u0 = MOONEP_INTERLEAVE ? blockIdx.x : (int64_t)blockIdx.x * p.units / gridDim.x;
+    const int64_t ustep = MOONEP_INTERLEAVE ? gridDim.x : 1;
+    const int64_t nun = MOONEP_INTERLEAVE ? (blockIdx.x < p.units ? (p.units - 1 - blockIdx.x) / gridDim.x + 1 : 0)
+                                          : (int64_t)(blockIdx.x + 1) * p.units / gridDim.x - u0;
     const int64_t row_bytes = (int64_t)p.hv * 16;
     const uint32_t last = (uint32_t)(row_bytes - (int64_t)(p.upt - 1) * CH);
     const uint64_t pol = policy_evict_first();
@@ -113,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
         int valid = 1;
         bool bad = false, fail = false;
         int64_t i = 0;
-        for (int64_t u = u0; u < u1; ++u, ++i) {
+        for (int64_t u = u0; i < nun; u += ustep, ++i) {
             const int s = (int)(i % NS);
             if (i >= NS) {
                 int ok = 1;
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
         // ------------------------------------------------------- consumers
         const int ct = threadIdx.x - 32;
         int64_t i = 0;
-        for (int64_t u = u0; u < u1; ++u, ++i) {
+        for (int64_t u = u0; i < nun; u += ustep, ++i) {
             const int s = (int)(i % NS);
             if (!mbar_wait_bounded(&full[s], (uint32_t)((i / NS) & 1), p.wait_limit)) {
                 if (ct == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);

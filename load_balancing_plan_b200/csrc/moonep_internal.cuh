@@ -54,6 +54,11 @@ constexpr int64_t kBaseWords = int64_t(1) << MOONEP_BASE_WORDS_LOG2;
 // block and keeps a running count per expert); kBlocks blocks at most.
 constexpr int64_t kBlocks = 296;
 
+// combine, combine_backward and prefetch: deal units to the CTAs round-robin
+// (1) instead of one contiguous share each (0)
+#ifndef MOONEP_INTERLEAVE
+#define MOONEP_INTERLEAVE 0
+#endif
 #ifndef MOONEP_RANGE_WAVES
 #define MOONEP_RANGE_WAVES 1
 #endif

@@ -21,9 +21,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kChunkVecs = 2048;   // 32 KB of fp32 per chunk
-#ifndef MOONEP_REDUCE_EVEN
-#define MOONEP_REDUCE_EVEN 0       // 1: equal interleaved units over one resident wave; 0: 32 KB units round-robin
-#endif
 
 #ifndef MOONEP_PREFETCH_CHUNK
 #define MOONEP_PREFETCH_CHUNK 32768  // bytes per bulk copy
@@ -199,92 +196,6 @@ __global__ void __launch_bounds__(kThreads) reduce_grad_kernel(const __grid_cons
     }
 }
 
-// The same reduction with the work split evenly: the replicated experts'
-// gradients, laid end to end, form V = nrx * vecs vectors, cut into G * m
-// equal units (G = a grid resident in one wave, m chosen so a unit is about
-// 32 KB); CTA b takes units b, b + G, b + 2G, ...  Every CTA moves the same
-// number of bytes (with fixed 32 KB units, 5,376 units over 1,184 CTAs left
-// the last wave half full), and at any moment the grid works on one window of
-// consecutive units, which keeps the DRAM accesses close together (contiguous
-// per-CTA ranges, the other even split, ran 15-40% slower).
-__global__ void __launch_bounds__(kThreads) reduce_grad_even_kernel(const __grid_constant__ CopyParams p) {
-    int32_t *ws = p.ws;
-    if (block_status_failed(ws)) return;
-    if (!cfg_matches(ws, p.cfg, p.lay.n_ranges)) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
-        return;
-    }
-    __shared__ int64_t s_slot[64];   // replica slots of the current expert (<= R <= 64)
-    __shared__ int s_np;
-    const int64_t nrx = __ldcg(ws + HDR_NRX);
-    const int64_t V = nrx * p.vecs;
-    const int64_t G = gridDim.x;
-    const int64_t m = max((int64_t)1, (V + G * kChunkVecs / 2) / (G * kChunkVecs));  // units per CTA
-    // units of whole 8 KB blocks (512 vectors), so every unit starts on a
-    // cache-line boundary
-    const int64_t unit = ((V + G * m - 1) / (G * m) + 511) & ~(int64_t)511;
-    const int B = p.cfg.B;
-    float4 *g_home = reinterpret_cast<float4 *>(const_cast<uint4 *>(p.src));
-    float4 *g_rep = reinterpret_cast<float4 *>(p.dst);
-    constexpr int kRepBatch = 4;
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int64_t k = 0; k < m; ++k) {
-    const int64_t lo = min(V, (k * G + blockIdx.x) * unit), hi = min(V, lo + unit);
-    for (int64_t v = lo; v < hi;) {
-        const int64_t x = v / p.vecs;
-        const int64_t beg = v - x * p.vecs;                         // within the expert
-        const int64_t end = min(hi - x * p.vecs, p.vecs);
-        const int e = __ldg(ws + p.lay.rx_expert + x);
-        __syncthreads();  // the previous expert's slot list is no longer read
-        if (threadIdx.x == 0) {
-            // the expert's pieces in receiver order; pieces without a slot
-            // (remote weights) carry no replica gradient
-            const int pb = __ldg(ws + p.lay.rep_ptr + e), pe = __ldg(ws + p.lay.rep_ptr + e + 1);
-            int n = 0;
-            for (int q = pb; q < pe; ++q) {
-                const int sl = __ldg(ws + p.lay.rep_slot + q);
-                if (sl >= 0) s_slot[n++] = ((int64_t)__ldg(ws + p.lay.rep_recv + q) * B + sl) * p.vecs;
-            }
-            s_np = n;
-        }
-        __syncthreads();
-        const int np = s_np;
-        float4 *home = g_home + (int64_t)e * p.vecs;
-        for (int64_t i = beg + threadIdx.x; i < end; i += 2 * kThreads) {
-            const int64_t i2 = i + kThreads;
-            const bool two = i2 < end;
-            float4 a0 = __ldcs(home + i);
-            float4 a1 = two ? __ldcs(home + i2) : z;
-            for (int q0 = 0; q0 < np; q0 += kRepBatch) {
-                float4 r0[kRepBatch], r1[kRepBatch];
-#pragma unroll
-                for (int qq = 0; qq < kRepBatch; ++qq) {
-                    if (q0 + qq < np) {
-                        const float4 *rp = g_rep + s_slot[q0 + qq];
-                        r0[qq] = __ldcs(rp + i);
-                        r1[qq] = two ? __ldcs(rp + i2) : z;
-                    }
-                }
-#pragma unroll
-                for (int qq = 0; qq < kRepBatch; ++qq)
-                    if (q0 + qq < np) {
-                        add4(a0, r0[qq]);
-                        add4(a1, r1[qq]);
-                    }
-            }
-            __stcs(home + i, a0);
-            if (two) __stcs(home + i2, a1);
-            for (int q = 0; q < np; ++q) {
-                float4 *rp = g_rep + s_slot[q];
-                __stcs(rp + i, z);
-                if (two) __stcs(rp + i2, z);
-            }
-        }
-        v = x * p.vecs + end;
-    }
-    }
-}
-
 }  // namespace
 
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s) {
@@ -297,19 +208,6 @@ cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s) {
 }
 
 cudaError_t launch_reduce_grad(const CopyParams &p, int sms, cudaStream_t s) {
-    if (MOONEP_REDUCE_EVEN) {
-        // one resident wave, the work split evenly over it
-        static std::atomic<int> per_sm{0};
-        int n = per_sm.load(std::memory_order_relaxed);
-        if (n == 0) {
-            cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reduce_grad_even_kernel, kThreads, 0);
-            if (err != cudaSuccess) return err;
-            if (n < 1) n = 1;
-            per_sm.store(n, std::memory_order_relaxed);
-        }
-        reduce_grad_even_kernel<<<sms * n, kThreads, 0, s>>>(p);
-        return cudaGetLastError();
-    }
     static std::atomic<size_t> smem_set[64];
     cudaError_t err = set_smem_limit((const void *)reduce_grad_kernel, 0, smem_set);
     if (err != cudaSuccess) return err;
