@@ -40,7 +40,7 @@ namespace {
 #define MOONEP_DISPATCH_LOADER 0     // 1: a loader warp fetches x with plain loads, TMA only stores; 0: TMA loads too
 #endif
 #ifndef MOONEP_DISPATCH_HINTS
-#define MOONEP_DISPATCH_HINTS 1      // bit 0: evict-first on the x loads, bit 1: on the row stores
+#define MOONEP_DISPATCH_HINTS 3      // bit 0: evict-first on the x loads, bit 1: on the row stores
 #endif
 constexpr int kStages = MOONEP_DISPATCH_STAGES;
 constexpr int kLookahead = MOONEP_DISPATCH_LOOKAHEAD;

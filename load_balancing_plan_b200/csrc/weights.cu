@@ -28,6 +28,9 @@ constexpr int kChunkVecs = 2048;   // 32 KB of fp32 per chunk
 #ifndef MOONEP_PREFETCH_STAGES
 #define MOONEP_PREFETCH_STAGES 6
 #endif
+#ifndef MOONEP_PREFETCH_STORE_HINT
+#define MOONEP_PREFETCH_STORE_HINT 1  // 1: evict-first L2 hint on the slot stores too
+#endif
 #ifndef MOONEP_PREFETCH_LOOKAHEAD
 #define MOONEP_PREFETCH_LOOKAHEAD 4
 #endif
@@ -96,7 +99,10 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
             const int gp = __ldg(ws + p.lay.slot_piece + sp);
             const int64_t slot = (int64_t)__ldg(ws + p.lay.rep_recv + gp) * B + __ldg(ws + p.lay.rep_slot + gp);
             const uint32_t bytes = (uint32_t)min((int64_t)kPfChunk, bytes_per - c * kPfChunk);
-            bulk_s2g_plain(dst_base + slot * bytes_per + c * kPfChunk, smem + (size_t)s * kPfChunk, bytes);
+            if (MOONEP_PREFETCH_STORE_HINT)
+                bulk_s2g(dst_base + slot * bytes_per + c * kPfChunk, smem + (size_t)s * kPfChunk, bytes, pol);
+            else
+                bulk_s2g_plain(dst_base + slot * bytes_per + c * kPfChunk, smem + (size_t)s * kPfChunk, bytes);
             bulk_commit();
             stored = j + 1;
         }
