@@ -50,9 +50,13 @@ constexpr int64_t kRangeTokens = MOONEP_RANGE_TOKENS;
 #define MOONEP_BASE_WORDS_LOG2 22
 #endif
 constexpr int64_t kBaseWords = int64_t(1) << MOONEP_BASE_WORDS_LOG2;
-// The plan counts ranges in blocks of consecutive ranges (one CTA walks a
-// block and keeps a running count per expert); kBlocks blocks at most.
-constexpr int64_t kBlocks = 296;
+// The plan counts ranges in blocks of consecutive ranges (one CTA counts a
+// block); kBlocks blocks at most, one per SM of a B200, so that each plan
+// CTA loads all the ids it counts in one batch.
+#ifndef MOONEP_BLOCKS
+#define MOONEP_BLOCKS 148
+#endif
+constexpr int64_t kBlocks = MOONEP_BLOCKS;
 
 // combine, combine_backward and prefetch: deal units to the CTAs round-robin
 // (1) instead of one contiguous share each (0)
