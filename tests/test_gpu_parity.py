@@ -183,6 +183,8 @@ def test_tiny_reduce_grad_full_size_grads(env):
     (64, 64, 32, 8, 32, 8, 0.0, "skew"),                # N at its maximum
     (5, 3, 1000, 4, 40, 3, 1.0, "skew"),                # T > ranges: several tokens per range
     (2, 2, 4, 2, 1 << 20, 2, 1.0, "skew"),              # H at its maximum (2 MB rows)
+    (2, 4, 64, 2, 16, 1024, 1.0, "skew"),               # B at its maximum
+    (64, 2, 8, 2, 16, 1024, 1.0, "skew"),               # R * B at its maximum (65536 slots)
 ])
 def test_edge_cases(env, case):
     R, L, S, K, H, B, hr, kind = case
