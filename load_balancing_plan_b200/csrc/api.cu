@@ -366,10 +366,8 @@ int moonep_copy_out(const moonep_cfg_t *cfg, void *ws, const void *recv, void *o
     p.src = (const uint4 *)recv;
     p.dst = (uint4 *)out;
     p.ws = (int32_t *)ws;
-    // the CTAs one wave holds (6 of 256 threads per SM), shared by the R fill runs
-    int per_rank = (int)((6 * (int64_t)d->sms + cfg->R - 1) / cfg->R);
-    if (per_rank < 1) per_rank = 1;
-    cudaError_t e = launch_copy_out(p, per_rank, (cudaStream_t)stream);
+    p.wait_limit = g_wait_limit.load();
+    cudaError_t e = launch_copy_out(p, d->sms, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "copy_out kernel launch");
     return MOONEP_OK;
 }

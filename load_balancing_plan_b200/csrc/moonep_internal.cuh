@@ -58,7 +58,7 @@ constexpr int64_t kBaseWords = int64_t(1) << MOONEP_BASE_WORDS_LOG2;
 #endif
 constexpr int64_t kBlocks = MOONEP_BLOCKS;
 
-// combine, combine_backward and prefetch: deal units to the CTAs round-robin
+// combine and combine_backward: deal units to the CTAs round-robin
 // (1) instead of one contiguous share each (0)
 #ifndef MOONEP_INTERLEAVE
 #define MOONEP_INTERLEAVE 0
@@ -230,6 +230,7 @@ struct CopyParams {
 struct CopyOutParams {
     moonep_cfg_t cfg;
     int64_t Q;            // token ranges of the plan (workspace check)
+    int64_t wait_limit;
     int64_t row_vecs;     // 16-byte vectors per row
     const uint4 *src;     // receive buffer [R, C_max, H]
     uint4 *dst;           // the caller's copy, same shape
@@ -422,7 +423,7 @@ const void *combine_kernel_ptr();
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s);
 cudaError_t launch_reduce_grad(const CopyParams &p, int sms, cudaStream_t s);
 int set_error(int code, const char *msg);
-cudaError_t launch_copy_out(const CopyOutParams &p, int blocks_per_rank, cudaStream_t s);
+cudaError_t launch_copy_out(const CopyOutParams &p, int sms, cudaStream_t s);
 cudaError_t launch_combine_backward(const BackwardParams &p, int grid, size_t smem, cudaStream_t s);
 cudaError_t combine_backward_config(int K, int hv, bool with_grad_w, uint32_t *chunk, int *upt, int *stages,
                                     size_t *smem);
