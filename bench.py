@@ -412,10 +412,40 @@ class Runner:
         return a.elapsed_time(z), h2d_bytes, d2h_bytes
 
 
+def bind_near_gpu(device_index):
+    """Restricts this process to the CPUs next to the GPU's PCIe root (its
+    NUMA node, as sysfs lists them), so that the pinned host buffers of the
+    e2e measurement are allocated in that node's memory and host<->device
+    copies do not cross the inter-socket link.  Returns a description, or None
+    if the list is not available (nothing changes then)."""
+    try:
+        import torch
+        pr = torch.cuda.get_device_properties(device_index)
+        path = "/sys/bus/pci/devices/%04x:%02x:%02x.0/local_cpulist" % (pr.pci_domain_id, pr.pci_bus_id,
+                                                                       pr.pci_device_id)
+        with open(path) as f:
+            spec = f.read().strip()
+        cpus = set()
+        for part in spec.split(","):
+            if "-" in part:
+                a, b = part.split("-")
+                cpus.update(range(int(a), int(b) + 1))
+            elif part:
+                cpus.add(int(part))
+        use = cpus & os.sched_getaffinity(0)
+        if not use:
+            return None
+        os.sched_setaffinity(0, use)
+        return "%d host cpus local to the GPU (%s)" % (len(use), spec)
+    except Exception:
+        return None
+
+
 def run_gpu(args):
     import torch
     rank, local_rank, world = rank_env()
     torch.cuda.set_device(local_rank)
+    host_cpus = bind_near_gpu(local_rank)
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -489,7 +519,7 @@ def run_gpu(args):
                    "weights_per_expert": "bf16 [%d x %d x %d]" % (wl.P, wl.H, wl.I),
                    "grads_per_expert": "fp32 [%d x %d]" % (wl.H, wl.I),
                    "accumulate": "fp32", "parallelism": "replicas%d" % world,
-                   "plan_mode": args.plan_mode, "launch": launch_mode,
+                   "plan_mode": args.plan_mode, "launch": launch_mode, "host_cpus": host_cpus,
                    "l2": "no flush: inputs larger than L2 (x %.2f GB, recv %.2f GB)"
                          % (run.prob.x.numel() * 2 / 1e9, run.prob.recv.numel() * 2 / 1e9)},
         "plan_us": round(mean["plan"] * 1e3, 2),

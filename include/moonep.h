@@ -138,8 +138,8 @@ typedef struct {
  * base [N][n_ranges] (copies of e in the earlier token ranges of the range's
  * block; written only where the range has a copy of e) and blk [N][n_blocks]
  * (copies of e in earlier blocks; a block is n_ranges / n_blocks consecutive
- * ranges): dispatch scratch, copy numbers start at base + blk.  Tables from `cnt` up to, not including, `base` are
- * contiguous. */
+ * ranges): dispatch scratch, copy numbers start at base + blk.  Tables
+ * from `cnt` up to, not including, `base` are contiguous. */
 #define MOONEP_WS_HEADER_WORDS 64
 typedef struct {
     int64_t words;      /* total size in int32 words                  */
