@@ -21,7 +21,11 @@
  *  - prefetch copies the duplicated experts' weights into slots [E, E+B) and
  *    reduce_grad adds the replica gradients to the home expert's gradient,
  *    then clears the used slots (twodots.gr "MoonEP balances AI experts in
- *    MoE models", the memory-contract paragraphs).
+ *    MoE models", the memory-contract paragraphs);
+ *  - the plan's two variants: remote weights beyond B slots and one home
+ *    group per receiver (or_plan_ex modes 1 and 2, with their citations);
+ *  - copy-out for zero_copy = false (or_copy_out) and the backward pair
+ *    (or_combine_backward, or_dispatch_backward).
  *
  * The pages give no planning algorithm.  The spill rule implemented here is
  * the library's documented rule: each home rank keeps its rows in expert
