@@ -330,6 +330,56 @@ def test_dispatch_wait_timeout_is_reported_or_complete(env):
     assert np.array_equal(prob.dest.cpu().numpy(), opl["dest"].reshape(-1))
 
 
+@pytest.mark.parametrize("kernel", ["prefetch", "combine", "combine_backward", "copy_out"])
+def test_pipeline_wait_timeout_is_reported_and_recoverable(env, kernel):
+    # every TMA pipeline gives up after wait_limit polls (0 here): it either
+    # finishes anyway or records MOONEP_ST_TIMEOUT and returns; the context
+    # stays usable and the next plan clears the status
+    torch, mp, harness = env
+    cfg = cfg_of(8, 4, 512, 4, 4096, 4, headroom=1.0)
+    r = inputs.routing(8, 4, 512, 4, 0, alpha=1.0)
+    E = 64 * 1024
+    prob = harness.Problem(cfg, w_elems=E)
+    prob.set_routing(r.topk_idx, r.topk_w)
+    prob.fill_x(0)
+    prob.fill_weights(0)
+
+    def run():
+        if kernel == "prefetch":
+            prob.prefetch()
+            return prob.w_slot
+        if kernel == "combine":
+            prob.combine()
+            return prob.out
+        if kernel == "combine_backward":
+            gy = torch.zeros_like(prob.recv)
+            gw = torch.zeros(prob.T * cfg["K"], dtype=torch.float32, device="cuda")
+            mp.moonep_combine_backward(cfg, prob.ws, prob.x, prob.recv, prob.dest, prob.w, gy, gw)
+            return gy
+        out = torch.full_like(prob.recv, 0x1357)
+        mp.moonep_copy_out(cfg, prob.ws, prob.recv, out)
+        return out
+
+    prob.plan()
+    prob.dispatch()
+    torch.cuda.synchronize()
+    try:
+        mp.moonep_set_wait_limit(0)
+        got = run().clone()
+        torch.cuda.synchronize()
+        status = prob.read_plan(tables=False)["status"]
+    finally:
+        mp.moonep_set_wait_limit(1 << 22)
+    assert status & mp.ST_ERROR_MASK & ~mp.ST_TIMEOUT == 0
+    prob.plan()
+    prob.dispatch()
+    ref = run().clone()
+    torch.cuda.synchronize()
+    assert prob.read_plan(tables=False)["status"] & mp.ST_ERROR_MASK == 0
+    if not status & mp.ST_TIMEOUT:
+        assert torch.equal(got, ref)
+
+
 # ---------------------------------------------------------------------------
 # full-size workloads (the benchmark's launch configuration), sampled
 # ---------------------------------------------------------------------------
