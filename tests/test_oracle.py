@@ -497,3 +497,52 @@ def test_copy_out_copies_exactly_the_rows_in_use(oracle_lib, mode_name, seed):
     assert n == used.sum() == R * S * K
     assert np.array_equal(out[used], recv[used])
     assert np.all(out[~used] == 0xBEEF)
+
+
+def test_plan_invariants_detect_planted_mistakes(oracle_lib):
+    # the invariant checker used on every plan must reject plausible mistakes:
+    # two copies of different experts swapped, a copy sent to a row outside
+    # its expert's segments, a capacity overrun, receivers out of order
+    R, L, S, K, B = 4, 2, 16, 2, 4
+    cfg = _cfg(R, L, S, K, 8, B, C_max=2 * S * K)
+    cnt = np.array([40, 14, 26, 12, 12, 8, 8, 8])
+    ids = pc.ids_from_counts(cnt, R, S, K)
+    pl = oracle_lib.plan(cfg, ids)
+    pc.check_plan(cfg, ids, pl)
+    assert pl["n_replicas"] >= 2
+
+    def rejects(mutate):
+        bad = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in pl.items()}
+        mutate(bad)
+        with pytest.raises(AssertionError):
+            pc.check_plan(cfg, ids, bad)
+
+    flat = ids.reshape(-1)
+    a = int(np.nonzero(flat == 0)[0][0])
+    b = int(np.nonzero(flat == 3)[0][0])
+
+    def swap(p):
+        d = p["dest"].reshape(-1)
+        d[a], d[b] = d[b], d[a]
+    rejects(swap)
+
+    def stray(p):
+        d = p["dest"].reshape(-1)
+        d[a] = (d[a] + cfg["C"]) % (R * cfg["C_max"])
+    rejects(stray)
+
+    def overrun(p):
+        al = p["alloc"].reshape(R * L, R)
+        al[0, 0] += 1
+        al[0, 1] -= 1
+    rejects(overrun)
+
+    rp = pl["rep_ptr"]
+    split = [e for e in range(R * L) if rp[e + 1] - rp[e] >= 2]
+    assert split                      # an expert spread over two receivers
+
+    def reorder(p):
+        e = split[0]
+        lo, hi = p["rep_ptr"][e], p["rep_ptr"][e + 1]
+        p["rep_recv"][lo:hi] = p["rep_recv"][lo:hi][::-1].copy()
+    rejects(reorder)
