@@ -159,3 +159,43 @@ def test_copy_out_arguments_checked_before_any_cuda_call(mp):
 def test_view_generation_of_unknown_workspace_is_zero(mp):
     assert mp.moonep_view_generation(0x1000) == 0
     assert mp.moonep_view_generation(None) == 0
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "moonep.h"
+
+int main(void) {
+    moonep_cfg_t c = {8, 8, 4096, 8, 7168, 8, 32768, 32768};
+    moonep_ws_layout_t lay;
+    moonep_rank_bytes_t rb;
+    if (moonep_ws_layout(&c, &lay) != MOONEP_OK) return 1;
+    if (moonep_plan_workspace_bytes(&c) != (size_t)lay.words * 4) return 2;
+    if (moonep_num_ranges(32768, 64) != lay.n_ranges) return 3;
+    if (moonep_rank_bytes(&c, 2 * 7168 * 2048, &rb) != MOONEP_OK) return 4;
+    if (rb.dispatch_bytes != (int64_t)32768 * 7168 * 2) return 5;
+    if (moonep_set_wait_limit(-1) != MOONEP_ERR_ARG || strlen(moonep_last_error()) == 0) return 6;
+    if (moonep_set_wait_limit(1 << 22) != MOONEP_OK) return 7;
+    c.C = 1;  /* C must equal S*K */
+    if (moonep_plan(&c, (const int32_t *)16, (void *)256, 0) != MOONEP_ERR_ARG) return 8;
+    if (moonep_view_generation((void *)4096) != 0) return 9;
+    printf("%s\n", moonep_version());
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(mp, tmp_path):
+    # the boundary is a C ABI: a C99 program that includes the header builds
+    # against the library and calls its host-side entry points
+    import subprocess
+    src = tmp_path / "use_moonep.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "use_moonep"
+    libdir = os.path.dirname(mp.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe), "-L", libdir, "-lmoonep", "-Wl,-rpath," + libdir])
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert "sm_100a" in out.stdout
