@@ -199,6 +199,11 @@ def test_header_is_plain_c_and_links(mp, tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, (out.returncode, out.stderr)
     assert "sm_100a" in out.stdout
+    # and as C++ (the header's extern "C" block)
+    exe2 = tmp_path / "use_moonep_cpp"
+    subprocess.check_call(["g++", "-std=c++17", "-x", "c++", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           str(src), "-o", str(exe2), "-L", libdir, "-lmoonep", "-Wl,-rpath," + libdir])
+    assert subprocess.run([str(exe2)], capture_output=True).returncode == 0
 
 
 C_GPU_PROGRAM = r"""
