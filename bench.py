@@ -632,11 +632,25 @@ class OracleArm:
         return int(max(1, min(self.wl.T, (seconds - r["plan_us"] * 1e-6) / per_tok)))
 
 
+def host_cpu():
+    """The host CPU's model name and the CPUs this process may use."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": len(os.sched_getaffinity(0))}
+
+
 def cpu_baseline(wl, route, seconds):
     arm = OracleArm(wl, route)
     n = arm.calibrate(seconds)
     r = arm.step(n)
-    return {"value": round(r["gbs"], 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+    return {"value": round(r["gbs"], 4), "unit": UNIT, "cores": 1, "kind": "oracle", **host_cpu(),
             "plan_us": round(r["plan_us"], 1), "rows_per_s": round(r["rows_per_s"], 1),
             "sample": "oracle plan over all %d ids, then dispatch+combine over the first %d of %d "
                       "tokens (%.1f s, single-threaded C)" % (wl.T * wl.K, r["tokens"], wl.T, r["seconds"])}
@@ -669,7 +683,7 @@ def run_reference(args):
                    "accumulate": "fp32", "parallelism": "cpu"},
         "plan_us": round(float(np.mean([r["plan_us"] for r in res])), 1),
         "rows_per_s": round(float(np.mean([r["rows_per_s"] for r in res])), 1),
-        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle", **host_cpu(),
                          "sample": "per step: oracle plan over all %d ids, dispatch+combine over the "
                                    "first %d tokens" % (wl.T * wl.K, n)},
         "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
