@@ -646,11 +646,28 @@ def host_cpu():
     return {"cpu_model": model, "nproc": len(os.sched_getaffinity(0))}
 
 
+class one_core:
+    """Pins the process to one of its CPUs for the duration (the oracle is
+    single-threaded C; this keeps it on one core), then restores the set."""
+
+    def __enter__(self):
+        self.saved = os.sched_getaffinity(0)
+        self.core = min(self.saved)
+        os.sched_setaffinity(0, {self.core})
+        return self
+
+    def __exit__(self, *exc):
+        os.sched_setaffinity(0, self.saved)
+        return False
+
+
 def cpu_baseline(wl, route, seconds):
+    info = host_cpu()
     arm = OracleArm(wl, route)
-    n = arm.calibrate(seconds)
-    r = arm.step(n)
-    return {"value": round(r["gbs"], 4), "unit": UNIT, "cores": 1, "kind": "oracle", **host_cpu(),
+    with one_core():
+        n = arm.calibrate(seconds)
+        r = arm.step(n)
+    return {"value": round(r["gbs"], 4), "unit": UNIT, "cores": 1, "kind": "oracle", **info,
             "plan_us": round(r["plan_us"], 1), "rows_per_s": round(r["rows_per_s"], 1),
             "sample": "oracle plan over all %d ids, then dispatch+combine over the first %d of %d "
                       "tokens (%.1f s, single-threaded C)" % (wl.T * wl.K, r["tokens"], wl.T, r["seconds"])}
@@ -664,14 +681,16 @@ def run_reference(args):
     target = wl.maxvio[0] if wl.maxvio else None
     route = inputs.routing(wl.R, wl.L, wl.S, wl.K, args.seed, maxvio=target)
     arm = OracleArm(wl, route)
-    n = arm.calibrate(args.cpu_seconds * 6.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        arm.step(n)
-    res = []
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        res.append(arm.step(n))
-    wall = time.perf_counter() - t0
+    info = host_cpu()
+    with one_core():
+        n = arm.calibrate(args.cpu_seconds * 6.0 / max(1, args.steps + args.warmup))
+        for _ in range(args.warmup):
+            arm.step(n)
+        res = []
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            res.append(arm.step(n))
+        wall = time.perf_counter() - t0
     gbs = float(np.mean([r["gbs"] for r in res]))
     out = {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT, "n_gpus": world,
@@ -683,7 +702,7 @@ def run_reference(args):
                    "accumulate": "fp32", "parallelism": "cpu"},
         "plan_us": round(float(np.mean([r["plan_us"] for r in res])), 1),
         "rows_per_s": round(float(np.mean([r["rows_per_s"] for r in res])), 1),
-        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle", **host_cpu(),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle", **info,
                          "sample": "per step: oracle plan over all %d ids, dispatch+combine over the "
                                    "first %d tokens" % (wl.T * wl.K, n)},
         "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
