@@ -1,6 +1,6 @@
 """Device-side harness around the C ABI: allocates the caller-owned buffers
-with torch, uploads seeded inputs, runs the five calls and reads results
-back.  Used by the GPU tests, the smoke check and the benchmark.
+with torch, uploads seeded inputs, runs the calls of the step and reads
+results back.  Used by the GPU tests, the smoke check and the benchmark.
 
 The stand-in expert here (y = bf16(float(recv) * scale[expert of row])) is
 harness, not product: the pages' group GEMM is out of scope and a
