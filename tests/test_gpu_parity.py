@@ -652,6 +652,7 @@ def test_layers_share_buffers(env):
     (8, 4, 64, 4, 64, 4, 1.0),      # B = E/R
     (8, 8, 128, 8, 64, 2, 1.0),     # fewer slots than L: both limits bind
     (16, 24, 64, 8, 32, 24, 1.0),   # many groups, long spill stream
+    (16, 48, 64, 8, 32, 48, 1.0),   # 768 experts: the whole CTA plans
 ])
 def test_one_group_mode(env, case):
     R, L, S, K, H, B, hr = case
