@@ -57,7 +57,15 @@ __device__ __forceinline__ void trace(int32_t *ws, int slot) {
 constexpr int kWarps = kPlanThreads / 32;
 constexpr int kMaxR = 64;
 constexpr int kIdBatch = 8;
-constexpr int kWarpPlannerMaxN = 512;  // above this many experts the whole CTA plans
+// Above this many experts the whole CTA plans.  Alone and warm, one warp
+// plans a few hundred experts faster (no block barriers), but right after
+// GBs of streaming traffic, as in a real step, the CTA-wide planner wins at
+// every size measured: 36 -> 28 us at 64 experts, 57 -> 40 us at 256, 42 ->
+// 30 us at 384.
+#ifndef MOONEP_WARP_PLANNER_MAX_N
+#define MOONEP_WARP_PLANNER_MAX_N 32
+#endif
+constexpr int kWarpPlannerMaxN = MOONEP_WARP_PLANNER_MAX_N;
 
 // Exclusive scan of n ints (in and out may alias) by one warp; returns the
 // total.  Lane l owns the contiguous run [l*per, (l+1)*per), per = ceil(n/32).
@@ -177,8 +185,8 @@ __device__ void scan_column(int32_t *col, int64_t Q) {
 }
 
 // The planner, run by NT threads of CTA 0: one warp (NT = 32, no block-wide
-// barriers, which dominate at a few hundred experts) or the whole CTA (NT =
-// kPlanThreads, for thousands of experts).  Every intermediate lives in
+// barriers; up to kWarpPlannerMaxN experts) or the whole CTA (NT =
+// kPlanThreads, above that).  Every intermediate lives in
 // shared memory (seven arrays of N ints and a few of R); global memory is
 // only written.  The receiver walk is sequential and always runs on warp 0.
 template <int NT>
