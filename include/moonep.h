@@ -118,7 +118,8 @@ typedef struct {
  * header occupies words [0, MOONEP_WS_HEADER_WORDS):
  *   0 status, 1 fallback_rows, 2 n_replicas, 3 migrated_rows, 4 n_ranges,
  *   5..12 the cfg it was planned for, 13 replicated-expert count,
- *   14 plan flags, 15 pieces with a slot.
+ *   14 plan flags, 15 pieces with a slot, 18 0x5A5A5A5A in a tables-only
+ *   copy made by moonep_plan_noalloc (0 in a full workspace).
  * Tables ([N] unless noted): cnt = copies per expert (tokens_per_expert);
  * keep, spill, home_off (row of e's local segment), fb_cnt, fb_off (row of
  * e's fallback segment); [R]: load (copies homed on r), deficit (C - load,
@@ -301,12 +302,21 @@ MOONEP_API int moonep_plan_read(const moonep_cfg_t *cfg, const void *ws, moonep_
  * lives in a static 2 MiB device array inside the library (held by every
  * GPU that loads it until exit) and the plan header and tables, words
  * [0, layout.tables_end) of the workspace layout, are copied into
- * tables_out (device, 16-byte aligned, caller-owned; readable with
- * moonep_plan_read).  Same kernel and results as moonep_plan; allocates
- * nothing.  Configurations whose workspace exceeds 2 MiB are refused with
- * MOONEP_ERR_ARG.  The first call on a device looks up the array's device
- * address; make that first call before any stream capture.  Every call shares
- * the array, so calls that overlap on the GPU race: serialise them. */
+ * tables_out (device, at least layout.tables_end int32 words, 16-byte
+ * aligned, caller-owned).  Same kernel and results as moonep_plan; allocates
+ * nothing.  The copy is tables only: it lacks the dispatch scratch that
+ * follows the tables in a full workspace, and its header word 18 says so.
+ * moonep_plan_read, moonep_prefetch, moonep_reduce_grad, moonep_copy_out,
+ * moonep_combine and the backward pair read only the header and tables and
+ * accept it as `ws`; moonep_dispatch refuses it (MOONEP_ST_CFG set in its
+ * status word, nothing else written) and needs a full moonep_plan workspace.
+ * Configurations whose workspace (moonep_plan_workspace_bytes) exceeds
+ * 2 MiB are refused with MOONEP_ERR_ARG before any GPU work.  The first call
+ * on a device looks up the array's device address and keeps it for the
+ * life of the CUDA context (after cudaDeviceReset the library must not be
+ * called on that device again in the process); make that first call before
+ * any stream capture.  Every call shares the array, so calls that overlap
+ * on the GPU race: serialise them. */
 MOONEP_API int moonep_plan_noalloc(const moonep_cfg_t *cfg, const int32_t *topk_idx, int32_t *tables_out,
                                    void *stream);
 

@@ -5,7 +5,7 @@
 // writes there, so no receive-buffer-to-compute-buffer copy exists;
 // agentlenshq "MoonshotAI/MoonEP", "How it works": fused permute).
 //
-// One CTA per token range (the ranges the plan counted: about 16 tokens each,
+// One CTA per token range (the ranges the plan counted: about 4 tokens each,
 // run in waves of two resident CTAs per SM, so that at any moment the stores
 // of all CTAs go to neighbouring rows of each expert's segment).  Warp 0
 // numbers the range's copies in ascending g: for each group of 32 ids it
@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
     int32_t *ws = p.ws;
     const int64_t q = blockIdx.x;
     if (block_status_failed(ws)) return;
-    if (!cfg_matches(ws, p.cfg, p.Q)) {
+    // a tables-only copy has no base/blk scratch: refuse it before reading them
+    if (!cfg_matches(ws, p.cfg, p.Q) || tables_only(ws)) {
         if (lane == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
     }
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(32 * (1 + kLoaderWarps), 1)
     int32_t *ws = p.ws;
     const int64_t q = blockIdx.x;
     if (block_status_failed(ws)) return;
-    if (!cfg_matches(ws, p.cfg, p.Q)) {
+    if (!cfg_matches(ws, p.cfg, p.Q) || tables_only(ws)) {
         if (threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
     }

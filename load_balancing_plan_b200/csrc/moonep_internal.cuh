@@ -27,6 +27,7 @@ enum : int {
     HDR_NSLOT = 15,  // pieces with a prefetch slot
     HDR_BAR_COUNT = 16,
     HDR_BAR_GEN = 17,
+    HDR_TABLES_ONLY = 18,  // kTablesOnlyMark: a copy of the header and tables without the dispatch scratch
     HDR_TOTAL_SPILL = 20,
     HDR_PEND = 21,
 };
@@ -260,6 +261,16 @@ __device__ __forceinline__ bool cfg_matches(const int32_t *ws, const moonep_cfg_
     return __ldcg(h + 0) == c.R && __ldcg(h + 1) == c.L && __ldcg(h + 2) == c.S &&
            __ldcg(h + 3) == c.K && __ldcg(h + 4) == c.H && __ldcg(h + 5) == c.B &&
            __ldcg(h + 6) == c.C && __ldcg(h + 7) == c.C_max && __ldcg(ws + HDR_NRANGES) == (int32_t)Q;
+}
+
+// A workspace whose header word HDR_TABLES_ONLY holds this value is a copy of
+// the plan header and tables alone (moonep_plan_noalloc's output): it lacks
+// the dispatch scratch (base, blk) that lies past tables_end.  The value is a
+// repeated byte so a single-word memset writes it.
+constexpr int32_t kTablesOnlyMark = 0x5A5A5A5A;
+
+__device__ __forceinline__ bool tables_only(const int32_t *ws) {
+    return __ldcg(ws + HDR_TABLES_ONLY) == kTablesOnlyMark;
 }
 
 __device__ __forceinline__ unsigned lanemask_lt() {

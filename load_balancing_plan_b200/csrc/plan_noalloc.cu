@@ -11,7 +11,15 @@
 // file-scope device array of kStaticWsBytes (2 MiB, held by every GPU that
 // loads the library until the process exits) and copies the plan header and
 // tables into the caller's output buffer.  It runs the same plan kernel as
-// moonep_plan and allocates nothing.
+// moonep_plan and allocates nothing.  The copy lacks the dispatch scratch
+// that follows the tables in a full workspace, so its header is marked
+// (word HDR_TABLES_ONLY) and moonep_dispatch refuses it; the calls that read
+// only the header and tables (plan_read, prefetch, reduce_grad, copy_out,
+// combine and the backward pair) accept it.
+//
+// The cached device address stays valid for the life of the CUDA context;
+// after cudaDeviceReset on that device it is stale, and the library must not
+// be called on that device again in this process.
 //
 // The array's name is only a host-side handle; its device address comes from
 // cudaGetSymbolAddress, taken once per device, with that device current, by
@@ -84,6 +92,15 @@ extern "C" MOONEP_API int moonep_plan_noalloc(const moonep_cfg_t *cfg, const int
     if (e != cudaSuccess) {
         char msg[256];
         snprintf(msg, sizeof msg, "moonep_plan_noalloc: copy of the tables: %s", cudaGetErrorString(e));
+        return moonep::set_error(MOONEP_ERR_CUDA, msg);
+    }
+    // mark the copy as tables only: it has no dispatch scratch, and dispatch
+    // refuses such a workspace (MOONEP_ST_CFG) instead of reading past its end
+    e = cudaMemsetAsync(tables_out + moonep::HDR_TABLES_ONLY, moonep::kTablesOnlyMark & 0xFF, sizeof(int32_t),
+                        (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof msg, "moonep_plan_noalloc: marking the copy: %s", cudaGetErrorString(e));
         return moonep::set_error(MOONEP_ERR_CUDA, msg);
     }
     return MOONEP_OK;

@@ -174,7 +174,15 @@ def moonep_plan_ex(cfg, flags, topk_idx, ws, stream=None) -> None:
 def moonep_plan_noalloc(cfg, topk_idx, tables_out, stream=None) -> None:
     """moonep_plan without a caller workspace: the library's static device
     workspace is used and the header + tables are copied to tables_out
-    (at least layout["tables_end"] int32 words)."""
+    (at least layout["tables_end"] int32 words).  The copy is tables only:
+    moonep_dispatch refuses it as a workspace.  A tensor smaller than the
+    copy is refused here (the C function sees only its address)."""
+    if hasattr(tables_out, "numel") and hasattr(tables_out, "element_size"):
+        need = 4 * moonep_ws_layout(cfg)["tables_end"]
+        have = int(tables_out.numel()) * int(tables_out.element_size())
+        if have < need:
+            raise MoonepError(ERR_ARG, "moonep_plan_noalloc: tables_out holds %d bytes, the plan tables need %d"
+                              % (have, need))
     _check(_lib.moonep_plan_noalloc(ctypes.byref(cfg_of(cfg)), _p(topk_idx), _p(tables_out),
                                     _stream(stream)))
 

@@ -39,6 +39,36 @@ def test_refuses_configuration_above_static_workspace(mp):
     assert "static workspace" in mp.last_error()
 
 
+@pytest.mark.parametrize("name", ["mid", "skew", "inference", "training"])
+def test_refuses_the_larger_workloads(mp, name):
+    # of the library's workloads only tiny (28 KB) and profile (0.55 MiB) fit
+    # the 2 MiB static workspace; mid already needs 2.07 MiB
+    cfg = inputs.WORKLOADS[name].cfg()
+    assert mp.moonep_plan_workspace_bytes(cfg) > (2 << 20)
+    with pytest.raises(mp.MoonepError) as ei:
+        mp.moonep_plan_noalloc(cfg, 256, 256, stream=0)
+    assert ei.value.code == mp.ERR_ARG
+    assert "static workspace" in mp.last_error()
+
+
+@pytest.mark.parametrize("name", ["tiny", "profile"])
+def test_small_workloads_fit(mp, name):
+    assert mp.moonep_plan_workspace_bytes(inputs.WORKLOADS[name].cfg()) <= (2 << 20)
+
+
+def test_binding_refuses_a_short_output_tensor(mp):
+    # the C function sees only an address; the binding checks the tensor's
+    # size before any GPU work (a CPU tensor is enough to show the refusal)
+    import torch
+    cfg = inputs.WORKLOADS["tiny"].cfg()
+    need = mp.moonep_ws_layout(cfg)["tables_end"]
+    short = torch.zeros(need - 1, dtype=torch.int32)
+    with pytest.raises(mp.MoonepError) as ei:
+        mp.moonep_plan_noalloc(cfg, 256, short, stream=0)
+    assert ei.value.code == mp.ERR_ARG
+    assert "tables_out holds" in str(ei.value)
+
+
 def _plan_both(mp, torch, cfg, route):
     dev = torch.device("cuda")
     ids = torch.from_numpy(route.topk_idx.reshape(-1).copy()).to(dev)
@@ -81,3 +111,51 @@ def test_two_calls_in_a_row_match_moonep_plan(mp):
     assert ref1["n_replicas"] > 0 and ref2["n_replicas"] > 0
     _same(ref1, got1)
     _same(ref2, got2)
+
+
+@pytest.mark.gpu
+def test_tables_only_copy_is_refused_by_dispatch_and_accepted_by_prefetch(mp):
+    """The copy holds no dispatch scratch: moonep_dispatch given it as a
+    workspace sets MOONEP_ST_CFG and writes nothing.  prefetch reads only the
+    tables and gives the same slots as with the full workspace.  The copy is
+    allocated with the full workspace size, so even a dispatch that ignored the
+    mark would read inside the buffer."""
+    import torch
+    from load_balancing_plan_b200 import harness
+    dev = torch.device("cuda")
+    wl = inputs.WORKLOADS["tiny"]
+    cfg = wl.cfg()
+    r = inputs.routing(wl.R, wl.L, wl.S, wl.K, 1, alpha=1.0)
+    E = 1024
+    full = harness.Problem(cfg, poison=True, w_elems=E)
+    full.set_routing(r.topk_idx, r.topk_w)
+    full.fill_x(0)
+    full.fill_weights(0)
+    full.plan()
+    full.prefetch()
+    lay = mp.moonep_ws_layout(cfg)
+    copy = torch.full((lay["words"],), 7, dtype=torch.int32, device=dev)
+    mp.moonep_plan_noalloc(cfg, full.ids, copy)
+    torch.cuda.synchronize()
+    assert int(copy[18]) == 0x5A5A5A5A
+    assert int(full.ws[18]) == 0
+    info = mp.moonep_plan_read(cfg, copy)
+    assert info["status"] & mp.ST_ERROR_MASK == 0 and info["n_replicas"] > 0
+
+    # dispatch on the copy: refused on the device, nothing written
+    recv = torch.full_like(full.recv, -1)
+    dest = torch.full_like(full.dest, -7)
+    mp.moonep_dispatch(cfg, copy, full.x, full.ids, recv, dest)
+    torch.cuda.synchronize()
+    info = mp.moonep_plan_read(cfg, copy)
+    assert info["status"] & mp.ST_CFG
+    assert bool((recv == -1).all()) and bool((dest == -7).all())
+
+    # prefetch with a fresh copy: same slots as with the full workspace
+    copy2 = torch.empty(lay["tables_end"], dtype=torch.int32, device=dev)
+    mp.moonep_plan_noalloc(cfg, full.ids, copy2)
+    w_slot = torch.full_like(full.w_slot, -1)
+    mp.moonep_prefetch(cfg, copy2, full.w_home, w_slot, E)
+    torch.cuda.synchronize()
+    assert mp.moonep_plan_read(cfg, copy2)["status"] & mp.ST_ERROR_MASK == 0
+    assert torch.equal(w_slot, full.w_slot)
