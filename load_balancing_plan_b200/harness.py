@@ -148,3 +148,24 @@ class Problem:
             yr = (xr * s[row_expert[rows]][:, None]).to(torch.bfloat16)
             y[rows] = yr.view(torch.int16)
         return y
+
+    def expert_scale_inplace(self, scale: np.ndarray, row_expert=None, chunk_rows: int = 1 << 16):
+        """The same stand-in expert applied to recv in place, a chunk of rows
+        at a time (for full-size buffers, where a copy of recv would not
+        fit): recv[row] = bf16(float(recv[row]) * scale[expert(row)]) for every
+        row with an expert."""
+        torch = _torch()
+        if row_expert is None:
+            row_expert = self.row_expert()
+        s = torch.from_numpy(np.asarray(scale, np.float32)).to(self.device)
+        nrows = self.recv.shape[0]
+        for r0 in range(0, nrows, chunk_rows):
+            re = row_expert[r0:r0 + chunk_rows]
+            rows = (re >= 0).nonzero().flatten()
+            if rows.numel() == 0:
+                continue
+            blk = self.recv[r0:r0 + chunk_rows]
+            xr = blk[rows].view(torch.bfloat16).float()
+            blk[rows] = (xr * s[re[rows]][:, None]).to(torch.bfloat16).view(torch.int16)
+            del xr
+        return self.recv

@@ -11,6 +11,7 @@ import pytest
 import oracle
 from load_balancing_plan_b200 import inputs
 from tests import planchecks as pc
+from tests import sampled
 
 pytestmark = pytest.mark.gpu
 
@@ -384,6 +385,25 @@ def test_pipeline_wait_timeout_is_reported_and_recoverable(env, kernel):
 # full-size workloads (the benchmark's launch configuration), sampled
 # ---------------------------------------------------------------------------
 
+def check_weighted_combine(torch, harness, prob, route, seed, n_tok=384, rng_seed=5):
+    """Combine after the stand-in expert, on sampled tokens of a full-size
+    problem whose prob.out holds the GPU combine of prob.recv after
+    expert_scale_inplace: bit-exact against the oracle's bf16 output on those
+    tokens (sampled.sampled_weighted_combine) and within 4e-3 of its fp32
+    sum."""
+    c = prob.cfg
+    K, H, N, T = c["K"], c["H"], prob.N, prob.T
+    rng = np.random.default_rng(rng_seed)
+    ts = np.sort(rng.choice(T, n_tok, replace=False))
+    out_o, acc_o = sampled.sampled_weighted_combine(oracle, route, seed, ts, N, K, H)
+    out_g = harness.to_u16(prob.out[torch.from_numpy(ts).cuda()])
+    assert np.array_equal(out_g, out_o)
+    got = inputs.bf16_bits_to_f32_np(out_g)
+    nz = acc_o != 0
+    assert np.all(got[~nz] == 0)
+    assert np.max(np.abs(got[nz] - acc_o[nz]) / np.abs(acc_o[nz])) <= 4e-3
+
+
 # (workload, target maxvio, seed); inference seed 1 needs the headroom
 FULL = [("mid", 2.0, 0), ("skew", 0.0, 0), ("skew", 8.0, 0), ("inference", 4.0, 0),
         ("inference", 4.0, 1), ("training", 8.0, 0)]
@@ -450,6 +470,12 @@ def test_full_size(env, name, maxvio, seed):
     out_o, acc_o = oracle.combine(mini, d_mini, y_mini, w_mini)
     out_g = harness.to_u16(prob.out[torch.from_numpy(ts).cuda()])
     assert np.array_equal(out_g, out_o)
+    # combine after the stand-in expert (scales != 1, replica rows scaled by
+    # their expert's scale), sampled tokens against the oracle
+    prob.expert_scale_inplace(inputs.expert_scales(N, seed), prob.row_expert(gpl))
+    prob.combine()
+    torch.cuda.synchronize()
+    check_weighted_combine(torch, harness, prob, r, seed)
     # prefetch: every used slot, sampled elements
     if w_elems:
         idx = np.sort(rng.choice(w_elems, 4096, replace=False))
@@ -581,6 +607,19 @@ def test_remote_weights_inference_workload(env):
     assert np.array_equal(rows, want)
     # with C_max = C and no fallback every receive row is used
     assert not np.any(np.all(harness.to_u16(prob.recv[::97]) == 0xFFFF, axis=1))
+    # combine of the dispatched rows themselves (identity expert), sampled
+    # tokens against the oracle; then after the stand-in expert, whose rows of
+    # pieces without a slot (remote weights) also take their expert's scale
+    ts = np.sort(np.random.default_rng(3).choice(wl.T, 256, replace=False))
+    xs = inputs.cb_bf16_np(1, inputs.STREAM_X, ts[:, None] * wl.H + np.arange(wl.H)[None, :])
+    mini = dict(R=1, L=1, S=len(ts), K=wl.K, H=wl.H, B=0, C=len(ts) * wl.K, C_max=len(ts) * wl.K)
+    d_mini = np.arange(len(ts) * wl.K, dtype=np.int32).reshape(1, len(ts), wl.K)
+    out_o, _ = oracle.combine(mini, d_mini, np.repeat(xs, wl.K, axis=0), r.topk_w.reshape(wl.T, wl.K)[ts])
+    assert np.array_equal(harness.to_u16(prob.out[torch.from_numpy(ts).cuda()]), out_o)
+    prob.expert_scale_inplace(inputs.expert_scales(wl.N, 1), prob.row_expert(gpl))
+    prob.combine()
+    torch.cuda.synchronize()
+    check_weighted_combine(torch, harness, prob, r, 1)
 
 
 # ---------------------------------------------------------------------------

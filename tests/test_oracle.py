@@ -546,3 +546,28 @@ def test_plan_invariants_detect_planted_mistakes(oracle_lib):
         lo, hi = p["rep_ptr"][e], p["rep_ptr"][e + 1]
         p["rep_recv"][lo:hi] = p["rep_recv"][lo:hi][::-1].copy()
     rejects(reorder)
+
+
+@pytest.mark.parametrize("seed", [0, 3])
+def test_sampled_weighted_combine_matches_the_whole_problem(oracle_lib, seed):
+    # the full-size GPU tests check combine on sampled tokens through a mini
+    # problem built from just those tokens' rows; on the tiny workload, which
+    # the oracle runs whole (plan, dispatch, stand-in expert, combine), the
+    # mini problem gives the same bf16 outputs and fp32 sums for the sample
+    from tests import sampled
+    oracle = oracle_lib
+    wl = inputs.WORKLOADS["tiny"]
+    cfg = wl.cfg()
+    r = inputs.routing(wl.R, wl.L, wl.S, wl.K, seed, alpha=1.0)
+    opl = oracle.plan(cfg, r.topk_idx)
+    assert opl["n_replicas"] > 0                        # replica rows are in the sample's reach
+    x = inputs.cb_bf16_np(seed, inputs.STREAM_X, np.arange(wl.T * wl.H)).reshape(wl.T, wl.H)
+    recv = np.zeros((wl.R * cfg["C_max"], wl.H), np.uint16)
+    oracle.dispatch(cfg, opl["dest"], x, recv)
+    y = recv.copy()
+    oracle.expert_scale(cfg, opl, recv, inputs.expert_scales(wl.N, seed), y)
+    out, acc = oracle.combine(cfg, opl["dest"], y, r.topk_w)
+    ts = np.sort(np.random.default_rng(seed).choice(wl.T, 48, replace=False))
+    out_s, acc_s = sampled.sampled_weighted_combine(oracle, r, seed, ts, wl.N, wl.K, wl.H)
+    assert np.array_equal(out_s, out[ts])
+    assert np.array_equal(acc_s.view(np.uint32), acc[ts].view(np.uint32))
