@@ -1,18 +1,27 @@
 """Benchmark of the MoonEP hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid]
-                    [--impl reference] [--no-sweep]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload training]
+                    [--impl reference] [--no-sweep] [--no-extras]
+                    [--only KERNEL]
 
-A step is one pass of the whole hot path over one MoE layer of the workload:
-moonep_plan -> moonep_prefetch -> moonep_dispatch -> moonep_combine ->
-moonep_reduce_grad (the combine gathers the dispatched rows themselves: the
-expert computation is out of scope).  Inputs are resident in HBM when the
+A step is one pass of the whole hot path over one MoE layer of the workload
+(default: the training workload, R=16 simulated ranks, 256 experts, 131,072
+tokens): moonep_plan -> moonep_prefetch -> moonep_dispatch -> moonep_combine
+-> moonep_reduce_grad (the combine gathers the dispatched rows themselves:
+the expert computation is out of scope).  Inputs are resident in HBM when the
 timed region starts and are larger than L2, so no flush is needed between
 steps.  Every kernel is timed with CUDA events on the launching stream;
 `value` is the dispatch+combine algorithmic bytes over their device time,
 summed over ranks; `e2e` is the same metric through the same calls with the
 router output and hidden states copied in from pinned host memory and the
 combined output copied back, inside the timed region.
+
+At one GPU the same line also carries the mid workload's step (`mid`), the
+inference workload's fallback rows per seed and their throughput cost
+(headroom rows versus remote weights, `inference`), and the skew sweep over
+maxvio 0..8 at five router seeds each (`sweep`).  Their router outputs are
+drawn in spawned worker processes while the GPU measures the main workload.
+--only KERNEL times one kernel alone (profiler captures).
 
 Under torchrun every rank runs its own independent replica of the workload
 ("replicas only": the path is simulated on one GPU, with no exchange between
@@ -74,19 +83,22 @@ def measured_peak():
 
 
 def recorded_traffic(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary, or None."""
+    """DRAM bytes per launch from the committed ncu summary
+    (profiles/dram_traffic.txt: kernel, workload, bytes, then how the figure
+    was obtained), as (bytes, source) or (None, None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         with open(path) as f:
             for line in f:
                 if line.startswith("#") or not line.strip():
                     continue
-                k, w, b = line.split()[:3]
-                if k == kernel and w == workload:
-                    return float(b)
+                parts = line.split(None, 3)
+                if len(parts) >= 3 and parts[0] == kernel and parts[1] == workload:
+                    src = parts[3].strip() if len(parts) > 3 else "profiles/dram_traffic.txt"
+                    return float(parts[2]), src
     except OSError:
         pass
-    return None
+    return None, None
 
 
 # ---------------------------------------------------------------------------
@@ -186,15 +198,18 @@ def barrier(world):
 # ---------------------------------------------------------------------------
 
 class Runner:
-    def __init__(self, wl, maxvio, seed, with_weights=True, plan_flags=0, seed_route=None, with_grads=True):
+    def __init__(self, wl, maxvio, seed, with_weights=True, plan_flags=0, seed_route=None, with_grads=True,
+                 route=None):
         import torch
         from load_balancing_plan_b200 import harness
         self.torch = torch
         self.wl = wl
         self.cfg = wl.cfg()
         t0 = time.time()
-        self.route = inputs.routing(wl.R, wl.L, wl.S, wl.K, seed if seed_route is None else seed_route,
-                                    maxvio=maxvio)
+        if route is None:
+            route = inputs.routing(wl.R, wl.L, wl.S, wl.K, seed if seed_route is None else seed_route,
+                                   maxvio=maxvio)
+        self.route = route
         self.plan_flags = plan_flags
         self.gen_s = time.time() - t0
         we = wl.w_elems if with_weights else 0
@@ -208,6 +223,12 @@ class Runner:
         self.with_weights = with_weights
         self.with_grads = with_weights and with_grads
         torch.cuda.synchronize()
+
+    def set_route(self, route):
+        """Next router output on the same buffers (same shapes)."""
+        self.route = route
+        self.prob.set_routing(route.topk_idx, route.topk_w)
+        self.torch.cuda.synchronize()
 
     def step(self, ev=None):
         p = self.prob
@@ -441,9 +462,104 @@ def bind_near_gpu(device_index):
         return None
 
 
+def _route_job(job):
+    """Router output for one (workload name, seed, target maxvio), drawn in a
+    worker process."""
+    name, seed, mv = job
+    wl = inputs.WORKLOADS[name]
+    return inputs.routing(wl.R, wl.L, wl.S, wl.K, seed, maxvio=mv)
+
+
+class RoutePool:
+    """Draws router outputs in spawned worker processes (no CUDA state is
+    inherited) while the GPU measures.  close() before anything is timed on
+    the host."""
+
+    def __init__(self, jobs, workers):
+        import multiprocessing as mpc
+        self.jobs = list(jobs)
+        self.pool = mpc.get_context("spawn").Pool(workers) if self.jobs and workers > 0 else None
+        self.res = {j: self.pool.apply_async(_route_job, (j,)) for j in self.jobs} if self.pool else {}
+
+    def get(self, job):
+        r = self.res.get(job)
+        return r.get() if r is not None else _route_job(job)
+
+    def wait(self):
+        for r in self.res.values():
+            r.wait()
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.close()
+            self.pool.join()
+            self.pool = None
+
+
+def layer_figures(run, steps, warmup, world, graph, peak):
+    """Plans once (checking the status), then times `steps` steps of the
+    layer.  Returns the per-kernel figures; device times are the max over
+    ranks and work units the sum."""
+    from load_balancing_plan_b200 import moonep as mp
+    run.step()
+    info = mp.moonep_plan_read(run.cfg, run.prob.ws)
+    if info["status"] & mp.ST_ERROR_MASK:
+        raise RuntimeError("plan failed: status 0x%x" % info["status"])
+    tabs = mp.moonep_plan_read(run.cfg, run.prob.ws, tables=True)
+    n_rx = len(set(np.asarray(tabs["rep_expert"]).tolist()))
+    n_slot = int((np.asarray(tabs["rep_slot"]) >= 0).sum())   # pieces whose weights are prefetched
+    w_el = run.prob.w_elems if run.with_weights else 0
+    g_el = run.prob.g_elems if run.with_grads else 0
+    ab = alg_bytes(run.cfg, n_slot, n_rx, w_el, g_el)
+    total_ms, per, clocks, launch_mode = run.timed(steps, warmup, world, graph=graph)
+    mean = {k: float(np.mean(v)) for k, v in per.items()}
+    dc_ms = sum(per["dispatch"]) + sum(per["combine"])
+    max_dc_ms, dc_bytes = reduce_over_ranks(dc_ms, (ab["dispatch"] + ab["combine"]) * steps, world)
+    T, K = run.prob.T, run.cfg["K"]
+    max_total_ms, rows = reduce_over_ranks(total_ms, T * K * steps, world)
+    value = dc_bytes / (max_dc_ms * 1e-3) / 1e9
+    shares = {k: sum(v) for k, v in per.items()}
+    dom = max(("dispatch", "combine", "prefetch", "reduce_grad"), key=lambda k: shares[k])
+    kernel_gbs = {k: (ab[k] / (mean[k] * 1e-3) / 1e9 if mean[k] > 0 and ab[k] else None)
+                  for k in ("dispatch", "combine", "prefetch", "reduce_grad")}
+    return dict(info=info, n_rx=n_rx, n_slot=n_slot, ab=ab, mean=mean, per=per, value=value,
+                ms_per_step=max_total_ms / steps, rows_per_s=rows / (max_total_ms * 1e-3),
+                dom=dom, kernel_gbs=kernel_gbs, clocks=clocks, launch_mode=launch_mode,
+                frac=value / world / peak)
+
+
+def short_figures(f, T, K):
+    """The per-layer figures an extra workload reports."""
+    info = f["info"]
+    return {"value": round(f["value"], 2), "unit": UNIT, "ms_per_step": round(f["ms_per_step"], 4),
+            "dispatch_combine_frac_of_peak": round(f["frac"], 4),
+            "plan_us": round(f["mean"]["plan"] * 1e3, 2),
+            "kernel_us": {k: round(v * 1e3, 2) for k, v in f["mean"].items()},
+            "kernel_gbs": {k: (round(v, 1) if v else None) for k, v in f["kernel_gbs"].items()},
+            "rows_per_s": round(f["rows_per_s"], 1),
+            "plan_info": {"n_replicas": info["n_replicas"], "slotted_replicas": f["n_slot"],
+                          "replicated_experts": f["n_rx"], "migrated_rows": info["migrated_rows"],
+                          "migrated_frac": round(info["migrated_rows"] / (T * K), 4),
+                          "fallback_rows": info["fallback_rows"]}}
+
+
+def wl_desc(wl, route, extra=""):
+    return ("%s: R=%d L=%d (N=%d experts) S=%d K=%d H=%d B=%d C=%d C_max=%d, router bias tuned to maxvio "
+            "%.2f (achieved %.3f)%s" % (wl.name, wl.R, wl.L, wl.N, wl.S, wl.K, wl.H, wl.B, wl.C, wl.C_max,
+                                         route.target if route.target is not None else -1, route.maxvio, extra))
+
+
 def run_gpu(args):
     import torch
     rank, local_rank, world = rank_env()
+    extras = world == 1 and not args.no_extras
+    # router outputs for the extra workloads, drawn while the GPU measures
+    jobs = []
+    if extras:
+        jobs += [("inference", s, inputs.WORKLOADS["inference"].maxvio[0]) for s in args.seeds]
+        if not args.no_sweep:
+            jobs += [("skew", s, mv) for mv in inputs.WORKLOADS["skew"].maxvio for s in args.seeds]
+    pool = RoutePool(jobs, min(args.route_workers, len(jobs)))
     torch.cuda.set_device(local_rank)
     host_cpus = bind_near_gpu(local_rank)
     if world > 1:
@@ -463,89 +579,76 @@ def run_gpu(args):
         # receivers locked to one home group leave rows on their home ranks
         import dataclasses
         wl = dataclasses.replace(wl, headroom=max(wl.headroom, 1.0))
+    peak, peak_kind = measured_peak()
     # inference (no gradients): plan -> prefetch -> dispatch -> combine
     run = Runner(wl, target, seed=args.seed, plan_flags=flags, seed_route=args.route_seed,
                  with_grads=wl.name != "inference")
-    from load_balancing_plan_b200 import moonep as mp
-    info = mp.moonep_plan_read(run.cfg, run.prob.ws)   # also checks the status
-    run.step()
-    info = mp.moonep_plan_read(run.cfg, run.prob.ws)
-    if info["status"] & mp.ST_ERROR_MASK:
-        raise RuntimeError("plan failed: status 0x%x" % info["status"])
-    tabs = mp.moonep_plan_read(run.cfg, run.prob.ws, tables=True)
-    n_rx = len(set(np.asarray(tabs["rep_expert"]).tolist()))
-    n_slot = int((np.asarray(tabs["rep_slot"]) >= 0).sum())   # pieces whose weights are prefetched
-    ab = alg_bytes(run.cfg, n_slot, n_rx, run.prob.w_elems, run.prob.g_elems)
+    f = layer_figures(run, args.steps, args.warmup, world, not args.eager, peak)
+    info, ab, mean, dom = f["info"], f["ab"], f["mean"], f["dom"]
+    achieved = ab[dom] / (mean[dom] * 1e-3) / 1e9
+    bwd = run.backward(max(10, args.steps // 10), args.warmup)
 
-    total_ms, per, clocks, launch_mode = run.timed(args.steps, args.warmup, world, graph=not args.eager)
-    mean = {k: float(np.mean(v)) for k, v in per.items()}
-    dc_ms = sum(per["dispatch"]) + sum(per["combine"])
-    max_dc_ms, dc_bytes = reduce_over_ranks(dc_ms, (ab["dispatch"] + ab["combine"]) * args.steps, world)
-    max_total_ms, rows = reduce_over_ranks(total_ms, run.prob.T * run.cfg["K"] * args.steps, world)
-    value = dc_bytes / (max_dc_ms * 1e-3) / 1e9
-    ms_per_step = max_total_ms / args.steps
-
+    # the host-timed part waits until the router workers are done
+    pool.wait()
+    pool.close()
     e2e_steps = max(8, args.steps // 8)
     e2e_ms, h2d, d2h = run.e2e(e2e_steps, 3)
     max_e2e_ms, e2e_bytes = reduce_over_ranks(e2e_ms, (ab["dispatch"] + ab["combine"]) * e2e_steps, world)
+    route_main = run.route
+    x_gb, recv_gb = run.prob.x.numel() * 2 / 1e9, run.prob.recv.numel() * 2 / 1e9
+    with_grads = run.with_grads
+    launches = run.launches_per_step() * args.steps
+    del run
+    torch.cuda.empty_cache()
 
-    peak, peak_kind = measured_peak()
-    shares = {k: sum(v) for k, v in per.items()}
-    dom = max(("dispatch", "combine", "prefetch", "reduce_grad"), key=lambda k: shares[k])
-    achieved = ab[dom] / (mean[dom] * 1e-3) / 1e9
-    kernel_gbs = {k: (ab[k] / (mean[k] * 1e-3) / 1e9 if mean[k] > 0 and ab[k] else None)
-                  for k in ("dispatch", "combine", "prefetch", "reduce_grad")}
-
-    bwd = run.backward(max(10, args.steps // 10), args.warmup)
-
-    sweep = None
-    if not args.no_sweep and world == 1:
-        sweep = run_sweep(args, peak)
+    extra = {}
+    if extras:
+        if args.workload != "mid":
+            extra["mid"] = run_mid(args, peak)
+        extra["inference"] = run_inference(args, peak, pool)
+        if not args.no_sweep:
+            extra["sweep"] = run_sweep(args, peak, pool)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(wl, run.route, args.cpu_seconds)
+        cpu = cpu_baseline(wl, route_main, args.cpu_seconds)
 
+    traffic, traffic_src = recorded_traffic(dom, wl.name)
     out = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "metric": METRIC, "value": round(f["value"], 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(f["ms_per_step"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "%s: R=%d L=%d (N=%d experts) S=%d K=%d H=%d B=%d C=%d C_max=%d, "
-                               "router bias tuned to maxvio %.2f (achieved %.3f), seed %d"
-                               % (wl.name, wl.R, wl.L, wl.N, wl.S, wl.K, wl.H, wl.B, wl.C, wl.C_max,
-                                  target if target is not None else -1, run.route.maxvio, args.seed),
-                   "step": "plan -> prefetch -> dispatch -> combine" + (" -> reduce_grad" if run.with_grads else ""),
+        "config": {"workload": wl_desc(wl, route_main, ", seed %d" % (args.seed if args.route_seed is None
+                                                                          else args.route_seed)),
+                   "step": "plan -> prefetch -> dispatch -> combine" + (" -> reduce_grad" if with_grads else ""),
                    "weights_per_expert": "bf16 [%d x %d x %d]" % (wl.P, wl.H, wl.I),
                    "grads_per_expert": "fp32 [%d x %d]" % (wl.H, wl.I),
                    "accumulate": "fp32", "parallelism": "replicas%d" % world,
-                   "plan_mode": args.plan_mode, "launch": launch_mode, "host_cpus": host_cpus,
-                   "l2": "no flush: inputs larger than L2 (x %.2f GB, recv %.2f GB)"
-                         % (run.prob.x.numel() * 2 / 1e9, run.prob.recv.numel() * 2 / 1e9)},
+                   "plan_mode": args.plan_mode, "launch": f["launch_mode"], "host_cpus": host_cpus,
+                   "l2": "no flush: inputs larger than L2 (x %.2f GB, recv %.2f GB)" % (x_gb, recv_gb)},
         "plan_us": round(mean["plan"] * 1e3, 2),
         "kernel_us": {k: round(v * 1e3, 2) for k, v in mean.items()},
-        "kernel_gbs": {k: (round(v, 1) if v else None) for k, v in kernel_gbs.items()},
-        "rows_per_s": round(rows / (max_total_ms * 1e-3), 1),
-        "dispatch_combine_frac_of_peak": round(value / world / peak, 4),
-        "dispatch_combine_frac_of_8tbs": round(value / world / 8000.0, 4),
-        "plan_info": {"n_replicas": info["n_replicas"], "slotted_replicas": n_slot,
+        "kernel_gbs": {k: (round(v, 1) if v else None) for k, v in f["kernel_gbs"].items()},
+        "rows_per_s": round(f["rows_per_s"], 1),
+        "dispatch_combine_frac_of_peak": round(f["value"] / world / peak, 4),
+        "dispatch_combine_frac_of_8tbs": round(f["value"] / world / 8000.0, 4),
+        "plan_info": {"n_replicas": info["n_replicas"], "slotted_replicas": f["n_slot"],
                       "migrated_rows": info["migrated_rows"],
-                      "migrated_frac": round(info["migrated_rows"] / (run.prob.T * wl.K), 4),
-                      "fallback_rows": info["fallback_rows"], "replicated_experts": n_rx},
+                      "migrated_frac": round(info["migrated_rows"] / (wl.T * wl.K), 4),
+                      "fallback_rows": info["fallback_rows"], "replicated_experts": f["n_rx"]},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "algorithmic_bytes": ab[dom],
-                     "traffic": recorded_traffic(dom, wl.name)},
+                     "algorithmic_bytes": ab[dom], "traffic": traffic, "traffic_source": traffic_src},
         "e2e": {"value": round(e2e_bytes / (max_e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(max_e2e_ms / e2e_steps, 4)},
-        "gpu_launches": run.launches_per_step() * args.steps,
-        "clocks": clocks,
+        "gpu_launches": launches,
+        "clocks": f["clocks"],
     }
     out["copy_out"] = bwd.pop("copy_out")
     out["backward"] = bwd
-    if sweep is not None:
-        out["sweep"] = sweep
+    out.update(extra)
     if cpu is not None:
         out["cpu_baseline"] = cpu
     if rank == 0:
@@ -555,35 +658,110 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def run_sweep(args, peak):
-    """plan / dispatch / combine over the skew-sweep workload at each target
-    maxvio (seed 0): rows/s should not move with the skew."""
+def run_mid(args, peak):
+    """The mid workload's whole step (plan -> prefetch -> dispatch -> combine
+    -> reduce_grad), seed 0."""
     import torch
-    wl = inputs.WORKLOADS["skew"]
-    res = {}
-    for mv in wl.maxvio:
-        run = Runner(wl, mv, seed=0, with_weights=False)
-        total_ms, per, _, _ = run.timed(args.sweep_steps, 3, graph=not args.eager)
-        from load_balancing_plan_b200 import moonep as mp
+    wl = inputs.WORKLOADS["mid"]
+    run = Runner(wl, wl.maxvio[0], seed=0)
+    f = layer_figures(run, args.extra_steps, 3, 1, not args.eager, peak)
+    out = {"workload": wl_desc(wl, run.route, ", seed 0"),
+           "step": "plan -> prefetch -> dispatch -> combine -> reduce_grad", **short_figures(f, wl.T, wl.K)}
+    del run
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_inference(args, peak, pool):
+    """The inference workload (B = 4 slots, C_max = 1.25 C): headroom-rule
+    fallback rows for every seed, then the step (plan -> prefetch -> dispatch
+    -> combine) timed on the seed with the most fallback rows under the
+    headroom rule and under remote weights (the pages' inference fallback),
+    on the same buffers: the difference is the fallback's throughput cost."""
+    import torch
+    from load_balancing_plan_b200 import moonep as mp
+    wl = inputs.WORKLOADS["inference"]
+    mv = wl.maxvio[0]
+    routes = {s: pool.get(("inference", s, mv)) for s in args.seeds}
+    run = Runner(wl, mv, seed=0, with_grads=False, route=routes[args.seeds[0]])
+    per_seed = {}
+    for s in args.seeds:
+        run.set_route(routes[s])
+        run.prob.plan()
         info = mp.moonep_plan_read(run.cfg, run.prob.ws)
-        ab = alg_bytes(run.cfg)
-        d = float(np.mean(per["dispatch"]))
-        c = float(np.mean(per["combine"]))
-        res["%g" % mv] = {
-            "maxvio": round(run.route.maxvio, 3),
-            "plan_us": round(float(np.mean(per["plan"])) * 1e3, 2),
-            "dispatch_gbs": round(ab["dispatch"] / (d * 1e-3) / 1e9, 1),
-            "combine_gbs": round(ab["combine"] / (c * 1e-3) / 1e9, 1),
-            "dispatch_combine_frac": round((ab["dispatch"] + ab["combine"]) / ((d + c) * 1e-3) / 1e9 / peak, 4),
-            "rows_per_s": round(run.prob.T * wl.K / (total_ms / args.sweep_steps * 1e-3), 1),
-            "migrated_frac": round(info["migrated_rows"] / (run.prob.T * wl.K), 4),
-            "n_replicas": info["n_replicas"], "fallback_rows": info["fallback_rows"],
-        }
-        del run
-        torch.cuda.empty_cache()
-    rps = [v["rows_per_s"] for v in res.values()]
-    return {"workload": "skew: R=8 L=32 S=8192 K=8 H=7168 B=32, seed 0, step = plan -> dispatch -> combine",
-            "points": res, "rows_per_s_spread": round(max(rps) / min(rps) - 1.0, 4)}
+        per_seed[str(s)] = {"maxvio": round(routes[s].maxvio, 3), "fallback_rows": info["fallback_rows"],
+                            "n_replicas": info["n_replicas"], "migrated_rows": info["migrated_rows"]}
+    worst = max(args.seeds, key=lambda s: (per_seed[str(s)]["fallback_rows"], -s))
+    run.set_route(routes[worst])
+    modes = {}
+    for mode, fl in (("headroom", 0), ("remote", mp.PLAN_REMOTE_WEIGHTS)):
+        run.plan_flags = fl
+        f = layer_figures(run, args.extra_steps, 3, 1, not args.eager, peak)
+        modes[mode] = short_figures(f, wl.T, wl.K)
+    hm, rm = modes["headroom"], modes["remote"]
+    out = {"workload": wl_desc(wl, routes[worst]), "step": "plan -> prefetch -> dispatch -> combine",
+           "fallback_rows_per_seed": per_seed, "timed_seed": worst,
+           "fallback_rows": hm["plan_info"]["fallback_rows"],
+           "fallback_cost": {"ms_per_step_headroom": hm["ms_per_step"], "ms_per_step_remote": rm["ms_per_step"],
+                             "step_time_ratio": round(hm["ms_per_step"] / rm["ms_per_step"], 4),
+                             "dispatch_combine_gbs_headroom": hm["value"],
+                             "dispatch_combine_gbs_remote": rm["value"]},
+           "headroom": hm, "remote": rm}
+    del run
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_sweep(args, peak, pool):
+    """plan -> dispatch -> combine on the skew-sweep workload at each target
+    maxvio and seed: rows/s should not move with the skew.  One set of
+    buffers serves every point (only the router output changes)."""
+    import torch
+    from load_balancing_plan_b200 import moonep as mp
+    wl = inputs.WORKLOADS["skew"]
+    ab = alg_bytes(wl.cfg())
+    run = None
+    points = {}
+    all_rps = []
+    for mv in wl.maxvio:
+        seeds = {}
+        for s in args.seeds:
+            route = pool.get(("skew", s, mv))
+            if run is None:
+                run = Runner(wl, mv, seed=0, with_weights=False, route=route)
+            else:
+                run.set_route(route)
+            total_ms, per, _, _ = run.timed(args.sweep_steps, 3, graph=not args.eager)
+            info = mp.moonep_plan_read(run.cfg, run.prob.ws)
+            if info["status"] & mp.ST_ERROR_MASK:
+                raise RuntimeError("sweep plan failed: status 0x%x" % info["status"])
+            d = float(np.mean(per["dispatch"]))
+            c = float(np.mean(per["combine"]))
+            rps = run.prob.T * wl.K / (total_ms / args.sweep_steps * 1e-3)
+            all_rps.append(rps)
+            seeds[str(s)] = {
+                "maxvio": round(route.maxvio, 3),
+                "plan_us": round(float(np.mean(per["plan"])) * 1e3, 2),
+                "dispatch_gbs": round(ab["dispatch"] / (d * 1e-3) / 1e9, 1),
+                "combine_gbs": round(ab["combine"] / (c * 1e-3) / 1e9, 1),
+                "dispatch_combine_frac": round((ab["dispatch"] + ab["combine"]) / ((d + c) * 1e-3) / 1e9 / peak, 4),
+                "rows_per_s": round(rps, 1),
+                "migrated_frac": round(info["migrated_rows"] / (run.prob.T * wl.K), 4),
+                "n_replicas": info["n_replicas"], "fallback_rows": info["fallback_rows"],
+            }
+        rp = [v["rows_per_s"] for v in seeds.values()]
+        points["%g" % mv] = {"seeds": seeds, "rows_per_s_mean": round(float(np.mean(rp)), 1),
+                             "rows_per_s_spread_over_seeds": round(max(rp) / min(rp) - 1.0, 4),
+                             "plan_us_mean": round(float(np.mean([v["plan_us"] for v in seeds.values()])), 2),
+                             "migrated_frac_mean": round(float(np.mean([v["migrated_frac"]
+                                                                        for v in seeds.values()])), 4)}
+    del run
+    torch.cuda.empty_cache()
+    means = [v["rows_per_s_mean"] for v in points.values()]
+    return {"workload": "skew: R=8 L=32 S=8192 K=8 H=7168 B=32, seeds %s, step = plan -> dispatch -> combine"
+                        % ",".join(str(s) for s in args.seeds),
+            "points": points, "rows_per_s_spread": round(max(all_rps) / min(all_rps) - 1.0, 4),
+            "rows_per_s_spread_of_means": round(max(means) / min(means) - 1.0, 4)}
 
 
 # ---------------------------------------------------------------------------
@@ -626,7 +804,11 @@ class OracleArm:
                 "rows_per_s": n * K / (t3 - t2), "tokens": n, "seconds": (t1 - t0) + (t3 - t2)}
 
     def calibrate(self, seconds):
-        n = min(self.wl.T, 128)
+        """Tokens per step so that a step takes about `seconds`: a first
+        small step touches the host buffers (its page faults would inflate
+        the estimate), a second, larger one is timed."""
+        self.step(min(self.wl.T, 128))
+        n = min(self.wl.T, 1024)
         r = self.step(n)
         per_tok = max(r["seconds"] - r["plan_us"] * 1e-6, 1e-7) / n
         return int(max(1, min(self.wl.T, (seconds - r["plan_us"] * 1e-6) / per_tok)))
@@ -710,12 +892,79 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+KERNELS = ("plan", "prefetch", "dispatch", "combine", "reduce_grad")
+
+
+def run_only(args):
+    """One kernel of the step alone, for profiler captures and kernel-alone
+    timings: the buffers that kernel needs (weights only for prefetch,
+    gradients only for reduce_grad), one plan (and a dispatch before combine),
+    then `warmup` untimed and `steps` timed launches of that kernel, each
+    bracketed by CUDA events on the launching stream.  Prints one JSON line
+    with the median launch time and the algorithmic GB/s."""
+    import torch
+    from load_balancing_plan_b200 import harness, moonep as mp
+    torch.cuda.set_device(0)
+    wl = inputs.WORKLOADS[args.workload]
+    route = inputs.routing(wl.R, wl.L, wl.S, wl.K, args.seed, maxvio=wl.maxvio[0] if wl.maxvio else None,
+                           alpha=wl.alpha)
+    cfg = wl.cfg()
+    k = args.only
+    if k == "plan":
+        # the plan reads only the ids and writes only the workspace
+        prob = type("PlanOnly", (), {})()
+        prob.ids = torch.from_numpy(np.ascontiguousarray(route.topk_idx.reshape(-1))).cuda()
+        prob.ws = torch.zeros(mp.moonep_plan_workspace_bytes(cfg) // 4, dtype=torch.int32, device="cuda")
+        prob.w_elems = prob.g_elems = 0
+        prob.plan = lambda: mp.moonep_plan(cfg, prob.ids, prob.ws)
+        prob.prefetch = prob.dispatch = prob.combine = prob.reduce_grad = None
+    else:
+        prob = harness.Problem(cfg, w_elems=wl.w_elems if k == "prefetch" else 0,
+                               g_elems=wl.g_elems if k == "reduce_grad" else 0)
+        prob.set_routing(route.topk_idx, route.topk_w)
+        prob.fill_x(args.seed)
+        prob.fill_weights(args.seed)
+        prob.fill_g_rep(args.seed)
+    prob.plan()
+    if k == "combine":
+        prob.dispatch()
+    torch.cuda.synchronize()
+    info = mp.moonep_plan_read(cfg, prob.ws)
+    if info["status"] & mp.ST_ERROR_MASK:
+        raise RuntimeError("plan failed: status 0x%x" % info["status"])
+    tabs = mp.moonep_plan_read(cfg, prob.ws, tables=True)
+    n_rx = len(set(np.asarray(tabs["rep_expert"]).tolist()))
+    n_slot = int((np.asarray(tabs["rep_slot"]) >= 0).sum())
+    ab = alg_bytes(cfg, n_slot, n_rx, prob.w_elems, prob.g_elems)[k]
+    fn = {"plan": prob.plan, "prefetch": prob.prefetch, "dispatch": prob.dispatch,
+          "combine": prob.combine, "reduce_grad": prob.reduce_grad}[k]
+    s = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        fn()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    for i in range(args.steps):
+        ev[2 * i].record(s)
+        fn()
+        ev[2 * i + 1].record(s)
+    torch.cuda.synchronize()
+    us = float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps)])) * 1e3
+    info = mp.moonep_plan_read(cfg, prob.ws)
+    if info["status"] & mp.ST_ERROR_MASK:
+        raise RuntimeError("%s failed: status 0x%x" % (k, info["status"]))
+    peak, peak_kind = measured_peak()
+    print(json.dumps({"kernel": k, "workload": wl_desc(wl, route, ", seed %d" % args.seed),
+                      "launches": args.warmup + args.steps + 1 + (k == "combine"), "us": round(us, 2),
+                      "algorithmic_bytes": ab, "gbs": round(ab / us / 1e3, 1),
+                      "frac_of_peak": round(ab / us / 1e3 / peak, 4), "peak_kind": peak_kind,
+                      "n_replicas": info["n_replicas"], "replicated_experts": n_rx}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mid", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--workload", default="training", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--route-seed", type=int, default=None,
@@ -724,6 +973,15 @@ def main(argv=None):
                     help="overflow beyond a receiver's slots: headroom rows on the home rank, or remote "
                          "weights; one_group: receivers take replicas of one home group only")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--only", choices=KERNELS, default=None,
+                    help="time one kernel alone on the workload (profiler captures)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="only the main workload (no mid, inference or sweep figures)")
+    ap.add_argument("--seeds", type=lambda v: [int(x) for x in v.split(",")], default=[0, 1, 2, 3, 4],
+                    help="router seeds of the sweep and the inference fallback count")
+    ap.add_argument("--extra-steps", type=int, default=20, help="timed steps of each extra workload")
+    ap.add_argument("--route-workers", type=int, default=6,
+                    help="worker processes drawing the extra workloads' router outputs")
     ap.add_argument("--eager", action="store_true", help="launch every step from the host (no CUDA graph)")
     ap.add_argument("--sweep-steps", type=int, default=20)
     ap.add_argument("--no-cpu", action="store_true")
@@ -734,6 +992,8 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_only(args)
     else:
         run_gpu(args)
 

@@ -93,6 +93,12 @@ WORKLOADS = {
     # the mid shapes at a quarter of the tokens and an eighth of the FFN size:
     # about 3 GB on the device, still far above L2, for profiler captures
     "profile": Workload("profile", R=8, L=8, S=1024, K=8, H=7168, B=8, I=256, maxvio=(2.0,)),
+    # the full FFN size (I = 2048, 58.7 MB of fp32 gradient per expert) over
+    # 16 experts, for captures of the weight and gradient kernels: at seed 0,
+    # 3 replicated experts with 3, 3 and 2 pieces (the mid workload has 3, 4
+    # and 1); prefetch moves 0.94 GB and reduce_grad 1.29 GB (as on mid), far
+    # above L2, while the weights or gradients take about 1.9 GB
+    "profile_w": Workload("profile_w", R=8, L=2, S=4096, K=2, H=7168, B=2, I=2048, maxvio=(2.0,)),
 }
 
 
