@@ -320,6 +320,82 @@ MOONEP_API int moonep_plan_read(const moonep_cfg_t *cfg, const void *ws, moonep_
 MOONEP_API int moonep_plan_noalloc(const moonep_cfg_t *cfg, const int32_t *topk_idx, int32_t *tables_out,
                                    void *stream);
 
+/* ------------------------------------------------------------------------
+ * Expert parallelism: one rank per GPU ("The Busiest Rank Sets Your Step
+ * Time", section "Installation and integration": eight ranks over NVLink,
+ * the weight tensor mapped from each home rank; twodots.gr "MoonEP balances
+ * AI experts in MoE models", memory-contract paragraphs: dispatch writes
+ * into the other ranks' receive buffers, prefetch reads weights from the
+ * home rank, reduce_grad reads the replica gradients from the receivers).
+ *
+ * Rank r holds its own S tokens (topk_idx, topk_w and x of [S][K], [S][K]
+ * and [S][H]; rows s of rank r are global tokens r*S + s), its receive
+ * buffer recv_r [C_max][H], its experts' weights [L][elems] and gradients
+ * [L][elems], and its slots [B][elems] (bf16 weights, fp32 replica
+ * gradients).  A step:
+ *   1. moonep_ep_count: histogram of the rank's ids into counts [N + 1]
+ *      (device int32: copies per expert, then the rank's status bits), plus
+ *      the per-range scratch dispatch needs, into the rank's workspace
+ *      (moonep_ep_workspace_bytes; layout from moonep_ep_ws_layout).
+ *   2. all-gather of every rank's counts into counts_all [R][N + 1] on every
+ *      rank, by the caller (for example NCCL's all-gather).
+ *   3. moonep_ep_plan: every rank plans from the same counts, so every rank
+ *      derives the same tables (identical to moonep_plan's for the R*S
+ *      tokens); the rank's copy numbers start after the lower ranks' copies.
+ *   4. moonep_ep_prefetch, moonep_ep_dispatch, (experts), moonep_ep_combine,
+ *      moonep_ep_reduce_grad, each on the rank's own stream.
+ * Between steps the caller orders the ranks (a barrier on every rank after
+ * its dispatch and before any combine reads the expert outputs; likewise
+ * around prefetch and reduce_grad): the kernels never wait on one another.
+ * Peer tables (recv_peers, y_peers, w_home_peers, g_rep_peers) are device
+ * arrays of R device pointers, entry q pointing at rank q's buffer as this
+ * GPU addresses it (peer-mapped memory, CUDA IPC or symmetric allocations;
+ * the rank's own buffer at entry r).  `dest` holds global flat rows
+ * q*C_max + row as in moonep_dispatch.  Copies use plain loads and bulk
+ * copies, never a multicast load.  The workspace status of every call
+ * behaves as in the single-GPU calls; a bad id on any rank makes every
+ * rank's plan fail (the status travels in counts). */
+
+/* Workspace layout and size of one rank's plan (the dispatch scratch
+ * covers the rank's S tokens). */
+MOONEP_API int moonep_ep_ws_layout(const moonep_cfg_t *cfg, moonep_ws_layout_t *out);
+MOONEP_API size_t moonep_ep_workspace_bytes(const moonep_cfg_t *cfg);
+
+/* Step 1.  topk_idx: device int32 [S][K], rank `rank`'s ids.  counts:
+ * device int32 [N + 1], written.  Clears the workspace header; no host
+ * sync. */
+MOONEP_API int moonep_ep_count(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_idx, void *ws,
+                               int32_t *counts, void *stream);
+
+/* Step 3.  counts_all: device int32 [R][N + 1], row q = rank q's counts.
+ * flags as in moonep_plan_ex.  The tables equal moonep_plan_ex's on the
+ * concatenated ids. */
+MOONEP_API int moonep_ep_plan(const moonep_cfg_t *cfg, int32_t flags, int32_t rank, const int32_t *counts_all,
+                              void *ws, void *stream);
+
+/* Dispatch of rank `rank`'s tokens: x device bf16 [S][H], topk_idx [S][K];
+ * row q*C_max + row of the plan goes to recv_peers[q] + row*H; dest [S][K]
+ * written with the flat rows. */
+MOONEP_API int moonep_ep_dispatch(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *x,
+                                  const int32_t *topk_idx, void *const *recv_peers, int32_t *dest, void *stream);
+
+/* Combine of rank `rank`'s tokens: out [S][H] from y_peers[q] (rank q's
+ * expert outputs [C_max][H]), dest and topk_w [S][K] of this rank; the
+ * arithmetic of moonep_combine. */
+MOONEP_API int moonep_ep_combine(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *y_peers,
+                                 const int32_t *dest, const float *topk_w, void *out, void *stream);
+
+/* Prefetch into rank `rank`'s slots: w_slot [B][elems] (bf16); slot b of
+ * the rank gets expert e's weights from w_home_peers[e / L] + (e % L)*elems. */
+MOONEP_API int moonep_ep_prefetch(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *w_home_peers,
+                                  void *w_slot, int64_t elems_per_expert, void *stream);
+
+/* reduce_grad for rank `rank`'s own experts: g_home [L][elems] (fp32) of
+ * this rank; each replica is read from and cleared in
+ * g_rep_peers[receiver] + slot*elems, added in ascending receiver order. */
+MOONEP_API int moonep_ep_reduce_grad(const moonep_cfg_t *cfg, int32_t rank, void *ws, float *g_home,
+                                     void *const *g_rep_peers, int64_t elems_per_expert, void *stream);
+
 /* Upper bound on polls of every bounded device wait (default 1 << 22).  A
  * wait that runs out sets MOONEP_ST_TIMEOUT and the kernel returns. */
 MOONEP_API int moonep_set_wait_limit(int64_t polls);

@@ -428,6 +428,225 @@ int moonep_reduce_grad(const moonep_cfg_t *cfg, void *ws, float *g_home, float *
     return MOONEP_OK;
 }
 
+// ---------------------------------------------------------------------------
+// expert parallelism: one rank's calls
+// ---------------------------------------------------------------------------
+
+static int check_rank(const moonep_cfg_t *cfg, int32_t rank) {
+    if (rank < 0 || rank >= cfg->R) return fail(MOONEP_ERR_ARG, "rank=%d outside [0, R=%d)", rank, cfg->R);
+    return MOONEP_OK;
+}
+
+int moonep_ep_ws_layout(const moonep_cfg_t *cfg, moonep_ws_layout_t *out) {
+    TRY(check_cfg(cfg));
+    if (!out) return fail(MOONEP_ERR_ARG, "out is NULL");
+    compute_layout_tokens(*cfg, cfg->S, *out);
+    return MOONEP_OK;
+}
+
+size_t moonep_ep_workspace_bytes(const moonep_cfg_t *cfg) {
+    if (check_cfg(cfg) != MOONEP_OK) return 0;
+    moonep_ws_layout_t l;
+    compute_layout_tokens(*cfg, cfg->S, l);
+    return (size_t)l.words * 4;
+}
+
+// the plan kernel in one of its expert-parallel modes
+static int ep_plan_launch(const moonep_cfg_t *cfg, int32_t mode, int32_t flags, int32_t rank, const int32_t *ids,
+                          void *ws, int32_t *counts_out, const int32_t *counts_all, void *stream) {
+    const int N = cfg->R * cfg->L;
+    DeviceInfo *d = nullptr;
+    TRY(device_info(N, &d));
+    PlanParams p{};
+    p.cfg = *cfg;
+    p.flags = flags;
+    p.N = N;
+    p.T = cfg->S;
+    compute_layout_tokens(*cfg, cfg->S, p.lay);
+    p.Q = p.lay.n_ranges;
+    const int64_t rpb = p.lay.n_blocks > 0 ? (p.Q + p.lay.n_blocks - 1) / p.lay.n_blocks : 0;
+    if ((size_t)(rpb * N) * sizeof(int) > d->plan_smem)
+        return fail(MOONEP_ERR_ARG, "plan: %lld ranges per block of %d experts exceed shared memory", (long long)rpb, N);
+    p.ids = ids;
+    p.ws = (int32_t *)ws;
+    p.wait_limit = g_wait_limit.load();
+    p.mode = mode;
+    p.rank = rank;
+    p.counts_out = counts_out;
+    p.counts_all = counts_all;
+    cudaError_t e = launch_plan(p, d->plan_grid, d->plan_smem, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "plan kernel launch");
+    return MOONEP_OK;
+}
+
+int moonep_ep_count(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_idx, void *ws, int32_t *counts,
+                    void *stream) {
+    TRY(check_cfg(cfg));
+    TRY(check_rank(cfg, rank));
+    TRY(check_ptr(topk_idx, 4, "topk_idx", cfg->S > 0));
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(counts, 4, "counts", true));
+    const int N = cfg->R * cfg->L;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)MOONEP_WS_HEADER_WORDS * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(header)");
+    e = cudaMemsetAsync(counts, 0, (size_t)(N + 1) * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counts)");
+    if (cfg->S == 0) {
+        DeviceInfo *d = nullptr;
+        return device_info(N, &d);
+    }
+    return ep_plan_launch(cfg, kPlanCount, 0, rank, topk_idx, ws, counts, nullptr, stream);
+}
+
+int moonep_ep_plan(const moonep_cfg_t *cfg, int32_t flags, int32_t rank, const int32_t *counts_all, void *ws,
+                   void *stream) {
+    TRY(check_cfg(cfg));
+    TRY(check_rank(cfg, rank));
+    if (flags & ~(MOONEP_PLAN_REMOTE_WEIGHTS | MOONEP_PLAN_ONE_GROUP))
+        return fail(MOONEP_ERR_ARG, "unknown plan flags 0x%x", flags);
+    if ((flags & MOONEP_PLAN_REMOTE_WEIGHTS) && (flags & MOONEP_PLAN_ONE_GROUP))
+        return fail(MOONEP_ERR_ARG, "plan flags 0x%x: remote weights and one group exclude each other", flags);
+    TRY(check_ptr(counts_all, 4, "counts_all", true));
+    TRY(check_ptr(ws, 16, "ws", true));
+    return ep_plan_launch(cfg, kPlanFromCounts, flags, rank, nullptr, ws, nullptr, counts_all, stream);
+}
+
+int moonep_ep_dispatch(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *x, const int32_t *topk_idx,
+                       void *const *recv_peers, int32_t *dest, void *stream) {
+    TRY(check_cfg(cfg));
+    TRY(check_rank(cfg, rank));
+    const int64_t T = cfg->S;
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(x, 16, "x", T > 0));
+    TRY(check_ptr(topk_idx, 4, "topk_idx", T > 0));
+    TRY(check_ptr(recv_peers, 8, "recv_peers", T > 0));
+    TRY(check_ptr(dest, 4, "dest", T > 0));
+    const int N = cfg->R * cfg->L;
+    DeviceInfo *d = nullptr;
+    TRY(device_info(N, &d));
+    if (T == 0) return MOONEP_OK;
+    DispatchParams p{};
+    p.cfg = *cfg;
+    p.N = N;
+    p.T = T;
+    compute_layout_tokens(*cfg, T, p.lay);
+    p.Q = p.lay.n_ranges;
+    p.row_bytes = (uint32_t)cfg->H * 2;
+    size_t smem = 0;
+    int ctas_per_sm = (int)((p.Q + d->sms - 1) / d->sms);
+    if (ctas_per_sm > 2) ctas_per_sm = 2;
+    cudaError_t e = dispatch_smem_config(N, p.row_bytes, ctas_per_sm < 1 ? 1 : ctas_per_sm, &p.piece_bytes, &p.npc,
+                                         &smem, true);
+    if (e != cudaSuccess) return fail(MOONEP_ERR_ARG, "dispatch: no shared-memory configuration for H=%d", cfg->H);
+    p.x = (const uint8_t *)x;
+    p.ids = topk_idx;
+    p.recv_peers = (uint8_t *const *)recv_peers;
+    p.dest = dest;
+    p.ws = (int32_t *)ws;
+    p.wait_limit = g_wait_limit.load();
+    p.ep_tag = rank + 1;
+    e = launch_dispatch(p, smem, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch kernel launch");
+    bump_generation(ws);
+    return MOONEP_OK;
+}
+
+int moonep_ep_combine(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *y_peers,
+                      const int32_t *dest, const float *topk_w, void *out, void *stream) {
+    TRY(check_cfg(cfg));
+    TRY(check_rank(cfg, rank));
+    const int64_t T = cfg->S;
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(y_peers, 8, "y_peers", T > 0));
+    TRY(check_ptr(dest, 4, "dest", T > 0));
+    TRY(check_ptr(topk_w, 4, "topk_w", T > 0));
+    TRY(check_ptr(out, 16, "out", T > 0));
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (T == 0) return MOONEP_OK;
+    CombineParams p{};
+    p.cfg = *cfg;
+    p.T = T;
+    p.hv = cfg->H / 8;
+    size_t smem = 0;
+    if (combine_config(cfg->K, p.hv, &p.chunk_bytes, &p.upt, &p.stages, &smem, true) != cudaSuccess)
+        return fail(MOONEP_ERR_ARG, "combine: no shared-memory configuration for K=%d H=%d", cfg->K, cfg->H);
+    p.units = T * p.upt;
+    p.rows_total = (int64_t)cfg->R * cfg->C_max;
+    p.y = nullptr;
+    p.y_peers = (const uint8_t *const *)y_peers;
+    p.dest = dest;
+    p.w = topk_w;
+    p.out = (uint4 *)out;
+    p.ws = (int32_t *)ws;
+    p.wait_limit = g_wait_limit.load();
+    p.ep_tag = rank + 1;
+    int64_t grid = d->combine_grid;
+    if (grid > p.units) grid = p.units;
+    if (grid < 1) grid = 1;
+    cudaError_t e = launch_combine(p, (int)grid, smem, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+    bump_generation(ws);
+    return MOONEP_OK;
+}
+
+int moonep_ep_prefetch(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *w_home_peers, void *w_slot,
+                       int64_t elems_per_expert, void *stream) {
+    TRY(check_cfg(cfg));
+    TRY(check_rank(cfg, rank));
+    if (elems_per_expert <= 0 || (elems_per_expert % 8) != 0)
+        return fail(MOONEP_ERR_ARG, "elems_per_expert=%lld must be a positive multiple of 8",
+                    (long long)elems_per_expert);
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(w_home_peers, 8, "w_home_peers", true));
+    TRY(check_ptr(w_slot, 16, "w_slot", cfg->B > 0));
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (cfg->B == 0) return MOONEP_OK;
+    CopyParams p{};
+    p.cfg = *cfg;
+    p.vecs = elems_per_expert * 2 / 16;
+    p.src = nullptr;
+    p.dst = (uint4 *)w_slot;
+    p.ws = (int32_t *)ws;
+    compute_layout_tokens(*cfg, cfg->S, p.lay);
+    p.wait_limit = g_wait_limit.load();
+    p.peers = (uint8_t *const *)w_home_peers;
+    p.ep_tag = rank + 1;
+    cudaError_t e = launch_prefetch(p, d->sms, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "prefetch kernel launch");
+    return MOONEP_OK;
+}
+
+int moonep_ep_reduce_grad(const moonep_cfg_t *cfg, int32_t rank, void *ws, float *g_home, void *const *g_rep_peers,
+                          int64_t elems_per_expert, void *stream) {
+    TRY(check_cfg(cfg));
+    TRY(check_rank(cfg, rank));
+    if (elems_per_expert <= 0 || (elems_per_expert % 4) != 0)
+        return fail(MOONEP_ERR_ARG, "elems_per_expert=%lld must be a positive multiple of 4",
+                    (long long)elems_per_expert);
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(g_home, 16, "g_home", true));
+    TRY(check_ptr(g_rep_peers, 8, "g_rep_peers", cfg->B > 0));
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (cfg->B == 0) return MOONEP_OK;
+    CopyParams p{};
+    p.cfg = *cfg;
+    p.vecs = elems_per_expert * 4 / 16;
+    p.src = (const uint4 *)g_home;
+    p.dst = nullptr;
+    p.ws = (int32_t *)ws;
+    compute_layout_tokens(*cfg, cfg->S, p.lay);
+    p.wait_limit = g_wait_limit.load();
+    p.peers = (uint8_t *const *)g_rep_peers;
+    p.ep_tag = rank + 1;
+    cudaError_t e = launch_reduce_grad(p, d->sms, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "reduce_grad kernel launch");
+    return MOONEP_OK;
+}
+
 int moonep_plan_read(const moonep_cfg_t *cfg, const void *ws, moonep_plan_info_t *info, int32_t *host_tables,
                      void *stream) {
     TRY(check_cfg(cfg));

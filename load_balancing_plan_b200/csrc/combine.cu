@@ -69,11 +69,15 @@ __device__ __forceinline__ uint4 pack8(const float *acc) {
     return v;
 }
 
+// kEp: expert parallelism.  The tokens are one rank's (T = S) and a source
+// row lives in the expert-output buffer of its rank, reached through a table
+// of peer pointers kept in shared memory after the weights.
+template <bool kEp>
 __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_constant__ CombineParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     int32_t *ws = p.ws;
     if (block_status_failed(ws)) return;
-    if (!cfg_matches(ws, p.cfg, num_ranges(p.T, (int64_t)p.cfg.R * p.cfg.L))) {
+    if (!cfg_matches(ws, p.cfg, num_ranges(p.T, (int64_t)p.cfg.R * p.cfg.L), p.ep_tag)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
     }
@@ -86,8 +90,11 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
     uint64_t *empty = full + kMaxStages;
     StageInfo *info = reinterpret_cast<StageInfo *>(empty + kMaxStages);
     float *sw = reinterpret_cast<float *>(info + kMaxStages);  // [kMaxStages][kMaxK]
+    const uint8_t **s_peer = reinterpret_cast<const uint8_t **>(sw + kMaxStages * kMaxK);  // [R] (kEp)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (kEp)
+        for (int r = threadIdx.x; r < p.cfg.R; r += kThreads) s_peer[r] = p.y_peers[r];
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
@@ -155,12 +162,17 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
             __syncwarp();
             if (valid) {
                 uint8_t *st = stages + (size_t)s * stage_bytes;
-                if (lane < K)
-                    bulk_g2s(st + (size_t)lane * CH, y + (int64_t)dk * row_bytes + (int64_t)c * CH, bytes, &full[s],
-                             pol);
-                if (lane + 32 < K)
-                    bulk_g2s(st + (size_t)(lane + 32) * CH, y + (int64_t)dk2 * row_bytes + (int64_t)c * CH, bytes,
-                             &full[s], pol);
+                const int64_t Cm = p.cfg.C_max;
+                if (lane < K) {
+                    const uint8_t *row = kEp ? s_peer[dk / Cm] + (int64_t)(dk % Cm) * row_bytes
+                                             : y + (int64_t)dk * row_bytes;
+                    bulk_g2s(st + (size_t)lane * CH, row + (int64_t)c * CH, bytes, &full[s], pol);
+                }
+                if (lane + 32 < K) {
+                    const uint8_t *row = kEp ? s_peer[dk2 / Cm] + (int64_t)(dk2 % Cm) * row_bytes
+                                             : y + (int64_t)dk2 * row_bytes;
+                    bulk_g2s(st + (size_t)(lane + 32) * CH, row + (int64_t)c * CH, bytes, &full[s], pol);
+                }
             }
         }
         // every copy issued must land before the CTA exits
@@ -206,14 +218,14 @@ __global__ void __launch_bounds__(kThreads, 1) combine_kernel(const __grid_const
 
 }  // namespace
 
-const void *combine_kernel_ptr() { return (const void *)combine_kernel; }
+const void *combine_kernel_ptr() { return (const void *)combine_kernel<false>; }
 
 // chunk: the row split into equal pieces (multiples of 16 bytes) of at most
 // MOONEP_COMBINE_CHUNK bytes, fewer when K is large (K*chunk <= 8 chunks);
 // stages fill MOONEP_COMBINE_SMEM_KB of shared memory (at most kMaxStages).
 // Large bulk copies matter: 8 KB copies move about 1.5x the bytes per second
 // of 4 KB ones on B200.
-cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages, size_t *smem) {
+cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages, size_t *smem, bool ep) {
     if (K < 1 || K > kMaxK || hv < 1) return cudaErrorInvalidValue;
     uint32_t cap = MOONEP_COMBINE_CHUNK;
     while ((uint32_t)K * cap > 8u * MOONEP_COMBINE_CHUNK && cap > 512) cap >>= 1;
@@ -221,7 +233,8 @@ cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages
     const int n = (int)((row + cap - 1) / cap);
     const uint32_t ch = (((row + n - 1) / n) + 15) & ~15u;
     const size_t stage = (size_t)K * ch;
-    const size_t fixed = 2 * kMaxStages * 8 + kMaxStages * sizeof(StageInfo) + kMaxStages * kMaxK * 4 + 128;
+    const size_t fixed = 2 * kMaxStages * 8 + kMaxStages * sizeof(StageInfo) + kMaxStages * kMaxK * 4 + 128 +
+                         (ep ? 64 * 8 : 0);
     int ns = (int)((MOONEP_COMBINE_SMEM_KB * 1024 - fixed) / stage);
     if (ns > kMaxStages) ns = kMaxStages;
     if (ns < 2) return cudaErrorInvalidValue;
@@ -233,10 +246,17 @@ cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages
 }
 
 cudaError_t launch_combine(const CombineParams &p, int grid, size_t smem, cudaStream_t s) {
+    if (p.y_peers) {
+        static std::atomic<size_t> smem_set_ep[64];
+        cudaError_t err = set_smem_limit((const void *)combine_kernel<true>, smem, smem_set_ep);
+        if (err != cudaSuccess) return err;
+        combine_kernel<true><<<grid, kThreads, smem, s>>>(p);
+        return cudaGetLastError();
+    }
     static std::atomic<size_t> smem_set[64];
-    cudaError_t err = set_smem_limit((const void *)combine_kernel, smem, smem_set);
+    cudaError_t err = set_smem_limit((const void *)combine_kernel<false>, smem, smem_set);
     if (err != cudaSuccess) return err;
-    combine_kernel<<<grid, kThreads, smem, s>>>(p);
+    combine_kernel<false><<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 

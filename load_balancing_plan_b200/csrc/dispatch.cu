@@ -134,6 +134,12 @@ __device__ __forceinline__ void init_counters(const DispatchParams &p, int32_t *
     }
 }
 
+// kEp: expert parallelism.  The CTA's tokens are one rank's (T = S), their
+// copy numbers start after the lower ranks' copies (the plan's blk prefix
+// carries them), and a row goes to the receive buffer of its destination
+// rank through a table of peer pointers (kept in shared memory after the
+// counters) instead of one buffer [R][C_max][H].
+template <bool kEp>
 __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__ DispatchParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int lane = threadIdx.x;
@@ -141,7 +147,7 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
     const int64_t q = blockIdx.x;
     if (block_status_failed(ws)) return;
     // a tables-only copy has no base/blk scratch: refuse it before reading them
-    if (!cfg_matches(ws, p.cfg, p.Q) || tables_only(ws)) {
+    if (!cfg_matches(ws, p.cfg, p.Q, p.ep_tag) || tables_only(ws)) {
         if (lane == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
     }
@@ -150,6 +156,10 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
     const int64_t t0 = range_begin(q, p.T, p.Q), t1 = range_begin(q + 1, p.T, p.Q);
     const int64_t ntok = t1 - t0;
     const int64_t g0 = t0 * K, nids = ntok * K;
+    uint8_t **s_peer = reinterpret_cast<uint8_t **>(sm.ctr + ((p.N + 1) & ~1));
+    if (kEp)
+        for (int r = lane; r < p.cfg.R; r += 32) s_peer[r] = p.recv_peers[r];
+    const int64_t Cm = p.cfg.C_max;
     init_counters(p, sm.ctr, q, g0, nids, lane, 32);
     if (lane == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.bars[s], 1);
@@ -207,7 +217,9 @@ __global__ void __launch_bounds__(32, 1) dispatch_kernel(const __grid_constant__
                     for (int k = 0; k < K; ++k) {
                         const int d = sm.ring[(i * K + k) % kRing];
                         if (d >= 0) {
-                            uint8_t *dst = p.recv + (int64_t)d * p.row_bytes + (int64_t)pc * p.piece_bytes;
+                            uint8_t *row = kEp ? s_peer[d / Cm] + (int64_t)(d % Cm) * p.row_bytes
+                                               : p.recv + (int64_t)d * p.row_bytes;
+                            uint8_t *dst = row + (int64_t)pc * p.piece_bytes;
                             if (MOONEP_DISPATCH_HINTS & 2)
                                 bulk_s2g(dst, src, bytes, pol);
                             else
@@ -372,12 +384,13 @@ __global__ void __launch_bounds__(32 * (1 + kLoaderWarps), 1)
 
 }  // namespace
 
-// Shared memory: kStages pieces + barriers + ring + N counters, sized so that
-// `ctas_per_sm` CTAs fit one SM (227 KB usable per SM on sm_100).
+// Shared memory: kStages pieces + barriers + ring + N counters (+ the peer
+// table under expert parallelism), sized so that `ctas_per_sm` CTAs fit one
+// SM (227 KB usable per SM on sm_100).
 cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uint32_t *piece_bytes, int *npc,
-                                 size_t *smem) {
+                                 size_t *smem, bool ep) {
     const size_t budget = (size_t)(228 * 1024) / (size_t)ctas_per_sm - 1024;  // 1 KB reserved per CTA
-    const size_t fixed = (size_t)kStages * 8 + (size_t)kRing * 4 + (size_t)N * 4 + 128;
+    const size_t fixed = (size_t)kStages * 8 + (size_t)kRing * 4 + (size_t)N * 4 + 128 + (ep ? 8 + 64 * 8 : 0);
     if (budget <= fixed) return cudaErrorInvalidValue;
     size_t maxp = (budget - fixed) / kStages;
     if (maxp > kMaxPiece) maxp = kMaxPiece;
@@ -397,6 +410,13 @@ cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uin
 }
 
 cudaError_t launch_dispatch(const DispatchParams &p, size_t smem, cudaStream_t s) {
+    if (p.recv_peers) {
+        static std::atomic<size_t> smem_set_ep[64];
+        cudaError_t err = set_smem_limit((const void *)dispatch_kernel<true>, smem, smem_set_ep);
+        if (err != cudaSuccess) return err;
+        dispatch_kernel<true><<<(unsigned)p.Q, 32, smem, s>>>(p);
+        return cudaGetLastError();
+    }
     if (MOONEP_DISPATCH_LOADER) {
         static std::atomic<size_t> smem_set2[64];
         const size_t smem2 = smem + (size_t)kStages * 8;  // the "empty" barriers
@@ -406,9 +426,9 @@ cudaError_t launch_dispatch(const DispatchParams &p, size_t smem, cudaStream_t s
         return cudaGetLastError();
     }
     static std::atomic<size_t> smem_set[64];
-    cudaError_t err = set_smem_limit((const void *)dispatch_kernel, smem, smem_set);
+    cudaError_t err = set_smem_limit((const void *)dispatch_kernel<false>, smem, smem_set);
     if (err != cudaSuccess) return err;
-    dispatch_kernel<<<(unsigned)p.Q, 32, smem, s>>>(p);
+    dispatch_kernel<false><<<(unsigned)p.Q, 32, smem, s>>>(p);
     return cudaGetLastError();
 }
 

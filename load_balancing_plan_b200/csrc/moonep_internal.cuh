@@ -28,6 +28,7 @@ enum : int {
     HDR_BAR_COUNT = 16,
     HDR_BAR_GEN = 17,
     HDR_TABLES_ONLY = 18,  // kTablesOnlyMark: a copy of the header and tables without the dispatch scratch
+    HDR_EP = 19,           // 0: the workspace of a single-GPU plan; rank + 1: of expert-parallel rank `rank`
     HDR_TOTAL_SPILL = 20,
     HDR_PEND = 21,
 };
@@ -102,9 +103,11 @@ __host__ __device__ inline int64_t max_pieces(int R, int L, int B) {
     return (int64_t)R * L + R;
 }
 
-// Fills the layout; returns false if the configuration is out of range.
-__host__ __device__ inline void compute_layout(const moonep_cfg_t &c, moonep_ws_layout_t &l) {
-    const int64_t N = (int64_t)c.R * c.L, R = c.R, T = (int64_t)c.R * c.S;
+// Fills the layout for a plan whose dispatch numbers the copies of T tokens:
+// all R*S of them on one GPU (compute_layout), or one rank's S under expert
+// parallelism, where each rank dispatches its own tokens.
+__host__ __device__ inline void compute_layout_tokens(const moonep_cfg_t &c, int64_t T, moonep_ws_layout_t &l) {
+    const int64_t N = (int64_t)c.R * c.L, R = c.R;
     const int64_t RB = (int64_t)c.R * c.B > 0 ? (int64_t)c.R * c.B : 1;
     const int64_t P = max_pieces(c.R, c.L, c.B);
     const int64_t NR = 2 * N + P;
@@ -153,9 +156,21 @@ __host__ __device__ inline void compute_layout(const moonep_cfg_t &c, moonep_ws_
     l.words = o;
 }
 
+__host__ __device__ inline void compute_layout(const moonep_cfg_t &c, moonep_ws_layout_t &l) {
+    compute_layout_tokens(c, (int64_t)c.R * c.S, l);
+}
+
 // ---------------------------------------------------------------------------
 // kernel parameter blocks
 // ---------------------------------------------------------------------------
+// plan kernel modes: the whole plan of one GPU's R*S tokens (kPlanFull);
+// under expert parallelism, first the counts of one rank's S tokens
+// (kPlanCount: histogram into counts_out, per-range scratch into ws), then,
+// once every rank's counts are gathered, the plan from them
+// (kPlanFromCounts: identical tables on every rank, and this rank's copy
+// numbers offset by the copies of the lower ranks)
+enum : int32_t { kPlanFull = 0, kPlanCount = 1, kPlanFromCounts = 2 };
+
 struct PlanParams {
     moonep_cfg_t cfg;
     int32_t flags;
@@ -165,6 +180,10 @@ struct PlanParams {
     int32_t *ws;
     moonep_ws_layout_t lay;
     int64_t wait_limit;
+    int32_t mode;              // kPlan*
+    int32_t rank;              // expert-parallel rank (kPlanCount, kPlanFromCounts)
+    int32_t *counts_out;       // kPlanCount: [N + 1] (counts, then status bits)
+    const int32_t *counts_all; // kPlanFromCounts: [R][N + 1], every rank's counts_out
 };
 
 struct DispatchParams {
@@ -181,6 +200,8 @@ struct DispatchParams {
     int32_t *ws;
     moonep_ws_layout_t lay;
     int64_t wait_limit;
+    uint8_t *const *recv_peers;  // expert parallelism: every rank's receive buffer [C_max][H] (device array of R)
+    int32_t ep_tag;              // 0, or rank + 1 under expert parallelism
 };
 
 struct CombineParams {
@@ -198,6 +219,8 @@ struct CombineParams {
     uint4 *out;
     int32_t *ws;
     int64_t wait_limit;
+    const uint8_t *const *y_peers;  // expert parallelism: every rank's expert outputs [C_max][H]
+    int32_t ep_tag;
 };
 
 struct BackwardParams {
@@ -226,6 +249,12 @@ struct CopyParams {
     uint4 *dst;
     int32_t *ws;
     moonep_ws_layout_t lay;
+    // expert parallelism (ep_tag = rank + 1): prefetch reads the home ranks'
+    // weights [L][elems] through peers and writes this rank's slots [B][elems]
+    // (dst); reduce_grad adds the receivers' replica slots [B][elems] (read
+    // and cleared through peers) into this rank's gradients [L][elems] (src)
+    uint8_t *const *peers;
+    int32_t ep_tag;
 };
 
 struct CopyOutParams {
@@ -256,11 +285,15 @@ __device__ __forceinline__ bool block_status_failed(const int32_t *ws) {
     return s_failed != 0;
 }
 
-__device__ __forceinline__ bool cfg_matches(const int32_t *ws, const moonep_cfg_t &c, int64_t Q) {
+// Whether the workspace holds a plan for this configuration, token ranges
+// and kind (ep_tag: 0 for a single-GPU plan, rank + 1 for an expert-parallel
+// rank's).
+__device__ __forceinline__ bool cfg_matches(const int32_t *ws, const moonep_cfg_t &c, int64_t Q, int32_t ep_tag = 0) {
     const int32_t *h = ws + HDR_CFG;
     return __ldcg(h + 0) == c.R && __ldcg(h + 1) == c.L && __ldcg(h + 2) == c.S &&
            __ldcg(h + 3) == c.K && __ldcg(h + 4) == c.H && __ldcg(h + 5) == c.B &&
-           __ldcg(h + 6) == c.C && __ldcg(h + 7) == c.C_max && __ldcg(ws + HDR_NRANGES) == (int32_t)Q;
+           __ldcg(h + 6) == c.C && __ldcg(h + 7) == c.C_max && __ldcg(ws + HDR_NRANGES) == (int32_t)Q &&
+           __ldcg(ws + HDR_EP) == ep_tag;
 }
 
 // A workspace whose header word HDR_TABLES_ONLY holds this value is a copy of
@@ -427,9 +460,9 @@ size_t plan_smem_bytes(int N);
 const void *plan_kernel_ptr();
 cudaError_t launch_dispatch(const DispatchParams &p, size_t smem, cudaStream_t s);
 cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uint32_t *piece_bytes,
-                                 int *npc, size_t *smem);
+                                 int *npc, size_t *smem, bool ep = false);
 cudaError_t launch_combine(const CombineParams &p, int grid, size_t smem, cudaStream_t s);
-cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages, size_t *smem);
+cudaError_t combine_config(int K, int hv, uint32_t *chunk, int *upt, int *stages, size_t *smem, bool ep = false);
 const void *combine_kernel_ptr();
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s);
 cudaError_t launch_reduce_grad(const CopyParams &p, int sms, cudaStream_t s);

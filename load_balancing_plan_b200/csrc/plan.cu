@@ -163,10 +163,11 @@ __device__ bool grid_barrier(int32_t *ws, int64_t limit) {
     return s_ok != 0;
 }
 
-// Exclusive prefix of one expert's per-range counts, in place (one warp).
-__device__ void scan_column(int32_t *col, int64_t Q) {
+// Exclusive prefix of one expert's per-range counts, in place (one warp),
+// starting from carry0.
+__device__ void scan_column(int32_t *col, int64_t Q, int carry0 = 0) {
     const int lane = threadIdx.x & 31;
-    int carry = 0;
+    int carry = carry0;
     for (int64_t q0 = 0; q0 < Q; q0 += 32 * 16) {
         int v[16];
 #pragma unroll
@@ -444,6 +445,66 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     }
 }
 
+// Expert parallelism: the plan from every rank's counts ([R][N + 1]: the
+// copies of each expert among the rank's tokens, then the rank's status
+// bits).  CTA 0 sums the columns into tokens_per_expert (cnt) and plans
+// exactly as the single-GPU plan does, so every rank derives the same
+// tables; the other CTAs turn this rank's per-block counts into copy
+// numbers, starting each expert at the copies the lower ranks hold (copies
+// are numbered in ascending g = (r*S + s)*K + k across ranks).  A kernel of
+// its own: the single-GPU plan kernel's code stays as small as before (its
+// in-step time is bound by instruction fetches of run-once code).
+__global__ void __launch_bounds__(kPlanThreads, 1) plan_from_counts_kernel(const __grid_constant__ PlanParams p) {
+    extern __shared__ __align__(16) int sm[];
+    const int N = p.N, R = p.cfg.R;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    int32_t *ws = p.ws;
+    const moonep_ws_layout_t &lay = p.lay;
+    const int64_t NB = lay.n_blocks;
+    const int64_t row = (int64_t)N + 1;
+    if (block_status_failed(ws)) return;  // this rank's count found a bad id
+    if (gridDim.x == 1 || blockIdx.x > 0) {
+        const int gw = gridDim.x == 1 ? warp : (blockIdx.x - 1) * kWarps + warp;
+        const int nw = gridDim.x == 1 ? kWarps : (gridDim.x - 1) * kWarps;
+        for (int e = gw; e < N; e += nw) {
+            int carry = 0;
+            for (int r = 0; r < p.rank; ++r) carry += __ldg(p.counts_all + r * row + e);
+            scan_column(ws + lay.blk + (int64_t)e * NB, NB, carry);
+        }
+        if (blockIdx.x > 0) return;
+    }
+    __shared__ int s_st;
+    if (tid == 0) s_st = 0;
+    __syncthreads();
+    for (int r = tid; r < R; r += kPlanThreads) {
+        const int st = __ldg(p.counts_all + r * row + N);
+        if (st) atomicOr(&s_st, st);
+    }
+    for (int e = tid; e < N; e += kPlanThreads) {
+        int c = 0;
+        for (int r = 0; r < R; ++r) c += __ldg(p.counts_all + r * row + e);
+        sm[e] = c;
+        ws[lay.cnt + e] = c;
+    }
+    for (int64_t i = tid; i < (int64_t)N * R; i += kPlanThreads) ws[lay.alloc + i] = 0;
+    __syncthreads();
+    if (s_st & MOONEP_ST_ERROR_MASK) {
+        // a bad id on some rank: no rank plans, so no rank dispatches
+        if (tid == 0) atomicOr(ws + HDR_STATUS, s_st & MOONEP_ST_ERROR_MASK);
+        return;
+    }
+    if (tid < 8) ws[HDR_CFG + tid] = (&p.cfg.R)[tid];
+    if (tid == 0) {
+        ws[HDR_NRANGES] = (int32_t)p.Q;
+        ws[HDR_EP] = p.rank + 1;
+    }
+    __syncthreads();
+    if (N > kWarpPlannerMaxN)
+        plan_tables<kPlanThreads>(p, sm);
+    else if (warp == 0)
+        plan_tables<32>(p, sm);
+}
+
 __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_constant__ PlanParams p) {
     extern __shared__ __align__(16) int sm[];
     const int N = p.N, K = p.cfg.K;
@@ -464,6 +525,9 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     // (cnt).
     bool bad = false;
     const int64_t NB = lay.n_blocks;
+    // copies per expert: into the plan's cnt, or (counting one rank's tokens
+    // under expert parallelism) into the rank's counts_out
+    int32_t *cnt_acc = p.mode == kPlanCount ? p.counts_out : ws + lay.cnt;
     for (int64_t b = blockIdx.x; b < NB; b += gridDim.x) {
         const int64_t qa = block_first_range(b, p.Q, NB), qb = block_first_range(b + 1, p.Q, NB);
         const int nr = (int)(qb - qa);
@@ -502,11 +566,16 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
                 run += c;
             }
             ws[lay.blk + (int64_t)e * NB + b] = run;
-            if (run) atomicAdd(ws + lay.cnt + e, run);
+            if (run) atomicAdd(cnt_acc + e, run);
         }
         __syncthreads();
     }
     if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_EXPERT_ID);
+    if (p.mode == kPlanCount) {
+        // the status travels with the counts, so every rank learns of it
+        if (bad) atomicOr(p.counts_out + N, MOONEP_ST_EXPERT_ID);
+        return;
+    }
     // the allocation table is only written after the barrier: clear it now,
     // spread over the whole grid
     for (int64_t i = (int64_t)blockIdx.x * kPlanThreads + tid; i < (int64_t)N * p.cfg.R;
@@ -561,6 +630,18 @@ size_t plan_smem_bytes(int N) {
 const void *plan_kernel_ptr() { return (const void *)plan_kernel; }
 
 cudaError_t launch_plan(const PlanParams &p, int grid, size_t smem, cudaStream_t s) {
+    if (p.mode == kPlanFromCounts) {
+        static std::atomic<size_t> smem_set[64];
+        cudaError_t err = set_smem_limit((const void *)plan_from_counts_kernel, smem, smem_set);
+        if (err != cudaSuccess) return err;
+        plan_from_counts_kernel<<<grid, kPlanThreads, smem, s>>>(p);
+        return cudaGetLastError();
+    }
+    if (p.mode == kPlanCount) {
+        // no grid barrier when only counting: an ordinary launch
+        plan_kernel<<<grid, kPlanThreads, smem, s>>>(p);
+        return cudaGetLastError();
+    }
     void *args[] = {(void *)&p};
     return cudaLaunchCooperativeKernel((const void *)plan_kernel, dim3(grid), dim3(kPlanThreads), args, smem, s);
 }

@@ -7,12 +7,15 @@
 // clears the used slots; "The Busiest Rank Sets Your Step Time", flowchart:
 // weight prefetch, reduce_grad).
 //
-// Both walk a list the plan leaves in the workspace (the replica pieces, and
-// the experts that have at least one) and split every expert into 32 KB
-// chunks.  prefetch moves each chunk with TMA bulk copies (one warp per SM,
-// a pipeline of shared-memory stages); reduce_grad hands chunks to a
-// persistent grid whose threads keep two 16-byte vectors of the home gradient
-// and up to four replicas each in flight before adding them in order.
+// Both walk lists the plan leaves in the workspace (the replica pieces, and
+// the experts that have at least one).  prefetch moves 32 KB chunks with TMA
+// bulk copies (one warp per SM, a pipeline of shared-memory stages).
+// reduce_grad deals units of a few KB of one expert's gradient to warps; each
+// warp keeps two units' loads in flight (the next unit's home and replica
+// vectors are loaded before the current unit is added and stored).  Under
+// expert parallelism (kEp) both reach the other ranks' buffers through a
+// table of peer pointers: prefetch reads the home rank's weights,
+// reduce_grad reads and clears the receivers' replica gradients.
 #include "moonep_internal.cuh"
 
 namespace moonep {
@@ -43,11 +46,17 @@ static_assert(kPfStages - kPfAhead - 1 >= 0, "stage reuse needs an older store g
 // the units (piece, 32 KB chunk) of this CTA: bulk load global -> shared
 // (mbarrier), bulk store shared -> global (bulk groups), kPfAhead loads in
 // flight, a stage reused once its store has read it.  Every wait is bounded.
+// The pieces are those with a slot: all of them on one GPU, this rank's
+// (kEp; they are contiguous in the plan's slot-piece list, which is
+// receiver-major) under expert parallelism, where the source is the home
+// rank's weights [L][elems] through the peer table and the destination the
+// rank's own slots [B][elems].
+template <bool kEp>
 __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__ CopyParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     int32_t *ws = p.ws;
     if (block_status_failed(ws)) return;
-    if (!cfg_matches(ws, p.cfg, p.lay.n_ranges)) {
+    if (!cfg_matches(ws, p.cfg, p.lay.n_ranges, p.ep_tag)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
     }
@@ -57,14 +66,22 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
     fence_mbar_init();
     fence_proxy_async_smem();
 
-    const int64_t P = __ldcg(ws + HDR_NSLOT);  // pieces with a slot (all, under the headroom rule)
+    const int B = p.cfg.B, L = p.cfg.L;
+    // slotted pieces handled: [sp0, sp0 + P) of the slot-piece list
+    int64_t sp0 = 0, P = 0;
+    if (kEp) {
+        const int rank = p.ep_tag - 1;
+        for (int r = 0; r < rank; ++r) sp0 += __ldg(ws + p.lay.slots_used + r);
+        P = __ldg(ws + p.lay.slots_used + rank);
+    } else {
+        P = __ldcg(ws + HDR_NSLOT);  // pieces with a slot (all, under the headroom rule)
+    }
     const int64_t bytes_per = p.vecs * 16;
     const int64_t cps = (bytes_per + kPfChunk - 1) / kPfChunk;
     const int64_t units = P * cps;
     const int64_t u0 = (int64_t)blockIdx.x * units / gridDim.x;
     const int64_t u1 = (int64_t)(blockIdx.x + 1) * units / gridDim.x;
     const int64_t n = u1 - u0;
-    const int B = p.cfg.B;
     const uint8_t *src_base = reinterpret_cast<const uint8_t *>(p.src);
     uint8_t *dst_base = reinterpret_cast<uint8_t *>(p.dst);
     const uint64_t pol = policy_evict_first();
@@ -74,14 +91,14 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
         if (it < n) {
             const int64_t u = u0 + it;
             const int64_t sp = u / cps, c = u - sp * cps;
-            const int gp = __ldg(ws + p.lay.slot_piece + sp);
+            const int gp = __ldg(ws + p.lay.slot_piece + sp0 + sp);
             const int e = __ldg(ws + p.lay.rep_expert + gp);
+            const uint8_t *src = kEp ? p.peers[e / L] + (int64_t)(e % L) * bytes_per : src_base + (int64_t)e * bytes_per;
             const uint32_t bytes = (uint32_t)min((int64_t)kPfChunk, bytes_per - c * kPfChunk);
             const int s = (int)(it % kPfStages);
             if (it >= kPfStages) bulk_wait_read<kPfStages - kPfAhead - 1>();
             mbar_arrive_expect_tx(&bars[s], bytes);
-            bulk_g2s(smem + (size_t)s * kPfChunk, src_base + (int64_t)e * bytes_per + c * kPfChunk, bytes, &bars[s],
-                     pol);
+            bulk_g2s(smem + (size_t)s * kPfChunk, src + c * kPfChunk, bytes, &bars[s], pol);
             issued = it + 1;
         }
         const int64_t j = it - kPfAhead;
@@ -96,8 +113,9 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
             if (fail) break;
             const int64_t u = u0 + j;
             const int64_t sp = u / cps, c = u - sp * cps;
-            const int gp = __ldg(ws + p.lay.slot_piece + sp);
-            const int64_t slot = (int64_t)__ldg(ws + p.lay.rep_recv + gp) * B + __ldg(ws + p.lay.rep_slot + gp);
+            const int gp = __ldg(ws + p.lay.slot_piece + sp0 + sp);
+            const int64_t slot = kEp ? (int64_t)__ldg(ws + p.lay.rep_slot + gp)
+                                     : (int64_t)__ldg(ws + p.lay.rep_recv + gp) * B + __ldg(ws + p.lay.rep_slot + gp);
             const uint32_t bytes = (uint32_t)min((int64_t)kPfChunk, bytes_per - c * kPfChunk);
             if (MOONEP_PREFETCH_STORE_HINT)
                 bulk_s2g(dst_base + slot * bytes_per + c * kPfChunk, smem + (size_t)s * kPfChunk, bytes, pol);
@@ -127,11 +145,10 @@ __device__ __forceinline__ void add4(float4 &a, const float4 &b) {
     a.w = __fadd_rn(a.w, b.w);
 }
 
-// g_home[e] = (((g_home[e] + rep_1) + rep_2) + ...) in ascending receiver
-// order (the plan's piece order within an expert), then rep_i = 0.  A
-// persistent grid strides over the units (replicated expert, 32 KB chunk);
-// consecutive units of a CTA are a grid apart, so every CTA sees every
-// expert and the experts' different replica counts even out.
+// reduce_grad, CTA form (MOONEP_REDUCE_GRAD_CTA=1; one GPU only; kept to
+// reproduce the comparison with the warp form): the same sums, a persistent
+// grid striding over the units (replicated expert, 32 KB chunk), thread 0
+// of each CTA collecting the unit's replica slots between two barriers.
 __global__ void __launch_bounds__(kThreads) reduce_grad_kernel(const __grid_constant__ CopyParams p) {
     int32_t *ws = p.ws;
     if (block_status_failed(ws)) return;
@@ -202,23 +219,259 @@ __global__ void __launch_bounds__(kThreads) reduce_grad_kernel(const __grid_cons
     }
 }
 
+
+// reduce_grad: g_home[e] = (((g_home[e] + rep_1) + rep_2) + ...) in ascending
+// receiver order (the plan's piece order within an expert), then rep_i = 0.
+// Each CTA first copies the plan's lists (replicated experts, their piece
+// ranges, and every piece's slot) into shared memory once.  Then every warp
+// strides over units of 32 x kRgVecs 16-byte vectors of one replicated
+// expert, unit u going to warp u mod (warps in the grid), so the warps in
+// flight at any moment work on neighbouring stretches of the same
+// gradients.  A warp loads its next unit (home vectors and the first
+// kRgBatch replicas) before it adds and stores the current one, so two
+// units' loads are in flight per warp; no barrier separates units.  On the
+// mid workload (3 replicated experts, 8 replicas, 1.29 GB) this runs 207 us
+// against 230 us for the CTA form; the form without the look-ahead unit
+// (8 vectors per lane, 2 replicas per batch) ran 210 us.
+//
+// kEp: expert parallelism.  Only the rank's own experts (a contiguous
+// stretch of the ascending replicated-expert list), their home gradients
+// [L][elems] local, each replica read and cleared through the peer table.
+#ifndef MOONEP_RG_VECS
+#define MOONEP_RG_VECS 6
+#endif
+#ifndef MOONEP_RG_BATCH
+#define MOONEP_RG_BATCH 1
+#endif
+#ifndef MOONEP_RG_THREADS
+#define MOONEP_RG_THREADS 256
+#endif
+#ifndef MOONEP_RG_MINB
+#define MOONEP_RG_MINB 1  // CTAs per SM the register budget is set for
+#endif
+constexpr int kRgVecs = MOONEP_RG_VECS;
+constexpr int kRgBatch = MOONEP_RG_BATCH;
+constexpr int kRgThreads = MOONEP_RG_THREADS;
+constexpr int kRgUnit = 32 * kRgVecs;
+
+template <bool kEp>
+__global__ void __launch_bounds__(kRgThreads, MOONEP_RG_MINB) reduce_grad_pipe_kernel(const __grid_constant__ CopyParams p) {
+    extern __shared__ __align__(16) int rg_sm[];
+    int32_t *ws = p.ws;
+    if (block_status_failed(ws)) return;
+    if (!cfg_matches(ws, p.cfg, p.lay.n_ranges, p.ep_tag)) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
+        return;
+    }
+    const int N = p.cfg.R * p.cfg.L, B = p.cfg.B, L = p.cfg.L;
+    const int nrx_all = __ldcg(ws + HDR_NRX);
+    const int P = __ldcg(ws + HDR_NREP);
+    // [N] expert, [N] first piece, [N] end piece, [max_pieces] slot, then
+    // (kEp) the peer table, 8-byte aligned
+    int *s_e = rg_sm, *s_pb = rg_sm + N, *s_pe = rg_sm + 2 * N, *s_slot = rg_sm + 3 * N;
+    float4 **s_peer = reinterpret_cast<float4 **>(rg_sm + ((3 * N + p.lay.max_pieces + 1) & ~1));
+    // the replicated experts handled: all, or (kEp) the rank's own, which
+    // form the stretch [x0, x0 + nrx) of the ascending list
+    int x0 = 0, nrx = nrx_all;
+    if (kEp) {
+        const int lo = (p.ep_tag - 1) * L, hi = lo + L;
+        int below = 0, mine = 0;
+        for (int b0 = 0; b0 < nrx_all; b0 += kRgThreads) {
+            const int x = b0 + threadIdx.x;
+            const int e = x < nrx_all ? __ldcg(ws + p.lay.rx_expert + x) : N;
+            below += __syncthreads_count(e < lo);
+            mine += __syncthreads_count(e >= lo && e < hi);
+        }
+        x0 = below;
+        nrx = mine;
+        for (int r = threadIdx.x; r < p.cfg.R; r += kRgThreads) s_peer[r] = reinterpret_cast<float4 *>(p.peers[r]);
+    }
+    for (int x = threadIdx.x; x < nrx; x += kRgThreads) {
+        const int e = __ldcg(ws + p.lay.rx_expert + x0 + x);
+        s_e[x] = kEp ? e - (p.ep_tag - 1) * L : e;  // row of the home gradient array
+        s_pb[x] = __ldcg(ws + p.lay.rep_ptr + e);
+        s_pe[x] = __ldcg(ws + p.lay.rep_ptr + e + 1);
+    }
+    // slot of every piece as receiver * B + slot; -1: no slot (remote
+    // weights: such a piece has no replica gradient)
+    for (int q = threadIdx.x; q < P; q += kRgThreads) {
+        const int sl = __ldcg(ws + p.lay.rep_slot + q);
+        s_slot[q] = sl >= 0 ? __ldcg(ws + p.lay.rep_recv + q) * B + sl : -1;
+    }
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    constexpr int kWarpsPerCta = kRgThreads / 32;
+    const int64_t gw = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    const int64_t tw = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t vecs = p.vecs;
+    const int64_t upe = (vecs + kRgUnit - 1) / kRgUnit;
+    const int64_t units = (int64_t)nrx * upe;
+    float4 *g_home = reinterpret_cast<float4 *>(const_cast<uint4 *>(p.src));
+    float4 *g_rep = reinterpret_cast<float4 *>(p.dst);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto replica = [&](int sl) -> float4 * {
+        return kEp ? s_peer[sl / B] + (int64_t)(sl % B) * vecs : g_rep + (int64_t)sl * vecs;
+    };
+
+    struct Unit {
+        int64_t off;
+        int e, pb, pe;
+    };
+    auto meta = [&](int64_t u) {
+        Unit m;
+        const int x = (int)(u / upe);
+        m.off = (u - (int64_t)x * upe) * kRgUnit + lane;
+        m.e = s_e[x];
+        m.pb = s_pb[x];
+        m.pe = s_pe[x];
+        return m;
+    };
+    auto load_batch = [&](const Unit &m, int q0, float4 (&r)[kRgBatch][kRgVecs], int (&sl)[kRgBatch]) {
+#pragma unroll
+        for (int qq = 0; qq < kRgBatch; ++qq) {
+            sl[qq] = q0 + qq < m.pe ? s_slot[q0 + qq] : -1;
+            const float4 *rp = replica(sl[qq] < 0 ? 0 : sl[qq]);
+#pragma unroll
+            for (int v = 0; v < kRgVecs; ++v) {
+                const int64_t i = m.off + 32 * v;
+                r[qq][v] = (sl[qq] >= 0 && i < vecs) ? __ldcs(rp + i) : z;
+            }
+        }
+    };
+    auto add_batch = [&](float4 (&h)[kRgVecs], float4 (&r)[kRgBatch][kRgVecs], int (&sl)[kRgBatch]) {
+#pragma unroll
+        for (int qq = 0; qq < kRgBatch; ++qq)
+            if (sl[qq] >= 0) {
+#pragma unroll
+                for (int v = 0; v < kRgVecs; ++v) add4(h[v], r[qq][v]);
+            }
+    };
+    auto load = [&](const Unit &m, float4 (&h)[kRgVecs], float4 (&r)[kRgBatch][kRgVecs], int (&sl)[kRgBatch]) {
+        const float4 *home = g_home + (int64_t)m.e * vecs;
+#pragma unroll
+        for (int v = 0; v < kRgVecs; ++v) {
+            const int64_t i = m.off + 32 * v;
+            h[v] = i < vecs ? __ldcs(home + i) : z;
+        }
+        load_batch(m, m.pb, r, sl);
+    };
+    auto finish = [&](const Unit &m, float4 (&h)[kRgVecs], float4 (&r)[kRgBatch][kRgVecs], int (&sl)[kRgBatch]) {
+        add_batch(h, r, sl);
+        // replicas beyond the first batch: loaded and added here
+        for (int q0 = m.pb + kRgBatch; q0 < m.pe; q0 += kRgBatch) {
+            load_batch(m, q0, r, sl);
+            add_batch(h, r, sl);
+        }
+        float4 *home = g_home + (int64_t)m.e * vecs;
+#pragma unroll
+        for (int v = 0; v < kRgVecs; ++v) {
+            const int64_t i = m.off + 32 * v;
+            if (i < vecs) __stcs(home + i, h[v]);
+        }
+        for (int q = m.pb; q < m.pe; ++q) {
+            const int sq = s_slot[q];
+            if (sq < 0) continue;
+            float4 *rp = replica(sq);
+#pragma unroll
+            for (int v = 0; v < kRgVecs; ++v) {
+                const int64_t i = m.off + 32 * v;
+                if (i < vecs) __stcs(rp + i, z);
+            }
+        }
+    };
+
+    float4 ha[kRgVecs], ra[kRgBatch][kRgVecs], hb[kRgVecs], rb[kRgBatch][kRgVecs];
+    int sla[kRgBatch], slb[kRgBatch];
+    if (gw >= units) return;
+    Unit ma = meta(gw);
+    load(ma, ha, ra, sla);
+    for (int64_t u = gw; u < units; u += 2 * tw) {
+        const bool has_b = u + tw < units;
+        Unit mb;
+        if (has_b) {
+            mb = meta(u + tw);
+            load(mb, hb, rb, slb);
+        }
+        finish(ma, ha, ra, sla);
+        if (!has_b) break;
+        if (u + 2 * tw < units) {
+            ma = meta(u + 2 * tw);
+            load(ma, ha, ra, sla);
+        }
+        finish(mb, hb, rb, slb);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s) {
     const size_t smem = (size_t)kPfStages * kPfChunk + kPfStages * 8;
+    if (p.peers) {
+        static std::atomic<size_t> smem_set_ep[64];
+        cudaError_t err = set_smem_limit((const void *)prefetch_kernel<true>, smem, smem_set_ep);
+        if (err != cudaSuccess) return err;
+        prefetch_kernel<true><<<grid, 32, smem, s>>>(p);
+        return cudaGetLastError();
+    }
     static std::atomic<size_t> smem_set[64];
-    cudaError_t err = set_smem_limit((const void *)prefetch_kernel, smem, smem_set);
+    cudaError_t err = set_smem_limit((const void *)prefetch_kernel<false>, smem, smem_set);
     if (err != cudaSuccess) return err;
-    prefetch_kernel<<<grid, 32, smem, s>>>(p);
+    prefetch_kernel<false><<<grid, 32, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+#ifndef MOONEP_REDUCE_GRAD_CTA
+#define MOONEP_REDUCE_GRAD_CTA 0
+#endif
+#ifndef MOONEP_RG_CTAS_PER_SM
+#define MOONEP_RG_CTAS_PER_SM 0  // 0: as many as fit (occupancy)
+#endif
+
+template <bool kEp>
+static cudaError_t launch_reduce_grad_pipe(const CopyParams &p, int sms, cudaStream_t s) {
+    const int N = p.cfg.R * p.cfg.L;
+    const size_t smem = (size_t)(((3 * N + p.lay.max_pieces + 1) & ~1) + 2 * 64) * sizeof(int);
+    const void *fn = (const void *)reduce_grad_pipe_kernel<kEp>;
+    static std::atomic<size_t> smem_set[64];
+    static std::atomic<int> per_sm_cache[64];
+    cudaError_t err = set_smem_limit(fn, smem, smem_set);
+    if (err != cudaSuccess) return err;
+    int per_sm = MOONEP_RG_CTAS_PER_SM;
+    if (per_sm <= 0) {
+        // CTAs per SM for this shared-memory size, cached per device (the
+        // size follows N; recomputed when it changes)
+        int dev = 0;
+        err = cudaGetDevice(&dev);
+        if (err != cudaSuccess) return err;
+        const int key = (int)(smem & 0x7fffffff);
+        static std::atomic<int> smem_key[64];
+        if (dev >= 0 && dev < 64 && smem_key[dev].load() == key && per_sm_cache[dev].load() > 0) {
+            per_sm = per_sm_cache[dev].load();
+        } else {
+            err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kRgThreads, smem);
+            if (err != cudaSuccess) return err;
+            if (per_sm < 1) per_sm = 1;
+            if (dev >= 0 && dev < 64) {
+                per_sm_cache[dev].store(per_sm);
+                smem_key[dev].store(key);
+            }
+        }
+    }
+    reduce_grad_pipe_kernel<kEp><<<sms * per_sm, kRgThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_grad(const CopyParams &p, int sms, cudaStream_t s) {
-    static std::atomic<size_t> smem_set[64];
-    cudaError_t err = set_smem_limit((const void *)reduce_grad_kernel, 0, smem_set);
-    if (err != cudaSuccess) return err;
-    reduce_grad_kernel<<<sms * 8, kThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    if (p.peers) return launch_reduce_grad_pipe<true>(p, sms, s);
+    if (MOONEP_REDUCE_GRAD_CTA) {
+        static std::atomic<size_t> smem_set[64];
+        cudaError_t err = set_smem_limit((const void *)reduce_grad_kernel, 0, smem_set);
+        if (err != cudaSuccess) return err;
+        reduce_grad_kernel<<<sms * 8, kThreads, 0, s>>>(p);
+        return cudaGetLastError();
+    }
+    return launch_reduce_grad_pipe<false>(p, sms, s);
 }
 
 }  // namespace moonep

@@ -81,6 +81,14 @@ _sig = {
     "moonep_dispatch_backward": ([_CP, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_copy_out": ([_CP, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_view_generation": ([_vp], _i64),
+    "moonep_ep_ws_layout": ([_CP, ctypes.POINTER(WsLayout)], ctypes.c_int),
+    "moonep_ep_workspace_bytes": ([_CP], ctypes.c_size_t),
+    "moonep_ep_count": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_ep_plan": ([_CP, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_ep_dispatch": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_ep_combine": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_ep_prefetch": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _i64, _vp], ctypes.c_int),
+    "moonep_ep_reduce_grad": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _i64, _vp], ctypes.c_int),
     "moonep_set_wait_limit": ([_i64], ctypes.c_int),
     "moonep_num_ranges": ([_i64, _i64], _i64),
     "moonep_last_error": ([], ctypes.c_char_p),
@@ -223,6 +231,52 @@ def moonep_prefetch(cfg, ws, w_home, w_slot, elems_per_expert, stream=None) -> N
 def moonep_reduce_grad(cfg, ws, g_home, g_rep, elems_per_expert, stream=None) -> None:
     _check(_lib.moonep_reduce_grad(ctypes.byref(cfg_of(cfg)), _p(ws), _p(g_home), _p(g_rep),
                                    int(elems_per_expert), _stream(stream)))
+
+
+# ---------------------------------------------------------------- expert parallelism
+# one rank's calls; peer tables are device arrays of R pointers (int64)
+
+def moonep_ep_ws_layout(cfg) -> dict:
+    out = WsLayout()
+    _check(_lib.moonep_ep_ws_layout(ctypes.byref(cfg_of(cfg)), ctypes.byref(out)))
+    return {n: getattr(out, n) for n in LAYOUT_FIELDS}
+
+
+def moonep_ep_workspace_bytes(cfg) -> int:
+    n = _lib.moonep_ep_workspace_bytes(ctypes.byref(cfg_of(cfg)))
+    if n == 0:
+        raise MoonepError(ERR_ARG, last_error())
+    return int(n)
+
+
+def moonep_ep_count(cfg, rank, topk_idx, ws, counts, stream=None) -> None:
+    _check(_lib.moonep_ep_count(ctypes.byref(cfg_of(cfg)), int(rank), _p(topk_idx), _p(ws), _p(counts),
+                                _stream(stream)))
+
+
+def moonep_ep_plan(cfg, flags, rank, counts_all, ws, stream=None) -> None:
+    _check(_lib.moonep_ep_plan(ctypes.byref(cfg_of(cfg)), int(flags), int(rank), _p(counts_all), _p(ws),
+                               _stream(stream)))
+
+
+def moonep_ep_dispatch(cfg, rank, ws, x, topk_idx, recv_peers, dest, stream=None) -> None:
+    _check(_lib.moonep_ep_dispatch(ctypes.byref(cfg_of(cfg)), int(rank), _p(ws), _p(x), _p(topk_idx),
+                                   _p(recv_peers), _p(dest), _stream(stream)))
+
+
+def moonep_ep_combine(cfg, rank, ws, y_peers, dest, topk_w, out, stream=None) -> None:
+    _check(_lib.moonep_ep_combine(ctypes.byref(cfg_of(cfg)), int(rank), _p(ws), _p(y_peers), _p(dest),
+                                  _p(topk_w), _p(out), _stream(stream)))
+
+
+def moonep_ep_prefetch(cfg, rank, ws, w_home_peers, w_slot, elems_per_expert, stream=None) -> None:
+    _check(_lib.moonep_ep_prefetch(ctypes.byref(cfg_of(cfg)), int(rank), _p(ws), _p(w_home_peers), _p(w_slot),
+                                   int(elems_per_expert), _stream(stream)))
+
+
+def moonep_ep_reduce_grad(cfg, rank, ws, g_home, g_rep_peers, elems_per_expert, stream=None) -> None:
+    _check(_lib.moonep_ep_reduce_grad(ctypes.byref(cfg_of(cfg)), int(rank), _p(ws), _p(g_home), _p(g_rep_peers),
+                                      int(elems_per_expert), _stream(stream)))
 
 
 def moonep_plan_read(cfg, ws, tables=False, stream=None):
