@@ -528,10 +528,18 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     // copies per expert: into the plan's cnt, or (counting one rank's tokens
     // under expert parallelism) into the rank's counts_out
     int32_t *cnt_acc = p.mode == kPlanCount ? p.counts_out : ws + lay.cnt;
+    // the range of token t is ((t + 1) * Q - 1) / T; in 32 bits when that
+    // cannot overflow (every configuration up to 2^32 / Q tokens)
+    const bool div32 = (uint64_t)(p.T + 1) * (uint64_t)p.Q < (uint64_t(1) << 32);
     for (int64_t b = blockIdx.x; b < NB; b += gridDim.x) {
         const int64_t qa = block_first_range(b, p.Q, NB), qb = block_first_range(b + 1, p.Q, NB);
         const int nr = (int)(qb - qa);
-        for (int i = tid; i < nr * N; i += kPlanThreads) sm[i] = 0;
+        {
+            const int nz = nr * N;
+            int4 *sm4 = reinterpret_cast<int4 *>(sm);
+            for (int i = tid; i < nz / 4; i += kPlanThreads) sm4[i] = make_int4(0, 0, 0, 0);
+            for (int i = (nz & ~3) + tid; i < nz; i += kPlanThreads) sm[i] = 0;
+        }
         __syncthreads();
         const int64_t i0 = range_begin(qa, p.T, p.Q) * K, i1 = range_begin(qb, p.T, p.Q) * K;
         for (int64_t b0 = i0; b0 < i1; b0 += (int64_t)kIdBatch * kPlanThreads) {
@@ -547,8 +555,9 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
                 if (i < i1) {
                     if ((unsigned)v[u] < (unsigned)N) {
                         // the range of token i / K: the last q with q*T/Q <= t
-                        const int64_t t = i / K;
-                        const int64_t q = ((t + 1) * p.Q - 1) / p.T;
+                        const int64_t t = (int64_t)((uint32_t)i / (uint32_t)K);  // i < T*K < 2^31
+                        const int64_t q = div32 ? (int64_t)(((uint32_t)(t + 1) * (uint32_t)p.Q - 1u) / (uint32_t)p.T)
+                                                : ((t + 1) * p.Q - 1) / p.T;
                         atomicAdd(&sm[(q - qa) * N + v[u]], 1);
                     } else {
                         bad = true;
@@ -559,6 +568,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
         __syncthreads();
         for (int e = tid; e < N; e += kPlanThreads) {
             int run = 0;
+#pragma unroll 8
             for (int r = 0; r < nr; ++r) {
                 // dispatch reads base[e][q] only where range q routes to e
                 const int c = sm[r * N + e];
