@@ -56,10 +56,12 @@ FALLBACK_HBM_GBS = 6650.0
 # ---------------------------------------------------------------------------
 
 def alg_bytes(cfg, n_replicas=0, n_rx=0, w_elems=0, g_elems=0):
-    """Bytes each step must move at minimum.  T = R*S tokens.
+    """Bytes each step must move at minimum.  T = R*S tokens; n_replicas =
+    replica pieces with a slot, n_rx = experts with at least one of them.
     dispatch: read x once, write K rows per token, read ids, write dest.
     combine: read K rows per token, write one, read weights and dest.
-    prefetch: read and write P*H*I bf16 per used slot.
+    prefetch: read each replicated expert's P*H*I bf16 weights once, write
+    them to every used slot.
     reduce_grad: read+write the home gradient of each replicated expert,
     read+zero every replica (fp32).  plan: read the ids."""
     T = cfg["R"] * cfg["S"]
@@ -68,7 +70,7 @@ def alg_bytes(cfg, n_replicas=0, n_rx=0, w_elems=0, g_elems=0):
     return dict(
         dispatch=T * row + T * K * row + 8 * T * K,
         combine=T * K * row + T * row + 8 * T * K,
-        prefetch=2 * 2 * w_elems * n_replicas,
+        prefetch=2 * w_elems * (n_rx + n_replicas),
         reduce_grad=4 * g_elems * (2 * n_rx + 2 * n_replicas),
         plan=4 * T * K,
     )
@@ -506,8 +508,9 @@ def layer_figures(run, steps, warmup, world, graph, peak):
     if info["status"] & mp.ST_ERROR_MASK:
         raise RuntimeError("plan failed: status 0x%x" % info["status"])
     tabs = mp.moonep_plan_read(run.cfg, run.prob.ws, tables=True)
-    n_rx = len(set(np.asarray(tabs["rep_expert"]).tolist()))
-    n_slot = int((np.asarray(tabs["rep_slot"]) >= 0).sum())   # pieces whose weights are prefetched
+    slotted = np.asarray(tabs["rep_slot"]) >= 0                # pieces whose weights are prefetched
+    n_slot = int(slotted.sum())
+    n_rx = len(set(np.asarray(tabs["rep_expert"])[slotted].tolist()))
     w_el = run.prob.w_elems if run.with_weights else 0
     g_el = run.prob.g_elems if run.with_grads else 0
     ab = alg_bytes(run.cfg, n_slot, n_rx, w_el, g_el)
@@ -605,6 +608,7 @@ def run_gpu(args):
     if extras:
         if args.workload != "mid":
             extra["mid"] = run_mid(args, peak)
+        extra["ep_emulated"] = run_ep(args, peak)
         extra["inference"] = run_inference(args, peak, pool)
         if not args.no_sweep:
             extra["sweep"] = run_sweep(args, peak, pool)
@@ -668,6 +672,66 @@ def run_mid(args, peak):
     out = {"workload": wl_desc(wl, run.route, ", seed 0"),
            "step": "plan -> prefetch -> dispatch -> combine -> reduce_grad", **short_figures(f, wl.T, wl.K)}
     del run
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ep(args, peak):
+    """The mid workload's step through the expert-parallel calls, its R = 8
+    ranks emulated on this GPU (each rank's own buffers, peers through
+    peer-pointer tables, the count all-gather a device copy): per rank count
+    -> (gather) -> plan -> prefetch -> dispatch -> combine -> reduce_grad,
+    rank after rank for each call.  Every kernel is launched once per rank;
+    the figures are the sums over the ranks' launches (CUDA events around
+    each phase on the launching stream).  One GPU per rank is not measured
+    here."""
+    import torch
+    from load_balancing_plan_b200 import ep
+    wl = inputs.WORKLOADS["mid"]
+    cfg = wl.cfg()
+    route = inputs.routing(wl.R, wl.L, wl.S, wl.K, 0, maxvio=wl.maxvio[0])
+    em = ep.Emulation(cfg, w_elems=wl.w_elems, g_elems=wl.g_elems)
+    em.set_routing(route.topk_idx, route.topk_w)
+    for q, rb in enumerate(em.ranks):
+        inputs.cb_fill_torch(rb.x.view(torch.bfloat16), 0, inputs.STREAM_X, offset=q * wl.S * wl.H)
+        inputs.cb_fill_torch(rb.w_home.view(torch.bfloat16), 0, inputs.STREAM_W, offset=q * wl.L * wl.w_elems)
+        inputs.cb_fill_torch(rb.g_home, 0, inputs.STREAM_G_HOME, offset=q * wl.L * wl.g_elems)
+    s = torch.cuda.current_stream()
+    phases = [("plan", em.plan), ("prefetch", em.prefetch), ("dispatch", em.dispatch),
+              ("combine", em.combine), ("reduce_grad", em.reduce_grad)]
+    for _ in range(3):
+        for _, fn in phases:
+            fn()
+    torch.cuda.synchronize()
+    info = em.ranks[0].read_plan(tables=True)
+    if info["status"] & 0xFF:
+        raise RuntimeError("expert-parallel plan failed: status 0x%x" % info["status"])
+    n_rx = len(set(np.asarray(info["rep_expert"]).tolist()))
+    ab = alg_bytes(cfg, info["n_replicas"], n_rx, wl.w_elems, wl.g_elems)
+    # one rank per GPU: every receiver reads its experts' weights from the
+    # home rank itself, one read and one write per slot
+    ab["prefetch"] = 2 * 2 * wl.w_elems * info["n_replicas"]
+    steps = args.extra_steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)] for _ in range(steps)]
+    for i in range(steps):
+        ev[i][0].record(s)
+        for j, (_, fn) in enumerate(phases):
+            fn()
+            ev[i][j + 1].record(s)
+    torch.cuda.synchronize()
+    us = {name: float(np.mean([ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)])) * 1e3
+          for j, (name, _) in enumerate(phases)}
+    total_ms = float(np.mean([ev[i][0].elapsed_time(ev[i][-1]) for i in range(steps)]))
+    dc = ab["dispatch"] + ab["combine"]
+    value = dc / ((us["dispatch"] + us["combine"]) * 1e-6) / 1e9
+    out = {"workload": wl_desc(wl, route, ", seed 0; %d ranks emulated on one GPU" % wl.R),
+           "step": "per rank: count -> (all-gather) -> plan -> prefetch -> dispatch -> combine -> reduce_grad",
+           "value": round(value, 2), "unit": UNIT, "dispatch_combine_frac_of_peak": round(value / peak, 4),
+           "ms_per_step": round(total_ms, 4), "launch": "eager, one launch per rank and call",
+           "phase_us": {k: round(v, 2) for k, v in us.items()},
+           "phase_gbs": {k: (round(ab[k] / (v * 1e-6) / 1e9, 1) if ab[k] and k != "plan" else None)
+                         for k, v in us.items()}}
+    del em
     torch.cuda.empty_cache()
     return out
 
@@ -933,8 +997,9 @@ def run_only(args):
     if info["status"] & mp.ST_ERROR_MASK:
         raise RuntimeError("plan failed: status 0x%x" % info["status"])
     tabs = mp.moonep_plan_read(cfg, prob.ws, tables=True)
-    n_rx = len(set(np.asarray(tabs["rep_expert"]).tolist()))
-    n_slot = int((np.asarray(tabs["rep_slot"]) >= 0).sum())
+    slotted = np.asarray(tabs["rep_slot"]) >= 0
+    n_slot = int(slotted.sum())
+    n_rx = len(set(np.asarray(tabs["rep_expert"])[slotted].tolist()))
     ab = alg_bytes(cfg, n_slot, n_rx, prob.w_elems, prob.g_elems)[k]
     fn = {"plan": prob.plan, "prefetch": prob.prefetch, "dispatch": prob.dispatch,
           "combine": prob.combine, "reduce_grad": prob.reduce_grad}[k]

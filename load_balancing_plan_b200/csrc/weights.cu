@@ -37,6 +37,12 @@ constexpr int kChunkVecs = 2048;   // 32 KB of fp32 per chunk
 #ifndef MOONEP_PREFETCH_LOOKAHEAD
 #define MOONEP_PREFETCH_LOOKAHEAD 4
 #endif
+#ifndef MOONEP_PREFETCH_ONCE
+#define MOONEP_PREFETCH_ONCE 1  // 1: one read per replicated expert, stored to all its slots
+#endif
+#ifndef MOONEP_PREFETCH_INTERLEAVE
+#define MOONEP_PREFETCH_INTERLEAVE 0  // 1: units dealt to the CTAs round-robin instead of contiguous shares
+#endif
 constexpr uint32_t kPfChunk = MOONEP_PREFETCH_CHUNK;
 constexpr int kPfStages = MOONEP_PREFETCH_STAGES;
 constexpr int kPfAhead = MOONEP_PREFETCH_LOOKAHEAD;
@@ -79,9 +85,12 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
     const int64_t bytes_per = p.vecs * 16;
     const int64_t cps = (bytes_per + kPfChunk - 1) / kPfChunk;
     const int64_t units = P * cps;
-    const int64_t u0 = (int64_t)blockIdx.x * units / gridDim.x;
-    const int64_t u1 = (int64_t)(blockIdx.x + 1) * units / gridDim.x;
-    const int64_t n = u1 - u0;
+    // the CTA's units: u0 + it * ustep for it < n
+    const int64_t ustep = MOONEP_PREFETCH_INTERLEAVE ? gridDim.x : 1;
+    const int64_t u0 = MOONEP_PREFETCH_INTERLEAVE ? blockIdx.x : (int64_t)blockIdx.x * units / gridDim.x;
+    const int64_t n = MOONEP_PREFETCH_INTERLEAVE
+                          ? (blockIdx.x < units ? (units - 1 - blockIdx.x) / gridDim.x + 1 : 0)
+                          : (int64_t)(blockIdx.x + 1) * units / gridDim.x - u0;
     const uint8_t *src_base = reinterpret_cast<const uint8_t *>(p.src);
     uint8_t *dst_base = reinterpret_cast<uint8_t *>(p.dst);
     const uint64_t pol = policy_evict_first();
@@ -89,7 +98,7 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
     int64_t issued = 0, stored = 0;
     for (int64_t it = 0; it < n + kPfAhead; ++it) {
         if (it < n) {
-            const int64_t u = u0 + it;
+            const int64_t u = u0 + it * ustep;
             const int64_t sp = u / cps, c = u - sp * cps;
             const int gp = __ldg(ws + p.lay.slot_piece + sp0 + sp);
             const int e = __ldg(ws + p.lay.rep_expert + gp);
@@ -111,7 +120,7 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
                     break;
                 }
             if (fail) break;
-            const int64_t u = u0 + j;
+            const int64_t u = u0 + j * ustep;
             const int64_t sp = u / cps, c = u - sp * cps;
             const int gp = __ldg(ws + p.lay.slot_piece + sp0 + sp);
             const int64_t slot = kEp ? (int64_t)__ldg(ws + p.lay.rep_slot + gp)
@@ -128,6 +137,95 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
     bulk_wait_all<0>();
     if (fail) {
         // let the loads still in flight land before the CTA exits
+        const int64_t drain = p.wait_limit > (int64_t(1) << 20) ? p.wait_limit : (int64_t(1) << 20);
+        for (int64_t u = stored; u < issued; ++u) {
+            int64_t w = 0;
+            while (!mbar_try_wait(&bars[u % kPfStages], (uint32_t)((u / kPfStages) & 1)))
+                if (++w > drain) break;
+        }
+        atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
+    }
+}
+
+// Prefetch on one GPU, reading each replicated expert once: a unit is one
+// 32 KB chunk of one replicated expert's weights, loaded into a stage once
+// and stored from there to the slot of every piece of that expert (an expert
+// replicated on n receivers costs one read and n writes, not n of each).
+// Units are dealt to the CTAs round-robin, so every CTA gets a like mix of
+// experts with few and many replicas.  Pieces without a slot (remote
+// weights) take no copy; an expert with none is not read.
+__global__ void __launch_bounds__(32, 1) prefetch_once_kernel(const __grid_constant__ CopyParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    int32_t *ws = p.ws;
+    if (block_status_failed(ws)) return;
+    if (!cfg_matches(ws, p.cfg, p.lay.n_ranges, p.ep_tag)) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
+        return;
+    }
+    if (threadIdx.x != 0) return;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)kPfStages * kPfChunk);
+    for (int s = 0; s < kPfStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+
+    const int B = p.cfg.B;
+    const int64_t nrx = __ldcg(ws + HDR_NRX);
+    const int64_t bytes_per = p.vecs * 16;
+    const int64_t cps = (bytes_per + kPfChunk - 1) / kPfChunk;
+    const int64_t units = nrx * cps;
+    const int64_t u0 = blockIdx.x, ustep = gridDim.x;
+    const int64_t n = blockIdx.x < units ? (units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const uint8_t *src_base = reinterpret_cast<const uint8_t *>(p.src);
+    uint8_t *dst_base = reinterpret_cast<uint8_t *>(p.dst);
+    const uint64_t pol = policy_evict_first();
+    bool fail = false;
+    int64_t issued = 0, stored = 0;
+    for (int64_t it = 0; it < n + kPfAhead; ++it) {
+        if (it < n) {
+            const int64_t u = u0 + it * ustep;
+            const int64_t x = u / cps, c = u - x * cps;
+            const int e = __ldg(ws + p.lay.rx_expert + x);
+            const int pb = __ldg(ws + p.lay.rep_ptr + e), pe = __ldg(ws + p.lay.rep_ptr + e + 1);
+            bool any = false;
+            for (int q = pb; q < pe && !any; ++q) any = __ldg(ws + p.lay.rep_slot + q) >= 0;
+            const uint32_t bytes = (uint32_t)min((int64_t)kPfChunk, bytes_per - c * kPfChunk);
+            const int s = (int)(it % kPfStages);
+            if (it >= kPfStages) bulk_wait_read<kPfStages - kPfAhead - 1>();
+            mbar_arrive_expect_tx(&bars[s], any ? bytes : 0u);
+            if (any) bulk_g2s(smem + (size_t)s * kPfChunk, src_base + (int64_t)e * bytes_per + c * kPfChunk, bytes,
+                              &bars[s], pol);
+            issued = it + 1;
+        }
+        const int64_t j = it - kPfAhead;
+        if (j >= 0 && j < n) {
+            const int s = (int)(j % kPfStages);
+            int64_t w = 0;
+            while (!mbar_try_wait(&bars[s], (uint32_t)((j / kPfStages) & 1)))
+                if (++w > p.wait_limit) {
+                    fail = true;
+                    break;
+                }
+            if (fail) break;
+            const int64_t u = u0 + j * ustep;
+            const int64_t x = u / cps, c = u - x * cps;
+            const int e = __ldg(ws + p.lay.rx_expert + x);
+            const int pb = __ldg(ws + p.lay.rep_ptr + e), pe = __ldg(ws + p.lay.rep_ptr + e + 1);
+            const uint32_t bytes = (uint32_t)min((int64_t)kPfChunk, bytes_per - c * kPfChunk);
+            for (int q = pb; q < pe; ++q) {
+                const int sl = __ldg(ws + p.lay.rep_slot + q);
+                if (sl < 0) continue;
+                const int64_t slot = (int64_t)__ldg(ws + p.lay.rep_recv + q) * B + sl;
+                if (MOONEP_PREFETCH_STORE_HINT)
+                    bulk_s2g(dst_base + slot * bytes_per + c * kPfChunk, smem + (size_t)s * kPfChunk, bytes, pol);
+                else
+                    bulk_s2g_plain(dst_base + slot * bytes_per + c * kPfChunk, smem + (size_t)s * kPfChunk, bytes);
+            }
+            bulk_commit();
+            stored = j + 1;
+        }
+    }
+    bulk_wait_all<0>();
+    if (fail) {
         const int64_t drain = p.wait_limit > (int64_t(1) << 20) ? p.wait_limit : (int64_t(1) << 20);
         for (int64_t u = stored; u < issued; ++u) {
             int64_t w = 0;
@@ -412,6 +510,13 @@ cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s) {
         cudaError_t err = set_smem_limit((const void *)prefetch_kernel<true>, smem, smem_set_ep);
         if (err != cudaSuccess) return err;
         prefetch_kernel<true><<<grid, 32, smem, s>>>(p);
+        return cudaGetLastError();
+    }
+    if (MOONEP_PREFETCH_ONCE) {
+        static std::atomic<size_t> smem_set1[64];
+        cudaError_t err = set_smem_limit((const void *)prefetch_once_kernel, smem, smem_set1);
+        if (err != cudaSuccess) return err;
+        prefetch_once_kernel<<<grid, 32, smem, s>>>(p);
         return cudaGetLastError();
     }
     static std::atomic<size_t> smem_set[64];
