@@ -959,6 +959,23 @@ def run_reference(args):
 KERNELS = ("plan", "prefetch", "dispatch", "combine", "reduce_grad")
 
 
+class PlanOnly:
+    """The buffers of the plan alone: it reads the ids and writes only the
+    workspace."""
+
+    def __init__(self, cfg, route):
+        import torch
+        from load_balancing_plan_b200 import moonep as mp
+        self.cfg, self.mp = cfg, mp
+        self.ids = torch.from_numpy(np.ascontiguousarray(route.topk_idx.reshape(-1))).cuda()
+        self.ws = torch.zeros(mp.moonep_plan_workspace_bytes(cfg) // 4, dtype=torch.int32, device="cuda")
+        self.w_elems = self.g_elems = 0
+        self.prefetch = self.dispatch = self.combine = self.reduce_grad = None
+
+    def plan(self):
+        self.mp.moonep_plan(self.cfg, self.ids, self.ws)
+
+
 def run_only(args):
     """One kernel of the step alone, for profiler captures and kernel-alone
     timings: the buffers that kernel needs (weights only for prefetch,
@@ -975,13 +992,7 @@ def run_only(args):
     cfg = wl.cfg()
     k = args.only
     if k == "plan":
-        # the plan reads only the ids and writes only the workspace
-        prob = type("PlanOnly", (), {})()
-        prob.ids = torch.from_numpy(np.ascontiguousarray(route.topk_idx.reshape(-1))).cuda()
-        prob.ws = torch.zeros(mp.moonep_plan_workspace_bytes(cfg) // 4, dtype=torch.int32, device="cuda")
-        prob.w_elems = prob.g_elems = 0
-        prob.plan = lambda: mp.moonep_plan(cfg, prob.ids, prob.ws)
-        prob.prefetch = prob.dispatch = prob.combine = prob.reduce_grad = None
+        prob = PlanOnly(cfg, route)
     else:
         prob = harness.Problem(cfg, w_elems=wl.w_elems if k == "prefetch" else 0,
                                g_elems=wl.g_elems if k == "reduce_grad" else 0)
