@@ -41,7 +41,7 @@ namespace {
 constexpr int kPlanThreads = 512;
 
 // MOONEP_PLAN_TRACE: development builds stamp %globaltimer (ns) at the phase
-// boundaries of CTA 0 into header words 32..47 of the workspace.
+// boundaries of CTA 0 into header words 32..55 of the workspace (12 stamps).
 #ifdef MOONEP_PLAN_TRACE
 __device__ __forceinline__ void trace(int32_t *ws, int slot) {
     if (threadIdx.x == 0) {
@@ -541,6 +541,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
             for (int i = (nz & ~3) + tid; i < nz; i += kPlanThreads) sm[i] = 0;
         }
         __syncthreads();
+        if (blockIdx.x == 0) TRACE(ws, 9);
         const int64_t i0 = range_begin(qa, p.T, p.Q) * K, i1 = range_begin(qb, p.T, p.Q) * K;
         for (int64_t b0 = i0; b0 < i1; b0 += (int64_t)kIdBatch * kPlanThreads) {
             int v[kIdBatch];
@@ -566,6 +567,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
             }
         }
         __syncthreads();
+        if (blockIdx.x == 0) TRACE(ws, 10);
         for (int e = tid; e < N; e += kPlanThreads) {
             int run = 0;
 #pragma unroll 8
@@ -579,6 +581,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
             if (run) atomicAdd(cnt_acc + e, run);
         }
         __syncthreads();
+        if (blockIdx.x == 0) TRACE(ws, 11);
     }
     if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_EXPERT_ID);
     if (p.mode == kPlanCount) {

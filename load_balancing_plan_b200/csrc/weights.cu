@@ -40,6 +40,11 @@ constexpr int kChunkVecs = 2048;   // 32 KB of fp32 per chunk
 #ifndef MOONEP_PREFETCH_ONCE
 #define MOONEP_PREFETCH_ONCE 1  // 1: one read per replicated expert, stored to all its slots
 #endif
+#ifndef MOONEP_PREFETCH_ONCE_LOOKAHEAD
+#define MOONEP_PREFETCH_ONCE_LOOKAHEAD 1  // loads ahead in the read-once pipeline (its store groups are larger)
+#endif
+constexpr int kPfOnceAhead = MOONEP_PREFETCH_ONCE_LOOKAHEAD;
+static_assert(MOONEP_PREFETCH_STAGES - MOONEP_PREFETCH_ONCE_LOOKAHEAD - 1 >= 0, "stage reuse needs an older store group");
 #ifndef MOONEP_PREFETCH_INTERLEAVE
 #define MOONEP_PREFETCH_INTERLEAVE 0  // 1: units dealt to the CTAs round-robin instead of contiguous shares
 #endif
@@ -153,7 +158,11 @@ __global__ void __launch_bounds__(32, 1) prefetch_kernel(const __grid_constant__
 // replicated on n receivers costs one read and n writes, not n of each).
 // Units are dealt to the CTAs round-robin, so every CTA gets a like mix of
 // experts with few and many replicas.  Pieces without a slot (remote
-// weights) take no copy; an expert with none is not read.
+// weights) take no copy; an expert with none is not read.  One load ahead
+// (not four): a unit's store group is n times larger than its load, and with
+// one load ahead four store groups may still be reading their stages when a
+// stage is reused (training workload, kernel alone: 531 us with 1 ahead, 555
+// with 2, 558 with 4; mid: 111, 113-115, 115).
 __global__ void __launch_bounds__(32, 1) prefetch_once_kernel(const __grid_constant__ CopyParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     int32_t *ws = p.ws;
@@ -180,7 +189,7 @@ __global__ void __launch_bounds__(32, 1) prefetch_once_kernel(const __grid_const
     const uint64_t pol = policy_evict_first();
     bool fail = false;
     int64_t issued = 0, stored = 0;
-    for (int64_t it = 0; it < n + kPfAhead; ++it) {
+    for (int64_t it = 0; it < n + kPfOnceAhead; ++it) {
         if (it < n) {
             const int64_t u = u0 + it * ustep;
             const int64_t x = u / cps, c = u - x * cps;
@@ -190,13 +199,13 @@ __global__ void __launch_bounds__(32, 1) prefetch_once_kernel(const __grid_const
             for (int q = pb; q < pe && !any; ++q) any = __ldg(ws + p.lay.rep_slot + q) >= 0;
             const uint32_t bytes = (uint32_t)min((int64_t)kPfChunk, bytes_per - c * kPfChunk);
             const int s = (int)(it % kPfStages);
-            if (it >= kPfStages) bulk_wait_read<kPfStages - kPfAhead - 1>();
+            if (it >= kPfStages) bulk_wait_read<kPfStages - kPfOnceAhead - 1>();
             mbar_arrive_expect_tx(&bars[s], any ? bytes : 0u);
             if (any) bulk_g2s(smem + (size_t)s * kPfChunk, src_base + (int64_t)e * bytes_per + c * kPfChunk, bytes,
                               &bars[s], pol);
             issued = it + 1;
         }
-        const int64_t j = it - kPfAhead;
+        const int64_t j = it - kPfOnceAhead;
         if (j >= 0 && j < n) {
             const int s = (int)(j % kPfStages);
             int64_t w = 0;

@@ -252,3 +252,36 @@ def test_ep_and_single_gpu_workspaces_do_not_mix(env):
     assert bool((rb0.dest == -7).all())
     for rb in em.ranks:
         assert bool((rb.recv == -1).all())
+
+
+@pytest.mark.parametrize("case", [
+    # R, L, S, K, H, B, headroom
+    (4, 3, 50, 1, 24, 2, 1.0),       # K = 1, H not a multiple of 64
+    (8, 2, 40, 2, 64, 0, 6.0),       # no prefetch slots: every spill falls back
+    (3, 5, 7, 3, 16, 5, 1.0),        # ranges of a token or two, odd R
+])
+def test_ep_edge_cases(env, case):
+    R, L, S, K, H, B, headroom = case
+    cfg = cfg_of(R, L, S, K, H, B, headroom=headroom)
+    rt = inputs.routing(R, L, S, K, 2, alpha=1.5)
+    em, opl = run_ep_compare(env, cfg, rt.topk_idx, rt.topk_w, seed=2)
+    assert opl["status"] & oracle.ST_CAPACITY == 0
+    if B == 0:
+        assert opl["n_replicas"] == 0 and opl["fallback_rows"] > 0
+
+
+def test_ep_empty_ranks(env):
+    # S = 0: nothing to count, plan or move; every call returns without error
+    torch, mp, ep, harness = env
+    cfg = cfg_of(4, 2, 0, 2, 16, 2)
+    em = ep.Emulation(cfg, w_elems=64, g_elems=64)
+    em.plan()
+    em.prefetch()
+    em.dispatch()
+    em.combine()
+    em.reduce_grad()
+    torch.cuda.synchronize()
+    for rb in em.ranks:
+        info = rb.read_plan(tables=False)
+        assert info["status"] & mp.ST_ERROR_MASK == 0
+        assert info["n_replicas"] == 0 and info["fallback_rows"] == 0
