@@ -202,9 +202,10 @@ int moonep_plan_ex(const moonep_cfg_t *cfg, int32_t flags, const int32_t *topk_i
     compute_layout(*cfg, p.lay);
     p.Q = p.lay.n_ranges;
     {
-        // phase A holds one block's (range, expert) histogram in shared memory
+        // phase A holds one block's (range, expert) histogram and its totals
+        // per expert in shared memory
         const int64_t rpb = p.lay.n_blocks > 0 ? (p.Q + p.lay.n_blocks - 1) / p.lay.n_blocks : 0;
-        if ((size_t)(rpb * N) * sizeof(int) > d->plan_smem)
+        if ((size_t)((rpb + 1) * N) * sizeof(int) > d->plan_smem)
             return fail(MOONEP_ERR_ARG, "plan: %lld ranges per block of %d experts exceed shared memory",
                         (long long)rpb, N);
     }
@@ -465,7 +466,7 @@ static int ep_plan_launch(const moonep_cfg_t *cfg, int32_t mode, int32_t flags, 
     compute_layout_tokens(*cfg, cfg->S, p.lay);
     p.Q = p.lay.n_ranges;
     const int64_t rpb = p.lay.n_blocks > 0 ? (p.Q + p.lay.n_blocks - 1) / p.lay.n_blocks : 0;
-    if ((size_t)(rpb * N) * sizeof(int) > d->plan_smem)
+    if ((size_t)((rpb + 1) * N) * sizeof(int) > d->plan_smem)
         return fail(MOONEP_ERR_ARG, "plan: %lld ranges per block of %d experts exceed shared memory", (long long)rpb, N);
     p.ids = ids;
     p.ws = (int32_t *)ws;

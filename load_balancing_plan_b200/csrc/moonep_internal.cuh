@@ -53,10 +53,11 @@ constexpr int64_t kRangeTokens = MOONEP_RANGE_TOKENS;
 #endif
 constexpr int64_t kBaseWords = int64_t(1) << MOONEP_BASE_WORDS_LOG2;
 // The plan counts ranges in blocks of consecutive ranges (one CTA counts a
-// block); kBlocks blocks at most, one per SM of a B200, so that each plan
-// CTA loads all the ids it counts in one batch.
+// block); kBlocks blocks at most, one per SM of a B200 but the one whose CTA
+// plans, so that each counting CTA loads all the ids it counts in one batch
+// and keeps its block's histogram over the grid barrier.
 #ifndef MOONEP_BLOCKS
-#define MOONEP_BLOCKS 148
+#define MOONEP_BLOCKS 147
 #endif
 constexpr int64_t kBlocks = MOONEP_BLOCKS;
 

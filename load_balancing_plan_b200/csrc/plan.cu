@@ -41,7 +41,8 @@ namespace {
 constexpr int kPlanThreads = 512;
 
 // MOONEP_PLAN_TRACE: development builds stamp %globaltimer (ns) at the phase
-// boundaries of CTA 0 into header words 32..55 of the workspace (12 stamps).
+// boundaries of CTA 0 into header words 32..55 of the workspace (12 stamps),
+// and the grid's start and counting-end spread into words 56..61.
 #ifdef MOONEP_PLAN_TRACE
 __device__ __forceinline__ void trace(int32_t *ws, int slot) {
     if (threadIdx.x == 0) {
@@ -51,12 +52,33 @@ __device__ __forceinline__ void trace(int32_t *ws, int slot) {
     }
 }
 #define TRACE(ws, slot) trace(ws, slot)
+// every CTA: words 56..57 the latest end of a counting phase, 58..59 the
+// complement of the earliest start, 60..61 the latest start
+__device__ __forceinline__ void trace_grid(int32_t *ws, bool start) {
+    if (threadIdx.x == 0) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        unsigned long long *w = reinterpret_cast<unsigned long long *>(ws + 56);
+        if (start) {
+            atomicMax(w + 1, ~t);
+            atomicMax(w + 2, t);
+        } else {
+            atomicMax(w, t);
+        }
+    }
+}
+#define TRACE_GRID(ws, start) trace_grid(ws, start)
 #else
 #define TRACE(ws, slot) ((void)0)
+#define TRACE_GRID(ws, start) ((void)0)
 #endif
 constexpr int kWarps = kPlanThreads / 32;
 constexpr int kMaxR = 64;
-constexpr int kIdBatch = 8;
+#ifndef MOONEP_ID_BATCH
+#define MOONEP_ID_BATCH 8  // ids per thread loaded together in the counting phase (16: the plan
+                           // ran 9 us slower in the step on training, its code no longer cold-friendly)
+#endif
+constexpr int kIdBatch = MOONEP_ID_BATCH;
 // Above this many experts the whole CTA plans.  Alone and warm, one warp
 // plans a few hundred experts faster (no block barriers), but right after
 // GBs of streaming traffic, as in a real step, the CTA-wide planner wins at
@@ -513,16 +535,24 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     const moonep_ws_layout_t &lay = p.lay;
 
     if (blockIdx.x == 0) TRACE(ws, 0);
-    // phase A: each CTA takes blocks of consecutive token ranges and counts
-    // the block's ids into a shared-memory histogram per (range, expert) --
-    // all of a block's ids are loaded in one batch of up to kIdBatch per
-    // thread, so a block costs about one memory latency however many ranges
-    // it holds.  Then one thread per expert walks the block's ranges in
-    // order: base[e][q] = copies of e in the block's earlier ranges (stored
-    // only where range q has a copy of e: a range of a few tokens routes to
-    // few experts, and dispatch reads no other entry), blk[e][b] = the
-    // block's total, which also goes into the global tokens_per_expert
-    // (cnt).
+    TRACE_GRID(ws, true);
+    // phase A: each counting CTA takes blocks of consecutive token ranges and
+    // counts the block's ids into a shared-memory histogram per (range,
+    // expert) and into the block's totals per expert -- all of a block's ids
+    // are loaded in one batch of up to kIdBatch per thread, so a block costs
+    // about one memory latency however many ranges it holds.  The totals go
+    // to blk[e][b] and into the global tokens_per_expert (cnt).  Then one
+    // thread per expert walks the block's ranges in order: base[e][q] =
+    // copies of e in the block's earlier ranges (stored only where range q
+    // has a copy of e: a range of a few tokens routes to few experts, and
+    // dispatch reads no other entry).
+    //
+    // For the plan proper on more than one CTA, CTA 0 counts no block (it
+    // plans after the barrier) and CTA k >= 1 counts block k - 1.  With one
+    // block per counting CTA the histogram stays in shared memory over the
+    // barrier and the range walk runs after it, beside the planner: only
+    // dispatch reads base, and the barrier's fence would otherwise wait for
+    // those thousands of scattered stores (3-4 us on the training workload).
     bool bad = false;
     const int64_t NB = lay.n_blocks;
     // copies per expert: into the plan's cnt, or (counting one rank's tokens
@@ -531,17 +561,37 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     // the range of token t is ((t + 1) * Q - 1) / T; in 32 bits when that
     // cannot overflow (every configuration up to 2^32 / Q tokens)
     const bool div32 = (uint64_t)(p.T + 1) * (uint64_t)p.Q < (uint64_t(1) << 32);
-    for (int64_t b = blockIdx.x; b < NB; b += gridDim.x) {
+    const bool planner_apart = p.mode == kPlanFull && gridDim.x > 1;
+    const int64_t b_step = planner_apart ? gridDim.x - 1 : gridDim.x;
+    const int64_t b_first = planner_apart ? (blockIdx.x == 0 ? NB : (int64_t)blockIdx.x - 1) : blockIdx.x;
+    const bool defer_walk = planner_apart && NB <= b_step;
+    int64_t walk_qa = 0;
+    int walk_nr = 0;
+    bool walk_pending = false;
+    auto walk = [&](int64_t qa, int nr) {
+        for (int e = tid; e < N; e += kPlanThreads) {
+            int run = 0;
+#pragma unroll 8
+            for (int r = 0; r < nr; ++r) {
+                // dispatch reads base[e][q] only where range q routes to e
+                const int c = sm[r * N + e];
+                if (c) ws[lay.base + (int64_t)e * p.Q + qa + r] = run;
+                run += c;
+            }
+        }
+    };
+    for (int64_t b = b_first; b < NB; b += b_step) {
         const int64_t qa = block_first_range(b, p.Q, NB), qb = block_first_range(b + 1, p.Q, NB);
         const int nr = (int)(qb - qa);
+        int *tot = sm + nr * N;  // the block's copies per expert
         {
-            const int nz = nr * N;
+            const int nz = nr * N + N;
             int4 *sm4 = reinterpret_cast<int4 *>(sm);
             for (int i = tid; i < nz / 4; i += kPlanThreads) sm4[i] = make_int4(0, 0, 0, 0);
             for (int i = (nz & ~3) + tid; i < nz; i += kPlanThreads) sm[i] = 0;
         }
         __syncthreads();
-        if (blockIdx.x == 0) TRACE(ws, 9);
+        if (blockIdx.x == 1) TRACE(ws, 9);
         const int64_t i0 = range_begin(qa, p.T, p.Q) * K, i1 = range_begin(qb, p.T, p.Q) * K;
         for (int64_t b0 = i0; b0 < i1; b0 += (int64_t)kIdBatch * kPlanThreads) {
             int v[kIdBatch];
@@ -560,6 +610,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
                         const int64_t q = div32 ? (int64_t)(((uint32_t)(t + 1) * (uint32_t)p.Q - 1u) / (uint32_t)p.T)
                                                 : ((t + 1) * p.Q - 1) / p.T;
                         atomicAdd(&sm[(q - qa) * N + v[u]], 1);
+                        atomicAdd(&tot[v[u]], 1);
                     } else {
                         bad = true;
                     }
@@ -567,22 +618,23 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
             }
         }
         __syncthreads();
-        if (blockIdx.x == 0) TRACE(ws, 10);
+        if (blockIdx.x == 1) TRACE(ws, 10);
         for (int e = tid; e < N; e += kPlanThreads) {
-            int run = 0;
-#pragma unroll 8
-            for (int r = 0; r < nr; ++r) {
-                // dispatch reads base[e][q] only where range q routes to e
-                const int c = sm[r * N + e];
-                if (c) ws[lay.base + (int64_t)e * p.Q + qa + r] = run;
-                run += c;
-            }
-            ws[lay.blk + (int64_t)e * NB + b] = run;
-            if (run) atomicAdd(cnt_acc + e, run);
+            const int c = tot[e];
+            ws[lay.blk + (int64_t)e * NB + b] = c;
+            if (c) atomicAdd(cnt_acc + e, c);
         }
-        __syncthreads();
-        if (blockIdx.x == 0) TRACE(ws, 11);
+        if (defer_walk) {
+            walk_qa = qa;
+            walk_nr = nr;
+            walk_pending = true;
+        } else {
+            walk(qa, nr);
+            __syncthreads();
+        }
+        if (blockIdx.x == 1) TRACE(ws, 11);
     }
+    TRACE_GRID(ws, false);
     if (bad) atomicOr(ws + HDR_STATUS, MOONEP_ST_EXPERT_ID);
     if (p.mode == kPlanCount) {
         // the status travels with the counts, so every rank learns of it
@@ -620,6 +672,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
         else if (warp == 0)
             plan_tables<32>(p, sm);
     } else {
+        // the block's range walk, from the histogram kept in shared memory
+        if (walk_pending) walk(walk_qa, walk_nr);
         const int gw = (blockIdx.x - 1) * kWarps + warp;
         const int nw = (gridDim.x - 1) * kWarps;
         for (int e = gw; e < N; e += nw) scan_column(ws + lay.blk + (int64_t)e * NB, NB);
@@ -631,12 +685,13 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
 }  // namespace
 
 // Dynamic shared memory of the plan: 7 arrays of N ints for the planner, or
-// phase A's (range, expert) histogram of a block, ceil(Q / NB) * N ints,
-// whichever is larger.  With Q <= max(kMinRanges, kBaseWords / N) and NB =
-// min(Q, kBlocks), ceil(Q / NB) * N <= kBaseWords / kBlocks + N.
+// phase A's (range, expert) histogram of a block and its totals,
+// (ceil(Q / NB) + 1) * N ints, whichever is larger.  With Q <=
+// max(kMinRanges, kBaseWords / N) and NB = min(Q, kBlocks),
+// ceil(Q / NB) * N <= kBaseWords / kBlocks + N.
 size_t plan_smem_bytes(int N) {
     const int64_t n = N > 0 ? N : 1;
-    const int64_t a = 7 * n, b = kBaseWords / kBlocks + n + 1;
+    const int64_t a = 7 * n, b = kBaseWords / kBlocks + 2 * n + 4;
     return (size_t)(a > b ? a : b) * sizeof(int);
 }
 

@@ -94,11 +94,11 @@ def test_layout_is_consistent(mp):
         N = c["R"] * c["L"]
         # whole waves of 296 ranges of about 4 tokens, at most 2^22 / N
         # entries per expert (T itself if fewer); blocks of consecutive
-        # ranges, at most 148
+        # ranges, at most 147 (one per counting CTA: all SMs but the planner's)
         w = max(1, min((T + 592) // 1184, (1 << 22) // (N * 296)))
         Q = min(T, 296 * w)
         assert lay["n_ranges"] == mp.moonep_num_ranges(T, N) == Q
-        assert lay["n_blocks"] == min(Q, 148)
+        assert lay["n_blocks"] == min(Q, 147)
         assert lay["blk"] == lay["base"] + N * max(Q, 1)
         assert lay["words"] >= lay["blk"] + N * max(lay["n_blocks"], 1)
         assert mp.moonep_plan_workspace_bytes(c) == 4 * lay["words"]
