@@ -9,7 +9,9 @@
 //
 // Both walk lists the plan leaves in the workspace (the replica pieces, and
 // the experts that have at least one).  prefetch moves 32 KB chunks with TMA
-// bulk copies (one warp per SM, a pipeline of shared-memory stages).
+// bulk copies (one warp per SM, a pipeline of shared-memory stages), reading
+// each chunk of a replicated expert once and storing it to every slot of
+// that expert.
 // reduce_grad deals units of a few KB of one expert's gradient to warps; each
 // warp keeps two units' loads in flight (the next unit's home and replica
 // vectors are loaded before the current unit is added and stored).  Under
