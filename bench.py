@@ -680,8 +680,8 @@ def run_ep(args, peak):
     """The mid workload's step through the expert-parallel calls, its R = 8
     ranks emulated on this GPU (each rank's own buffers, peers through
     peer-pointer tables, the count all-gather a device copy): per rank count
-    -> (gather) -> plan -> prefetch -> dispatch -> combine -> reduce_grad,
-    rank after rank for each call.  Every kernel is launched once per rank;
+    -> (gather) -> plan -> prefetch -> dispatch -> combine -> combine_backward
+    -> dispatch_backward -> reduce_grad, rank after rank for each call.  Every kernel is launched once per rank;
     the figures are the sums over the ranks' launches (CUDA events around
     each phase on the launching stream).  One GPU per rank is not measured
     here."""
@@ -697,8 +697,19 @@ def run_ep(args, peak):
         inputs.cb_fill_torch(rb.w_home.view(torch.bfloat16), 0, inputs.STREAM_W, offset=q * wl.L * wl.w_elems)
         inputs.cb_fill_torch(rb.g_home, 0, inputs.STREAM_G_HOME, offset=q * wl.L * wl.g_elems)
     s = torch.cuda.current_stream()
+    # the backward pair: each rank's combine output stands in for its
+    # grad_out; grad_y lands on the ranks that hold the rows
+    dev = em.ranks[0].recv.device
+    grad_y = [torch.empty_like(rb.recv) for rb in em.ranks]
+    grad_y_peers = ep.peer_table(grad_y, dev)
+    grad_w = [torch.empty_like(rb.w) for rb in em.ranks]
+    grad_x = [torch.empty_like(rb.x) for rb in em.ranks]
+    grad_out = [rb.out for rb in em.ranks]
     phases = [("plan", em.plan), ("prefetch", em.prefetch), ("dispatch", em.dispatch),
-              ("combine", em.combine), ("reduce_grad", em.reduce_grad)]
+              ("combine", em.combine),
+              ("combine_backward", lambda: em.combine_backward(grad_out, grad_y_peers, grad_w)),
+              ("dispatch_backward", lambda: em.dispatch_backward(grad_y_peers, grad_x)),
+              ("reduce_grad", em.reduce_grad)]
     for _ in range(3):
         for _, fn in phases:
             fn()
@@ -711,6 +722,9 @@ def run_ep(args, peak):
     # one rank per GPU: every receiver reads its experts' weights from the
     # home rank itself, one read and one write per slot
     ab["prefetch"] = 2 * 2 * wl.w_elems * info["n_replicas"]
+    T, K, H = wl.T, wl.K, wl.H
+    ab["combine_backward"] = T * 2 * H + 2 * T * K * 2 * H + 12 * T * K
+    ab["dispatch_backward"] = T * K * 2 * H + T * 2 * H + 4 * T * K
     steps = args.extra_steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)] for _ in range(steps)]
     for i in range(steps):
@@ -725,13 +739,14 @@ def run_ep(args, peak):
     dc = ab["dispatch"] + ab["combine"]
     value = dc / ((us["dispatch"] + us["combine"]) * 1e-6) / 1e9
     out = {"workload": wl_desc(wl, route, ", seed 0; %d ranks emulated on one GPU" % wl.R),
-           "step": "per rank: count -> (all-gather) -> plan -> prefetch -> dispatch -> combine -> reduce_grad",
+           "step": "per rank: count -> (all-gather) -> plan -> prefetch -> dispatch -> combine -> combine_backward "
+                   "-> dispatch_backward -> reduce_grad",
            "value": round(value, 2), "unit": UNIT, "dispatch_combine_frac_of_peak": round(value / peak, 4),
            "ms_per_step": round(total_ms, 4), "launch": "eager, one launch per rank and call",
            "phase_us": {k: round(v, 2) for k, v in us.items()},
            "phase_gbs": {k: (round(ab[k] / (v * 1e-6) / 1e9, 1) if ab[k] and k != "plan" else None)
                          for k, v in us.items()}}
-    del em
+    del em, grad_y, grad_w, grad_x, grad_out
     torch.cuda.empty_cache()
     return out
 

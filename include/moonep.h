@@ -343,11 +343,14 @@ MOONEP_API int moonep_plan_noalloc(const moonep_cfg_t *cfg, const int32_t *topk_
  *      derives the same tables (identical to moonep_plan's for the R*S
  *      tokens); the rank's copy numbers start after the lower ranks' copies.
  *   4. moonep_ep_prefetch, moonep_ep_dispatch, (experts), moonep_ep_combine,
- *      moonep_ep_reduce_grad, each on the rank's own stream.
+ *      and for training moonep_ep_combine_backward, (experts' backward),
+ *      moonep_ep_dispatch_backward, moonep_ep_reduce_grad, each on the
+ *      rank's own stream.
  * Between steps the caller orders the ranks (a barrier on every rank after
  * its dispatch and before any combine reads the expert outputs; likewise
  * around prefetch and reduce_grad): the kernels never wait on one another.
- * Peer tables (recv_peers, y_peers, w_home_peers, g_rep_peers) are device
+ * Peer tables (recv_peers, y_peers, grad_y_peers, grad_recv_peers,
+ * w_home_peers, g_rep_peers) are device
  * arrays of R device pointers, entry q pointing at rank q's buffer as this
  * GPU addresses it (peer-mapped memory, CUDA IPC or symmetric allocations;
  * the rank's own buffer at entry r).  `dest` holds global flat rows
@@ -384,6 +387,24 @@ MOONEP_API int moonep_ep_dispatch(const moonep_cfg_t *cfg, int32_t rank, void *w
  * arithmetic of moonep_combine. */
 MOONEP_API int moonep_ep_combine(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *y_peers,
                                  const int32_t *dest, const float *topk_w, void *out, void *stream);
+
+/* Combine backward of rank `rank`'s tokens: grad_out [S][H] (bf16) and
+ * dest, topk_w [S][K] of this rank; grad_y_peers[q] + row*H receives
+ * grad_y of row q*C_max + row (rank q's [C_max][H] bf16 buffer), and
+ * grad_w [S][K] (fp32, or NULL) reads y from y_peers as moonep_ep_combine
+ * does; the arithmetic, the order of the grad_w sums and the rows written
+ * are those of moonep_combine_backward.  y_peers may be NULL when grad_w is
+ * NULL. */
+MOONEP_API int moonep_ep_combine_backward(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *grad_out,
+                                          const void *const *y_peers, const int32_t *dest, const float *topk_w,
+                                          void *const *grad_y_peers, float *grad_w, void *stream);
+
+/* Dispatch backward of rank `rank`'s tokens: grad_x [S][H] (bf16) from
+ * grad_recv_peers[q] (rank q's [C_max][H] gradient of the dispatched rows)
+ * and this rank's dest [S][K]; the arithmetic of moonep_dispatch_backward. */
+MOONEP_API int moonep_ep_dispatch_backward(const moonep_cfg_t *cfg, int32_t rank, void *ws,
+                                           const void *const *grad_recv_peers, const int32_t *dest, void *grad_x,
+                                           void *stream);
 
 /* Prefetch into rank `rank`'s slots: w_slot [B][elems] (bf16); slot b of
  * the rank gets expert e's weights from w_home_peers[e / L] + (e % L)*elems. */

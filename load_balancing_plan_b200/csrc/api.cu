@@ -553,16 +553,16 @@ int moonep_ep_dispatch(const moonep_cfg_t *cfg, int32_t rank, void *ws, const vo
     return MOONEP_OK;
 }
 
-int moonep_ep_combine(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *y_peers,
-                      const int32_t *dest, const float *topk_w, void *out, void *stream) {
+static int ep_combine_impl(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *y_peers,
+                           const int32_t *dest, const float *topk_w, void *out, void *stream, bool weighted) {
     TRY(check_cfg(cfg));
     TRY(check_rank(cfg, rank));
     const int64_t T = cfg->S;
     TRY(check_ptr(ws, 16, "ws", true));
-    TRY(check_ptr(y_peers, 8, "y_peers", T > 0));
+    TRY(check_ptr(y_peers, 8, weighted ? "y_peers" : "grad_recv_peers", T > 0));
     TRY(check_ptr(dest, 4, "dest", T > 0));
-    TRY(check_ptr(topk_w, 4, "topk_w", T > 0));
-    TRY(check_ptr(out, 16, "out", T > 0));
+    TRY(check_ptr(topk_w, 4, "topk_w", weighted && T > 0));
+    TRY(check_ptr(out, 16, weighted ? "out" : "grad_x", T > 0));
     DeviceInfo *d = nullptr;
     TRY(device_info(cfg->R * cfg->L, &d));
     if (T == 0) return MOONEP_OK;
@@ -578,7 +578,7 @@ int moonep_ep_combine(const moonep_cfg_t *cfg, int32_t rank, void *ws, const voi
     p.y = nullptr;
     p.y_peers = (const uint8_t *const *)y_peers;
     p.dest = dest;
-    p.w = topk_w;
+    p.w = weighted ? topk_w : nullptr;
     p.out = (uint4 *)out;
     p.ws = (int32_t *)ws;
     p.wait_limit = g_wait_limit.load();
@@ -588,7 +588,63 @@ int moonep_ep_combine(const moonep_cfg_t *cfg, int32_t rank, void *ws, const voi
     if (grid < 1) grid = 1;
     cudaError_t e = launch_combine(p, (int)grid, smem, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
-    bump_generation(ws);
+    if (weighted) bump_generation(ws);
+    return MOONEP_OK;
+}
+
+int moonep_ep_combine(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *y_peers,
+                      const int32_t *dest, const float *topk_w, void *out, void *stream) {
+    return ep_combine_impl(cfg, rank, ws, y_peers, dest, topk_w, out, stream, true);
+}
+
+int moonep_ep_dispatch_backward(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *const *grad_recv_peers,
+                                const int32_t *dest, void *grad_x, void *stream) {
+    return ep_combine_impl(cfg, rank, ws, grad_recv_peers, dest, nullptr, grad_x, stream, false);
+}
+
+int moonep_ep_combine_backward(const moonep_cfg_t *cfg, int32_t rank, void *ws, const void *grad_out,
+                               const void *const *y_peers, const int32_t *dest, const float *topk_w,
+                               void *const *grad_y_peers, float *grad_w, void *stream) {
+    TRY(check_cfg(cfg));
+    TRY(check_rank(cfg, rank));
+    const int64_t T = cfg->S;
+    TRY(check_ptr(ws, 16, "ws", true));
+    TRY(check_ptr(grad_out, 16, "grad_out", T > 0));
+    TRY(check_ptr(dest, 4, "dest", T > 0));
+    TRY(check_ptr(topk_w, 4, "topk_w", T > 0));
+    TRY(check_ptr(grad_y_peers, 8, "grad_y_peers", T > 0));
+    if (grad_w) {
+        TRY(check_ptr(grad_w, 4, "grad_w", true));
+        TRY(check_ptr(y_peers, 8, "y_peers (needed for grad_w)", T > 0));
+    }
+    DeviceInfo *d = nullptr;
+    TRY(device_info(cfg->R * cfg->L, &d));
+    if (T == 0) return MOONEP_OK;
+    BackwardParams p{};
+    p.cfg = *cfg;
+    p.T = T;
+    p.hv = cfg->H / 8;
+    size_t smem = 0;
+    if (combine_backward_config(cfg->K, p.hv, grad_w != nullptr, &p.chunk_bytes, &p.upt, &p.stages, &smem) !=
+        cudaSuccess)
+        return fail(MOONEP_ERR_ARG, "combine_backward: no shared-memory configuration for K=%d H=%d", cfg->K, cfg->H);
+    p.rows_total = (int64_t)cfg->R * cfg->C_max;
+    p.wait_limit = g_wait_limit.load();
+    p.grad_out = (const uint4 *)grad_out;
+    p.y = nullptr;
+    p.y_peers = grad_w ? (const uint8_t *const *)y_peers : nullptr;
+    p.dest = dest;
+    p.w = topk_w;
+    p.grad_y = nullptr;
+    p.grad_y_peers = (uint8_t *const *)grad_y_peers;
+    p.grad_w = grad_w;
+    p.ws = (int32_t *)ws;
+    p.ep_tag = rank + 1;
+    int64_t grid = d->backward_grid;
+    if (grid > T) grid = T;
+    if (grid < 1) grid = 1;
+    cudaError_t e = launch_combine_backward(p, (int)grid, smem, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "combine_backward kernel launch");
     return MOONEP_OK;
 }
 

@@ -18,6 +18,12 @@
 // in shared memory.  After a token's last chunk the consumers reduce the
 // partial sums (warp butterflies, then the 8 warps in order), so grad_w does
 // not depend on timing.  Every wait is bounded; no multicast.
+//
+// Expert parallelism (kEp): the tokens are one rank's (T = S) and a row
+// q * C_max + j of dest is row j of rank q's buffer.  The producer turns each
+// destination into two device addresses once per token (y through y_peers,
+// grad_y through grad_y_peers) and hands the grad_y address to the consumers
+// in shared memory, so the stores reach the peers' buffers directly.
 #include <cuda_bf16.h>
 
 #include "moonep_internal.cuh"
@@ -40,11 +46,12 @@ struct StageInfo {
     int32_t pad;
 };
 
+template <bool kEp>
 __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __grid_constant__ BackwardParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     int32_t *ws = p.ws;
     if (block_status_failed(ws)) return;
-    if (!cfg_matches(ws, p.cfg, num_ranges(p.T, (int64_t)p.cfg.R * p.cfg.L))) {
+    if (!cfg_matches(ws, p.cfg, num_ranges(p.T, (int64_t)p.cfg.R * p.cfg.L), p.ep_tag)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_CFG);
         return;
     }
@@ -60,7 +67,8 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
     StageInfo *info = reinterpret_cast<StageInfo *>(empty + kMaxStages);
     float *sw = reinterpret_cast<float *>(info + kMaxStages);        // [kMaxStages][kMaxK] weights
     int32_t *sd = reinterpret_cast<int32_t *>(sw + kMaxStages * kMaxK);  // [kMaxStages][kMaxK] dests
-    float *s_red = reinterpret_cast<float *>(sd + kMaxStages * kMaxK);   // [kMaxK][kConsumerWarps]
+    uint4 **sgy = reinterpret_cast<uint4 **>(sd + kMaxStages * kMaxK);   // [kMaxStages][kMaxK] grad_y rows (kEp)
+    float *s_red = reinterpret_cast<float *>(sgy + kMaxStages * kMaxK);   // [kMaxK][kConsumerWarps]
     float *s_part = s_red + kMaxK * kConsumerWarps;                       // [K][kConsumers]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -97,6 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
         int64_t cur = -1;
         int dk = 0, dk2 = 0;
         float wk = 0.f, wk2 = 0.f;
+        const uint8_t *yk = nullptr, *yk2 = nullptr;  // the K rows of y (kEp: on their ranks)
+        uint4 *gk = nullptr, *gk2 = nullptr;          // the K rows of grad_y (kEp)
         int valid = 1;
         bool bad = false, fail = false;
         int64_t i = 0;
@@ -121,15 +131,39 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
                 const bool okl = dk >= 0 && (int64_t)dk < p.rows_total && dk2 >= 0 && (int64_t)dk2 < p.rows_total;
                 valid = __all_sync(0xffffffffu, okl) ? 1 : 0;
                 bad |= !valid;
+                if (valid) {
+                    if (kEp) {
+                        const uint32_t Cm = (uint32_t)p.cfg.C_max;
+                        const uint32_t q = (uint32_t)dk / Cm, q2 = (uint32_t)dk2 / Cm;
+                        const int64_t j = (int64_t)((uint32_t)dk - q * Cm), j2 = (int64_t)((uint32_t)dk2 - q2 * Cm);
+                        if (lane < K) {
+                            gk = reinterpret_cast<uint4 *>(__ldg(reinterpret_cast<const uint64_t *>(p.grad_y_peers) + q)) +
+                                 j * p.hv;
+                            if (want_w) yk = reinterpret_cast<const uint8_t *>(
+                                                 __ldg(reinterpret_cast<const uint64_t *>(p.y_peers) + q)) + j * row_bytes;
+                        }
+                        if (lane + 32 < K) {
+                            gk2 = reinterpret_cast<uint4 *>(__ldg(reinterpret_cast<const uint64_t *>(p.grad_y_peers) + q2)) +
+                                  j2 * p.hv;
+                            if (want_w) yk2 = reinterpret_cast<const uint8_t *>(
+                                                  __ldg(reinterpret_cast<const uint64_t *>(p.y_peers) + q2)) + j2 * row_bytes;
+                        }
+                    } else if (want_w) {
+                        yk = ysrc + (int64_t)dk * row_bytes;
+                        yk2 = ysrc + (int64_t)dk2 * row_bytes;
+                    }
+                }
             }
             const uint32_t bytes = c == p.upt - 1 ? last : CH;
             if (lane < K) {
                 sw[s * kMaxK + lane] = wk;
                 sd[s * kMaxK + lane] = dk;
+                if (kEp) sgy[s * kMaxK + lane] = gk;
             }
             if (lane + 32 < K) {
                 sw[s * kMaxK + lane + 32] = wk2;
                 sd[s * kMaxK + lane + 32] = dk2;
+                if (kEp) sgy[s * kMaxK + lane + 32] = gk2;
             }
             __syncwarp();  // every lane's weights and rows before lane 0's release
             if (lane == 0) {
@@ -144,12 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
                 uint8_t *st = stages + (size_t)s * stage_bytes;
                 if (lane == 0) bulk_g2s(st, gsrc + t * row_bytes + (int64_t)c * CH, bytes, &full[s], pol);
                 if (want_w) {
-                    if (lane < K)
-                        bulk_g2s(st + (size_t)(1 + lane) * CH, ysrc + (int64_t)dk * row_bytes + (int64_t)c * CH,
-                                 bytes, &full[s], pol);
+                    if (lane < K) bulk_g2s(st + (size_t)(1 + lane) * CH, yk + (int64_t)c * CH, bytes, &full[s], pol);
                     if (lane + 32 < K)
-                        bulk_g2s(st + (size_t)(33 + lane) * CH, ysrc + (int64_t)dk2 * row_bytes + (int64_t)c * CH,
-                                 bytes, &full[s], pol);
+                        bulk_g2s(st + (size_t)(33 + lane) * CH, yk2 + (int64_t)c * CH, bytes, &full[s], pol);
                 }
             }
         }
@@ -177,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
                 const uint8_t *st = stages + (size_t)s * stage_bytes;
                 const float *wv = sw + s * kMaxK;
                 const int32_t *dv = sd + s * kMaxK;
+                uint4 *const *gv_rows = sgy + s * kMaxK;
                 const int nv = (int)(inf.bytes >> 4);
                 const int64_t col = (int64_t)inf.c * (CH >> 4);
                 for (int v = ct; v < nv; v += kConsumers) {
@@ -196,7 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             oh[q] = __floats2bfloat162_rn(__fmul_rn(w, gf[2 * q]), __fmul_rn(w, gf[2 * q + 1]));
-                        __stcs(p.grad_y + (int64_t)dv[k] * p.hv + col + v, o);
+                        uint4 *dst = kEp ? gv_rows[k] : p.grad_y + (int64_t)dv[k] * p.hv;
+                        __stcs(dst + col + v, o);
                         if (want_w) {
                             const uint4 yv = *reinterpret_cast<const uint4 *>(st + (size_t)(1 + k) * CH + (size_t)v * 16);
                             const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&yv);
@@ -241,13 +274,17 @@ __global__ void __launch_bounds__(kThreads, 1) combine_backward_kernel(const __g
 
 // chunk: the row split into the fewest equal pieces (multiples of 16 bytes,
 // at most 32 KB) such that three stages of (1 + K) pieces fit in shared
-// memory beside the fixed tables; large bulk copies move the most bytes
+// memory beside the fixed tables; large bulk copies move the most bytes.
+// Both forms of the kernel use the same layout (the grad_y row pointers are
+// reserved in the single-GPU form too), so they split rows alike and sum
+// grad_w in the same order.
 cudaError_t combine_backward_config(int K, int hv, bool with_grad_w, uint32_t *chunk, int *upt, int *stages,
                                     size_t *smem) {
     if (K < 1 || K > kMaxK || hv < 1) return cudaErrorInvalidValue;
     const size_t rows = 1 + (with_grad_w ? (size_t)K : 0);
     const size_t fixed = 2 * kMaxStages * 8 + kMaxStages * sizeof(StageInfo) + 2 * kMaxStages * kMaxK * 4 +
-                         kMaxK * kConsumerWarps * 4 + (with_grad_w ? (size_t)K * kConsumers * 4 : 0) + 128;
+                         (size_t)kMaxStages * kMaxK * 8 + kMaxK * kConsumerWarps * 4 +
+                         (with_grad_w ? (size_t)K * kConsumers * 4 : 0) + 128;
     const size_t budget = 220 * 1024;
     if (fixed + rows * 16 * 3 > budget) return cudaErrorInvalidValue;
     const uint32_t row = (uint32_t)hv * 16;
@@ -269,10 +306,17 @@ cudaError_t combine_backward_config(int K, int hv, bool with_grad_w, uint32_t *c
 }
 
 cudaError_t launch_combine_backward(const BackwardParams &p, int grid, size_t smem, cudaStream_t s) {
+    if (p.grad_y_peers) {
+        static std::atomic<size_t> smem_set_ep[64];
+        cudaError_t err = set_smem_limit((const void *)combine_backward_kernel<true>, smem, smem_set_ep);
+        if (err != cudaSuccess) return err;
+        combine_backward_kernel<true><<<grid, kThreads, smem, s>>>(p);
+        return cudaGetLastError();
+    }
     static std::atomic<size_t> smem_set[64];
-    cudaError_t err = set_smem_limit((const void *)combine_backward_kernel, smem, smem_set);
+    cudaError_t err = set_smem_limit((const void *)combine_backward_kernel<false>, smem, smem_set);
     if (err != cudaSuccess) return err;
-    combine_backward_kernel<<<grid, kThreads, smem, s>>>(p);
+    combine_backward_kernel<false><<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -240,6 +240,11 @@ struct BackwardParams {
     uint4 *grad_y;
     float *grad_w;        // may be NULL
     int32_t *ws;
+    // expert parallelism (NULL otherwise): row dest[t][k] = q * C_max + j is
+    // row j of rank q's buffer, reached through these device tables [R]
+    const uint8_t *const *y_peers;
+    uint8_t *const *grad_y_peers;
+    int32_t ep_tag;       // rank + 1, or 0
 };
 
 struct CopyParams {

@@ -12,6 +12,11 @@ mapped from each home rank):
     moonep_ep_dispatch   rows written into the destination ranks' buffers
     (expert computation; a barrier so every rank's rows have landed)
     moonep_ep_combine    rows read back from the ranks that computed them
+  training, backward:
+    moonep_ep_combine_backward  grad of the dispatched rows written on the ranks
+                         that hold them (and the router weights' grad)
+    (expert backward; a barrier)
+    moonep_ep_dispatch_backward grad of the hidden states read back
     moonep_ep_reduce_grad replica gradients read (and cleared) on the receivers
 
 The data path runs in the library's kernels; this module only allocates,
@@ -91,6 +96,15 @@ class RankBuffers:
 
     def combine(self, y_peers, stream=None):
         mp.moonep_ep_combine(self.cfg, self.rank, self.ws, y_peers, self.dest, self.w, self.out, stream)
+
+    def combine_backward(self, grad_out, y_peers, grad_y_peers, grad_w=None, stream=None):
+        """grad_out [S][H] bf16 (int16) of this rank; grad_w [S][K] fp32 or None."""
+        mp.moonep_ep_combine_backward(self.cfg, self.rank, self.ws, grad_out, y_peers, self.dest, self.w,
+                                      grad_y_peers, grad_w, stream)
+
+    def dispatch_backward(self, grad_recv_peers, grad_x, stream=None):
+        """grad_x [S][H] bf16 (int16) of this rank, from every rank's grad_recv."""
+        mp.moonep_ep_dispatch_backward(self.cfg, self.rank, self.ws, grad_recv_peers, self.dest, grad_x, stream)
 
     def prefetch(self, w_home_peers, stream=None):
         mp.moonep_ep_prefetch(self.cfg, self.rank, self.ws, w_home_peers, self.w_slot, self.w_elems, stream)
@@ -189,6 +203,18 @@ class Emulation:
         yp = self.recv_peers if y_peers is None else y_peers
         for rb in self.ranks:
             rb.combine(yp, stream)
+
+    def combine_backward(self, grad_out, grad_y_peers, grad_w=None, y_peers=None, stream=None):
+        """grad_out, grad_w: per-rank lists ([S][H] bf16, [S][K] fp32 or
+        None); grad_y_peers: peer table of the ranks' grad_y buffers."""
+        yp = self.recv_peers if y_peers is None else y_peers
+        for r, rb in enumerate(self.ranks):
+            rb.combine_backward(grad_out[r], yp, grad_y_peers, None if grad_w is None else grad_w[r], stream)
+
+    def dispatch_backward(self, grad_recv_peers, grad_x, stream=None):
+        """grad_x: per-rank list of [S][H] bf16 outputs."""
+        for r, rb in enumerate(self.ranks):
+            rb.dispatch_backward(grad_recv_peers, grad_x[r], stream)
 
     def prefetch(self, stream=None):
         for rb in self.ranks:

@@ -87,6 +87,8 @@ _sig = {
     "moonep_ep_plan": ([_CP, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp], ctypes.c_int),
     "moonep_ep_dispatch": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_ep_combine": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_ep_combine_backward": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_ep_dispatch_backward": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_ep_prefetch": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _i64, _vp], ctypes.c_int),
     "moonep_ep_reduce_grad": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _i64, _vp], ctypes.c_int),
     "moonep_set_wait_limit": ([_i64], ctypes.c_int),
@@ -267,6 +269,17 @@ def moonep_ep_dispatch(cfg, rank, ws, x, topk_idx, recv_peers, dest, stream=None
 def moonep_ep_combine(cfg, rank, ws, y_peers, dest, topk_w, out, stream=None) -> None:
     _check(_lib.moonep_ep_combine(ctypes.byref(cfg_of(cfg)), int(rank), _p(ws), _p(y_peers), _p(dest),
                                   _p(topk_w), _p(out), _stream(stream)))
+
+
+def moonep_ep_combine_backward(cfg, rank, ws, grad_out, y_peers, dest, topk_w, grad_y_peers, grad_w=None,
+                               stream=None) -> None:
+    _check(_lib.moonep_ep_combine_backward(ctypes.byref(cfg_of(cfg)), int(rank), _p(ws), _p(grad_out), _p(y_peers),
+                                           _p(dest), _p(topk_w), _p(grad_y_peers), _p(grad_w), _stream(stream)))
+
+
+def moonep_ep_dispatch_backward(cfg, rank, ws, grad_recv_peers, dest, grad_x, stream=None) -> None:
+    _check(_lib.moonep_ep_dispatch_backward(ctypes.byref(cfg_of(cfg)), int(rank), _p(ws), _p(grad_recv_peers),
+                                            _p(dest), _p(grad_x), _stream(stream)))
 
 
 def moonep_ep_prefetch(cfg, rank, ws, w_home_peers, w_slot, elems_per_expert, stream=None) -> None:

@@ -3,9 +3,10 @@ ranks emulated on one device: each rank has its own workspace and buffers,
 peers are reached through peer-pointer tables, and the count all-gather is a
 copy (load_balancing_plan_b200.ep.Emulation).  Every rank's plan tables must
 equal the oracle's plan of the concatenated ids; each rank's destinations,
-receive rows, combined outputs, prefetched slots and reduced gradients must
-equal the oracle's (bit-exact; combine also within 4e-3 of the oracle's fp32
-sum).  The kernels of different ranks never wait for one another, so running
+receive rows, combined outputs, prefetched slots, reduced gradients and the
+backward pair's grad_y and grad_x must equal the oracle's (bit-exact; combine
+also within 4e-3 of the oracle's fp32 sum; grad_w within its fp32 dot-product
+bound).  The kernels of different ranks never wait for one another, so running
 them one after another on one GPU computes exactly what one GPU per rank
 would."""
 import numpy as np
@@ -118,6 +119,7 @@ def run_ep_compare(env, cfg, ids, w, seed=0, E=256, mode=0):
         assert np.all(g[~nz] == 0)
         if nz.any():
             assert np.max(np.abs(g[nz] - a[nz]) / np.abs(a[nz])) <= 4e-3
+    ep_backward_compare(env, em, cfg, opl, y_o, w, seed)
     # reduce_grad: each home rank's gradients, every receiver's cleared slots
     em.reduce_grad()
     torch.cuda.synchronize()
@@ -129,6 +131,42 @@ def run_ep_compare(env, cfg, ids, w, seed=0, E=256, mode=0):
         if B:
             assert np.array_equal(rb.g_rep.cpu().numpy().view(np.uint32), gr_o[r * B:(r + 1) * B].view(np.uint32)), r
     return em, opl
+
+
+def ep_backward_compare(env, em, cfg, opl, y_o, w, seed):
+    """The training backward pair, rank by rank: combine_backward writes
+    grad_y into the ranks that hold the rows (and grad_w from y read on
+    them); dispatch_backward then reads that grad_y back.  grad_y and grad_x
+    bit-exact to the oracle; grad_w within the fp32 bound of its H-term dot
+    product, |err| <= H * 2^-24 * sum |grad_out * y|."""
+    torch, mp, ep, harness = env
+    R, S, K, H, Cm = (cfg[n] for n in ("R", "S", "K", "H", "C_max"))
+    T = R * S
+    G = inputs.cb_bf16_np(seed + 7, inputs.STREAM_Y, np.arange(T * H)).reshape(T, H)
+    g_d = [harness.as_i16(G[r * S:(r + 1) * S]).to(rb.recv.device) for r, rb in enumerate(em.ranks)]
+    grad_y = [torch.full((max(Cm, 1), H), -1, dtype=torch.int16, device=rb.recv.device) for rb in em.ranks]
+    grad_w = [torch.full((max(S * K, 1),), float("nan"), dtype=torch.float32, device=rb.recv.device)
+              for rb in em.ranks]
+    grad_x = [torch.full((max(S, 1), H), -1, dtype=torch.int16, device=rb.recv.device) for rb in em.ranks]
+    gy_peers = ep.peer_table(grad_y, em.ranks[0].recv.device)
+    for r, rb in enumerate(em.ranks):
+        rb.combine_backward(g_d[r], em.recv_peers, gy_peers, grad_w[r])
+    for r, rb in enumerate(em.ranks):
+        rb.dispatch_backward(gy_peers, grad_x[r])
+    torch.cuda.synchronize()
+    for rb in em.ranks:
+        assert rb.read_plan(tables=False)["status"] & mp.ST_ERROR_MASK == 0
+    gy_o = np.full((R * Cm, H), 0xFFFF, np.uint16)
+    gw_o = oracle.combine_backward(cfg, opl["dest"], G, y_o, w, gy_o)
+    gx_o, _ = oracle.dispatch_backward(cfg, opl["dest"], gy_o)
+    d = np.asarray(opl["dest"]).reshape(-1, K)
+    f64 = lambda u: inputs.bf16_bits_to_f32_np(u).astype(np.float64)
+    mag = np.einsum("th,tkh->tk", np.abs(f64(G)), np.abs(f64(y_o)[d]))
+    for r in range(R):
+        assert np.array_equal(harness.to_u16(grad_y[r][:Cm]), gy_o[r * Cm:(r + 1) * Cm]), r
+        got = grad_w[r][:S * K].cpu().numpy().reshape(S, K).astype(np.float64)
+        assert np.all(np.abs(got - gw_o[r * S:(r + 1) * S]) <= H * 2.0 ** -24 * mag[r * S:(r + 1) * S] + 1e-30), r
+        assert np.array_equal(harness.to_u16(grad_x[r][:S]), gx_o[r * S:(r + 1) * S]), r
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
