@@ -63,7 +63,11 @@ def alg_bytes(cfg, n_replicas=0, n_rx=0, w_elems=0, g_elems=0):
     prefetch: read each replicated expert's P*H*I bf16 weights once, write
     them to every used slot.
     reduce_grad: read+write the home gradient of each replicated expert,
-    read+zero every replica (fp32).  plan: read the ids."""
+    read+zero every replica (fp32).  plan: read the ids.
+    combine_backward: read grad_out once and the K expert-output rows of each
+    token, write the K grad_y rows and grad_w, read weights and dest.
+    dispatch_backward: read the K grad rows of each token, write grad_x, read
+    dest."""
     T = cfg["R"] * cfg["S"]
     K, H = cfg["K"], cfg["H"]
     row = 2 * H
@@ -73,6 +77,8 @@ def alg_bytes(cfg, n_replicas=0, n_rx=0, w_elems=0, g_elems=0):
         prefetch=2 * w_elems * (n_rx + n_replicas),
         reduce_grad=4 * g_elems * (2 * n_rx + 2 * n_replicas),
         plan=4 * T * K,
+        combine_backward=T * row + 2 * T * K * row + 12 * T * K,
+        dispatch_backward=T * K * row + T * row + 4 * T * K,
     )
 
 
@@ -353,8 +359,9 @@ class Runner:
         kept = grad_y
         co = lambda: mp.moonep_copy_out(cfg, p.ws, p.recv, kept, s)
         res = {}
-        for name, fn, nbytes in (("combine_backward", cb, T * 2 * H + 2 * T * K * 2 * H + 12 * T * K),
-                                 ("dispatch_backward", db, T * K * 2 * H + T * 2 * H + 4 * T * K),
+        ab = alg_bytes(cfg)
+        for name, fn, nbytes in (("combine_backward", cb, ab["combine_backward"]),
+                                 ("dispatch_backward", db, ab["dispatch_backward"]),
                                  ("copy_out", co, 2 * T * K * 2 * H)):
             for _ in range(warmup):
                 fn()
@@ -722,9 +729,6 @@ def run_ep(args, peak):
     # one rank per GPU: every receiver reads its experts' weights from the
     # home rank itself, one read and one write per slot
     ab["prefetch"] = 2 * 2 * wl.w_elems * info["n_replicas"]
-    T, K, H = wl.T, wl.K, wl.H
-    ab["combine_backward"] = T * 2 * H + 2 * T * K * 2 * H + 12 * T * K
-    ab["dispatch_backward"] = T * K * 2 * H + T * 2 * H + 4 * T * K
     steps = args.extra_steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)] for _ in range(steps)]
     for i in range(steps):
@@ -971,7 +975,7 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
-KERNELS = ("plan", "prefetch", "dispatch", "combine", "reduce_grad")
+KERNELS = ("plan", "prefetch", "dispatch", "combine", "reduce_grad", "combine_backward", "dispatch_backward")
 
 
 class PlanOnly:
@@ -1016,8 +1020,16 @@ def run_only(args):
         prob.fill_weights(args.seed)
         prob.fill_g_rep(args.seed)
     prob.plan()
-    if k == "combine":
+    pre = 0
+    if k in ("combine", "combine_backward", "dispatch_backward"):
         prob.dispatch()
+        pre = 1
+    if k in ("combine_backward", "dispatch_backward"):
+        # the training backward pair on the dispatched rows: grad_out = x,
+        # the expert outputs = the dispatched rows
+        grad_y = torch.empty_like(prob.recv)
+        grad_w = torch.empty(prob.T * cfg["K"], dtype=torch.float32, device=prob.recv.device)
+        grad_x = torch.empty_like(prob.out)
     torch.cuda.synchronize()
     info = mp.moonep_plan_read(cfg, prob.ws)
     if info["status"] & mp.ST_ERROR_MASK:
@@ -1027,9 +1039,14 @@ def run_only(args):
     n_slot = int(slotted.sum())
     n_rx = len(set(np.asarray(tabs["rep_expert"])[slotted].tolist()))
     ab = alg_bytes(cfg, n_slot, n_rx, prob.w_elems, prob.g_elems)[k]
-    fn = {"plan": prob.plan, "prefetch": prob.prefetch, "dispatch": prob.dispatch,
-          "combine": prob.combine, "reduce_grad": prob.reduce_grad}[k]
     s = torch.cuda.current_stream()
+    if k == "combine_backward":
+        fn = lambda: mp.moonep_combine_backward(cfg, prob.ws, prob.x, prob.recv, prob.dest, prob.w, grad_y, grad_w, s)
+    elif k == "dispatch_backward":
+        fn = lambda: mp.moonep_dispatch_backward(cfg, prob.ws, prob.recv, prob.dest, grad_x, s)
+    else:
+        fn = {"plan": prob.plan, "prefetch": prob.prefetch, "dispatch": prob.dispatch,
+              "combine": prob.combine, "reduce_grad": prob.reduce_grad}[k]
     for _ in range(args.warmup):
         fn()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
@@ -1044,7 +1061,7 @@ def run_only(args):
         raise RuntimeError("%s failed: status 0x%x" % (k, info["status"]))
     peak, peak_kind = measured_peak()
     print(json.dumps({"kernel": k, "workload": wl_desc(wl, route, ", seed %d" % args.seed),
-                      "launches": args.warmup + args.steps + 1 + (k == "combine"), "us": round(us, 2),
+                      "launches": args.warmup + args.steps + 1 + pre, "us": round(us, 2),
                       "algorithmic_bytes": ab, "gbs": round(ab / us / 1e3, 1),
                       "frac_of_peak": round(ab / us / 1e3 / peak, 4), "peak_kind": peak_kind,
                       "n_replicas": info["n_replicas"], "replicated_experts": n_rx}), flush=True)
