@@ -383,7 +383,12 @@ class Runner:
         pipelined: two input and two output buffer sets, host-to-device copies
         on one stream, device-to-host copies on another, the hot path on the
         compute stream, ordered by events (a step's kernels wait for its
-        inputs; a buffer is refilled only after the step that used it)."""
+        inputs; a buffer is refilled only after the step that used it).
+        Returns (ms, h2d bytes, d2h bytes, link ms): the last is a separate
+        measurement of the host link alone, after the timed region: the same
+        steps' host-to-device and device-to-host copies, the same bytes and
+        buffers, the two directions at once, no kernels; it is the bound the
+        end-to-end time is compared with."""
         torch = self.torch
         p = self.prob
         T, K = self.prob.T, self.cfg["K"]
@@ -439,7 +444,31 @@ class Runner:
         p.ids, p.w, p.x, p.out = ids_d[0], w_d[0], x_d[0], out_d[0]
         h2d_bytes = ids_h.numel() * 4 + w_h.numel() * 4 + x_h.numel() * 2
         d2h_bytes = outs_h[0].numel() * 2
-        return a.elapsed_time(z), h2d_bytes, d2h_bytes
+
+        # the host link alone: both directions' copies of every step at once
+        def link(nsteps):
+            for i in range(nsteps):
+                b = i & 1
+                with torch.cuda.stream(h2d):
+                    ids_d[b][:n].copy_(ids_h, non_blocking=True)
+                    w_d[b][:n].copy_(w_h, non_blocking=True)
+                    x_d[b].copy_(x_h, non_blocking=True)
+                with torch.cuda.stream(d2h):
+                    outs_h[b].copy_(out_d[b], non_blocking=True)
+
+        link(2)
+        torch.cuda.synchronize()
+        la = torch.cuda.Event(enable_timing=True)
+        lh = torch.cuda.Event(enable_timing=True)
+        ld = torch.cuda.Event(enable_timing=True)
+        la.record(h2d)
+        d2h.wait_event(la)
+        link(steps)
+        lh.record(h2d)
+        ld.record(d2h)
+        torch.cuda.synchronize()
+        link_ms = max(la.elapsed_time(lh), la.elapsed_time(ld))
+        return a.elapsed_time(z), h2d_bytes, d2h_bytes, link_ms
 
 
 def bind_near_gpu(device_index):
@@ -602,8 +631,9 @@ def run_gpu(args):
     pool.wait()
     pool.close()
     e2e_steps = max(8, args.steps // 8)
-    e2e_ms, h2d, d2h = run.e2e(e2e_steps, 3)
+    e2e_ms, h2d, d2h, link_ms = run.e2e(e2e_steps, 3)
     max_e2e_ms, e2e_bytes = reduce_over_ranks(e2e_ms, (ab["dispatch"] + ab["combine"]) * e2e_steps, world)
+    max_link_ms, _ = reduce_over_ranks(link_ms, 0, world)
     route_main = run.route
     x_gb, recv_gb = run.prob.x.numel() * 2 / 1e9, run.prob.recv.numel() * 2 / 1e9
     with_grads = run.with_grads
@@ -653,7 +683,9 @@ def run_gpu(args):
                      "algorithmic_bytes": ab[dom], "traffic": traffic, "traffic_source": traffic_src},
         "e2e": {"value": round(e2e_bytes / (max_e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(max_e2e_ms / e2e_steps, 4)},
+                "ms_per_step": round(max_e2e_ms / e2e_steps, 4),
+                "host_link_ms_per_step": round(max_link_ms / e2e_steps, 4),
+                "frac_of_host_link": round(max_link_ms / max_e2e_ms, 4)},
         "gpu_launches": launches,
         "clocks": f["clocks"],
     }

@@ -32,7 +32,10 @@ namespace moonep {
 
 namespace {
 
-constexpr int kConsumerWarps = 8;
+#ifndef MOONEP_CB_WARPS
+#define MOONEP_CB_WARPS 8
+#endif
+constexpr int kConsumerWarps = MOONEP_CB_WARPS;
 constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kThreads = 32 + kConsumers;
 constexpr int kMaxStages = 8;
