@@ -715,9 +715,9 @@ def run_mid(args, peak):
     return out
 
 
-def run_ep(args, peak):
-    """The mid workload's step through the expert-parallel calls, its R = 8
-    ranks emulated on this GPU (each rank's own buffers, peers through
+def run_ep(args, peak, workload="mid"):
+    """A workload's step (mid by default) through the expert-parallel calls,
+    its R ranks emulated on this GPU (each rank's own buffers, peers through
     peer-pointer tables, the count all-gather a device copy): per rank count
     -> (gather) -> plan -> prefetch -> dispatch -> combine -> combine_backward
     -> dispatch_backward -> reduce_grad, rank after rank for each call.  Every kernel is launched once per rank;
@@ -726,7 +726,7 @@ def run_ep(args, peak):
     here."""
     import torch
     from load_balancing_plan_b200 import ep
-    wl = inputs.WORKLOADS["mid"]
+    wl = inputs.WORKLOADS[workload]
     cfg = wl.cfg()
     route = inputs.routing(wl.R, wl.L, wl.S, wl.K, 0, maxvio=wl.maxvio[0])
     em = ep.Emulation(cfg, w_elems=wl.w_elems, g_elems=wl.g_elems)
@@ -1113,8 +1113,9 @@ def main(argv=None):
                     help="overflow beyond a receiver's slots: headroom rows on the home rank, or remote "
                          "weights; one_group: receivers take replicas of one home group only")
     ap.add_argument("--no-sweep", action="store_true")
-    ap.add_argument("--only", choices=KERNELS, default=None,
-                    help="time one kernel alone on the workload (profiler captures)")
+    ap.add_argument("--only", choices=KERNELS + ("ep",), default=None,
+                    help="time one kernel alone on the workload (profiler captures); ep: the workload's "
+                         "expert-parallel step, its ranks emulated on this GPU")
     ap.add_argument("--no-extras", action="store_true",
                     help="only the main workload (no mid, inference or sweep figures)")
     ap.add_argument("--seeds", type=lambda v: [int(x) for x in v.split(",")], default=[0, 1, 2, 3, 4],
@@ -1132,6 +1133,14 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.only == "ep":
+        # the expert-parallel step alone (ranks emulated on this GPU), for
+        # profiler captures: 3 untimed steps, then --steps timed ones
+        import torch
+        torch.cuda.set_device(0)
+        peak, _ = measured_peak()
+        args.extra_steps = args.steps
+        print(json.dumps(dict(run_ep(args, peak, args.workload), kernel="ep")), flush=True)
     elif args.only:
         run_only(args)
     else:
