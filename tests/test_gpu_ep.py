@@ -297,6 +297,8 @@ def test_ep_and_single_gpu_workspaces_do_not_mix(env):
     (4, 3, 50, 1, 24, 2, 1.0),       # K = 1, H not a multiple of 64
     (8, 2, 40, 2, 64, 0, 6.0),       # no prefetch slots: every spill falls back
     (3, 5, 7, 3, 16, 5, 1.0),        # ranges of a token or two, odd R
+    (8, 8, 40, 64, 16, 8, 0.0),      # K at its maximum: a second id per producer lane
+    (2, 2, 300, 2, 20008, 2, 1.0),   # long rows: several chunks per token in the gathers
 ])
 def test_ep_edge_cases(env, case):
     R, L, S, K, H, B, headroom = case
