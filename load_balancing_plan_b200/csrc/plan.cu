@@ -88,6 +88,12 @@ constexpr int kIdBatch = MOONEP_ID_BATCH;
 #define MOONEP_WARP_PLANNER_MAX_N 32
 #endif
 constexpr int kWarpPlannerMaxN = MOONEP_WARP_PLANNER_MAX_N;
+// The receiver walk: first all receivers at once, checked, then one after
+// another only if a chunk limit stops some receiver (1); always one after
+// another (0).  On 16 receivers the sequential walk took 5-7 us of the plan.
+#ifndef MOONEP_PLAN_SPEC_WALK
+#define MOONEP_PLAN_SPEC_WALK 1
+#endif
 
 // Exclusive scan of n ints (in and out may alias) by one warp; returns the
 // total.  Lane l owns the contiguous run [l*per, (l+1)*per), per = ceil(n/32).
@@ -138,6 +144,19 @@ __device__ int block_excl_scan(const int *in, int *out, int n, int *s_tmp) {
     return total;
 }
 
+// first m in [0, M) with a[m] > v, or M (a strictly increasing); one thread
+__device__ __forceinline__ int first_above(const int *a, int M, int v) {
+    int lo = 0, hi = M;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (a[mid] > v)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    return lo;
+}
+
 // first m >= i with ce[m] > v (ce strictly increasing over [0, M)); warp-wide
 __device__ int advance_chunk(const int *ce, int M, int i, int v) {
     const int lane = threadIdx.x & 31;
@@ -155,10 +174,34 @@ __device__ int advance_chunk(const int *ce, int M, int i, int v) {
 
 // Bounded grid barrier over gridDim.x CTAs (counters zeroed by the caller's
 // memset before the launch).  Returns false if this CTA gave up waiting.
+// MOONEP_BARRIER_ONCE (the default) builds the form for a kernel that passes
+// one barrier per launch: thread 0 of each CTA releases the CTA's writes
+// (the CTA barrier orders them before its fence) and adds one to the
+// counter, then waits until the counter reaches the grid size; no
+// generation word and no reset, so the last CTA to arrive is not delayed by
+// two more atomics.  0 builds the reusable form with a generation word.
+#ifndef MOONEP_BARRIER_ONCE
+#define MOONEP_BARRIER_ONCE 1
+#endif
 __device__ bool grid_barrier(int32_t *ws, int64_t limit) {
     __shared__ int s_ok;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (MOONEP_BARRIER_ONCE && threadIdx.x == 0) {
+        volatile int32_t *count = ws + HDR_BAR_COUNT;
+        __threadfence();
+        atomicAdd(ws + HDR_BAR_COUNT, 1);
+        bool ok = true;
+        int64_t n = 0;
+        while (*count < (int)gridDim.x) {
+            if (++n > limit) {
+                ok = false;
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence();
+        s_ok = ok;
+    } else if (!MOONEP_BARRIER_ONCE && threadIdx.x == 0) {
         volatile int32_t *gen = ws + HDR_BAR_GEN;
         int g = *gen;
         __threadfence();
@@ -289,8 +332,62 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         // receiver walk: receiver r takes the stream from p_r until its
         // deficit is filled or (headroom rule) it has touched B chunks or
         // (one-group rule) the stream leaves its first chunk's home group
-        int pos = 0, i0 = 0;
-        for (int r = 0; r < R; ++r) {
+        int pos = 0;
+        bool walked = false;
+#if MOONEP_PLAN_SPEC_WALK
+        {
+            // All receivers at once, two per lane: if no chunk limit stops a
+            // receiver, receiver r starts at min(D_r, total) (D_r: the
+            // deficits of the receivers before it that take part) and takes
+            // min(d_r, total - start).  Each lane then checks its receivers'
+            // limits at those starts; if every take fits, these starts and
+            // takes are exactly the walk's (each receiver's take is the
+            // walk's take at the walk's start, by induction over r), else
+            // the walk below runs one receiver after another.
+            int a[2], st[2], tk[2], ci[2], np[2];
+            bool ok = true;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = lane + 32 * h;
+                a[h] = (r < R && (remote || B > 0)) ? max(s_def[r], 0) : 0;
+            }
+            const int ia = warp_incl_scan(a[0]);
+            const int ta = __shfl_sync(0xffffffffu, ia, 31);
+            const int ib = warp_incl_scan(a[1]);
+            const int da[2] = {ia - a[0], ta + ib - a[1]};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                st[h] = min(da[h], total_spill);
+                tk[h] = min(a[h], total_spill - st[h]);
+                ci[h] = 0;
+                np[h] = 0;
+                if (tk[h] > 0) {
+                    const int i0 = first_above(s_ce, M, st[h]);
+                    int i1 = remote ? M - 1 : min(i0 + B - 1, M - 1);
+                    if (one_group) i1 = min(i1, first_above(s_ch, M, (s_ch[i0] / L + 1) * L - 1) - 1);
+                    if (s_ce[i1] - st[h] < tk[h]) ok = false;
+                    ci[h] = i0;
+                    np[h] = first_above(s_ce, M, st[h] + tk[h] - 1) - i0 + 1;
+                }
+            }
+            walked = __all_sync(0xffffffffu, ok);
+            if (walked) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = lane + 32 * h;
+                    if (r < R) {
+                        s_rp[r] = st[h];
+                        s_rt[r] = tk[h];
+                        s_ri0[r] = ci[h];
+                        s_rnp[r] = np[h];
+                    }
+                }
+                pos = min(ta + __shfl_sync(0xffffffffu, ib, 31), total_spill);
+            }
+        }
+#endif
+        int i0 = 0;
+        for (int r = 0; r < R && !walked; ++r) {
             const int d = s_def[r];
             int take = 0, np = 0, ir = i0;
             const int pr = pos;
@@ -649,7 +746,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     if (blockIdx.x == 0) TRACE(ws, 1);
     if (blockIdx.x == 0 && tid < 8) ws[HDR_CFG + tid] = (&p.cfg.R)[tid];
     if (blockIdx.x == 0 && tid == 0) ws[HDR_NRANGES] = (int32_t)p.Q;
-    __threadfence();
+    if (!MOONEP_BARRIER_ONCE) __threadfence();
 
     if (!grid_barrier(ws, p.wait_limit)) {
         if (tid == 0) atomicOr(ws + HDR_STATUS, MOONEP_ST_TIMEOUT);
