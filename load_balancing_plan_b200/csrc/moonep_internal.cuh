@@ -185,6 +185,7 @@ struct PlanParams {
     int32_t rank;              // expert-parallel rank (kPlanCount, kPlanFromCounts)
     int32_t *counts_out;       // kPlanCount: [N + 1] (counts, then status bits)
     const int32_t *counts_all; // kPlanFromCounts: [R][N + 1], every rank's counts_out
+    uint64_t mK, mT;           // floor((2^64 - 1) / d) + 1 for d = K and d = T (set at launch)
 };
 
 struct DispatchParams {

@@ -94,6 +94,19 @@ constexpr int kWarpPlannerMaxN = MOONEP_WARP_PLANNER_MAX_N;
 #ifndef MOONEP_PLAN_SPEC_WALK
 #define MOONEP_PLAN_SPEC_WALK 1
 #endif
+// Counting: the block's totals per expert from its histogram's columns after
+// the counting (1) or by a second shared-memory atomic per id (0); the
+// token and range of an id by multiply-high with a reciprocal made at launch
+// (1) or by 32-bit division (0).  floor(n / d) = hi64(n * m) with
+// m = floor((2^64 - 1) / d) + 1 holds for every n, d < 2^32, d >= 2: m
+// exceeds 2^64 / d by at most 1, so n * m / 2^64 exceeds n / d by less than
+// 2^-32 < 1 / d, which cannot carry n / d past the next integer.
+#ifndef MOONEP_PLAN_TOT_SUM
+#define MOONEP_PLAN_TOT_SUM 0  // 1 measured no faster alone, and slower with the multiply-high division
+#endif
+#ifndef MOONEP_PLAN_FASTDIV
+#define MOONEP_PLAN_FASTDIV 1
+#endif
 
 // Exclusive scan of n ints (in and out may alias) by one warp; returns the
 // total.  Lane l owns the contiguous run [l*per, (l+1)*per), per = ceil(n/32).
@@ -703,11 +716,20 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
                 if (i < i1) {
                     if ((unsigned)v[u] < (unsigned)N) {
                         // the range of token i / K: the last q with q*T/Q <= t
-                        const int64_t t = (int64_t)((uint32_t)i / (uint32_t)K);  // i < T*K < 2^31
-                        const int64_t q = div32 ? (int64_t)(((uint32_t)(t + 1) * (uint32_t)p.Q - 1u) / (uint32_t)p.T)
-                                                : ((t + 1) * p.Q - 1) / p.T;
+                        int64_t t, q;
+                        if (MOONEP_PLAN_FASTDIV) {
+                            const uint32_t iu = (uint32_t)i;  // i < T*K < 2^31
+                            t = K == 1 ? (int64_t)iu : (int64_t)__umul64hi((uint64_t)iu, p.mK);
+                            const uint32_t nq = (uint32_t)(t + 1) * (uint32_t)p.Q - 1u;
+                            q = div32 ? (p.T == 1 ? (int64_t)nq : (int64_t)__umul64hi((uint64_t)nq, p.mT))
+                                      : ((t + 1) * p.Q - 1) / p.T;
+                        } else {
+                            t = (int64_t)((uint32_t)i / (uint32_t)K);  // i < T*K < 2^31
+                            q = div32 ? (int64_t)(((uint32_t)(t + 1) * (uint32_t)p.Q - 1u) / (uint32_t)p.T)
+                                      : ((t + 1) * p.Q - 1) / p.T;
+                        }
                         atomicAdd(&sm[(q - qa) * N + v[u]], 1);
-                        atomicAdd(&tot[v[u]], 1);
+                        if (!MOONEP_PLAN_TOT_SUM) atomicAdd(&tot[v[u]], 1);
                     } else {
                         bad = true;
                     }
@@ -717,7 +739,13 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
         __syncthreads();
         if (blockIdx.x == 1) TRACE(ws, 10);
         for (int e = tid; e < N; e += kPlanThreads) {
-            const int c = tot[e];
+            int c = 0;
+            if (MOONEP_PLAN_TOT_SUM) {
+#pragma unroll 8
+                for (int r = 0; r < nr; ++r) c += sm[r * N + e];
+            } else {
+                c = tot[e];
+            }
             ws[lay.blk + (int64_t)e * NB + b] = c;
             if (c) atomicAdd(cnt_acc + e, c);
         }
@@ -794,7 +822,12 @@ size_t plan_smem_bytes(int N) {
 
 const void *plan_kernel_ptr() { return (const void *)plan_kernel; }
 
-cudaError_t launch_plan(const PlanParams &p, int grid, size_t smem, cudaStream_t s) {
+static uint64_t reciprocal64(int64_t d) { return d >= 2 ? ~uint64_t(0) / (uint64_t)d + 1 : 0; }
+
+cudaError_t launch_plan(const PlanParams &p_in, int grid, size_t smem, cudaStream_t s) {
+    PlanParams p = p_in;
+    p.mK = reciprocal64(p.cfg.K);
+    p.mT = reciprocal64(p.T);
     if (p.mode == kPlanFromCounts) {
         static std::atomic<size_t> smem_set[64];
         cudaError_t err = set_smem_limit((const void *)plan_from_counts_kernel, smem, smem_set);
