@@ -186,6 +186,8 @@ def test_tiny_reduce_grad_full_size_grads(env):
     (2, 2, 4, 2, 1 << 20, 2, 1.0, "skew"),              # H at its maximum (2 MB rows)
     (2, 4, 64, 2, 16, 1024, 1.0, "skew"),               # B at its maximum
     (64, 2, 8, 2, 16, 1024, 1.0, "skew"),               # R * B at its maximum (65536 slots)
+    (1, 3, 1, 2, 16, 1, 0.0, "uniform"),                # one token (T = 1): range and token of each id
+    (2, 3, 1, 1, 16, 1, 1.0, "uniform"),                # one token per rank, K = 1
 ])
 def test_edge_cases(env, case):
     R, L, S, K, H, B, hr, kind = case
