@@ -136,7 +136,7 @@ typedef struct {
  * the first entry p of e with j < route_end[p]); seg_off, seg_len
  * [R][2L+B] (L local, B slot, L fallback segments per rank); alloc [N][R]
  * (rows of expert e on rank r, fallback included: the allocation table);
- * base [N][n_ranges] (copies of e in the earlier token ranges of the range's
+ * base [n_ranges][N] (copies of e in the earlier token ranges of the range's
  * block; written only where the range has a copy of e) and blk [N][n_blocks]
  * (copies of e in earlier blocks; a block is n_ranges / n_blocks consecutive
  * ranges): dispatch scratch, copy numbers start at base + blk.  Tables

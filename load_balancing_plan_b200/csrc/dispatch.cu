@@ -115,7 +115,7 @@ __device__ __forceinline__ void init_counters(const DispatchParams &p, int32_t *
                                               int64_t nids, int tid, int nthreads) {
     const int32_t *ws = p.ws;
     const int64_t NB = p.lay.n_blocks;
-    const int32_t *base = ws + p.lay.base + q;                          // base[e][q] = base[e * Q]
+    const int32_t *base = ws + p.lay.base + q * p.N;                    // base[q][e] = base[e]
     const int32_t *blk = ws + p.lay.blk + block_of_range(q, p.Q, NB);   // blk[e][b] = blk[e * NB]
     for (int64_t l0 = 0; l0 < nids; l0 += (int64_t)kInitBatch * nthreads) {
         int e[kInitBatch], v[kInitBatch];
@@ -127,7 +127,7 @@ __device__ __forceinline__ void init_counters(const DispatchParams &p, int32_t *
 #pragma unroll
         for (int u = 0; u < kInitBatch; ++u)
             if ((unsigned)e[u] < (unsigned)p.N)
-                v[u] = __ldg(base + (int64_t)e[u] * p.Q) + __ldg(blk + (int64_t)e[u] * NB);
+                v[u] = __ldg(base + e[u]) + __ldg(blk + (int64_t)e[u] * NB);
 #pragma unroll
         for (int u = 0; u < kInitBatch; ++u)
             if ((unsigned)e[u] < (unsigned)p.N) ctr[e[u]] = v[u];

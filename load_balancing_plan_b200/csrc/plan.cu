@@ -108,6 +108,13 @@ constexpr int kWarpPlannerMaxN = MOONEP_WARP_PLANNER_MAX_N;
 #define MOONEP_PLAN_FASTDIV 1
 #endif
 
+// The planner and its scans run once per plan, cold: after a step's GBs of
+// streaming no line of their code is in any cache, and each line fetched costs
+// a round trip to L2 or HBM.  Their loops are therefore not unrolled
+// (`#pragma unroll 1`): at 512 threads and up to a few thousand experts they
+// run one or a few iterations per thread, so unrolled copies only lengthen
+// the code.  Inside the training step this took the plan from 32.5 to 26 us.
+//
 // Exclusive scan of n ints (in and out may alias) by one warp; returns the
 // total.  Lane l owns the contiguous run [l*per, (l+1)*per), per = ceil(n/32).
 __device__ int warp_excl_scan(const int *in, int *out, int n) {
@@ -115,10 +122,12 @@ __device__ int warp_excl_scan(const int *in, int *out, int n) {
     const int per = (n + 31) >> 5;
     const int lo = min(lane * per, n), hi = min(lo + per, n);
     int sum = 0;
+    #pragma unroll 1
     for (int i = lo; i < hi; ++i) sum += in[i];
     const int incl = warp_incl_scan(sum);
     const int total = __shfl_sync(0xffffffffu, incl, 31);
     int run = incl - sum;
+    #pragma unroll 1
     for (int i = lo; i < hi; ++i) {
         const int v = in[i];
         out[i] = run;
@@ -135,6 +144,7 @@ __device__ int block_excl_scan(const int *in, int *out, int n, int *s_tmp) {
     const int per = (n + kPlanThreads - 1) / kPlanThreads;
     const int lo = min(tid * per, n), hi = min(lo + per, n);
     int sum = 0;
+    #pragma unroll 1
     for (int i = lo; i < hi; ++i) sum += in[i];
     const int incl = warp_incl_scan(sum);
     if (lane == 31) s_tmp[warp] = incl;
@@ -147,6 +157,7 @@ __device__ int block_excl_scan(const int *in, int *out, int n, int *s_tmp) {
     }
     __syncthreads();
     int run = s_tmp[warp] + incl - sum;
+    #pragma unroll 1
     for (int i = lo; i < hi; ++i) {
         const int v = in[i];
         out[i] = run;
@@ -241,25 +252,28 @@ __device__ bool grid_barrier(int32_t *ws, int64_t limit) {
     return s_ok != 0;
 }
 
-// Exclusive prefix of one expert's per-range counts, in place (one warp),
-// starting from carry0.
+// Exclusive prefix of one expert's per-block counts, in place (one warp),
+// starting from carry0.  The column has Q <= kBlocks entries (one per block
+// of token ranges): lane l owns the run [l*per, (l+1)*per), per =
+// ceil(Q / 32) <= kScanPer, so one warp scan covers the column.
+constexpr int kScanPer = (int)((kBlocks + 31) / 32);
 __device__ void scan_column(int32_t *col, int64_t Q, int carry0 = 0) {
     const int lane = threadIdx.x & 31;
-    int carry = carry0;
-    for (int64_t q0 = 0; q0 < Q; q0 += 32 * 16) {
-        int v[16];
+    const int per = (int)((Q + 31) >> 5);
+    const int lo = min(lane * per, (int)Q), hi = min(lo + per, (int)Q);
+    int v[kScanPer];
+    int sum = 0;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            int64_t q = q0 + u * 32 + lane;
-            v[u] = q < Q ? __ldcg(col + q) : 0;
-        }
+    for (int u = 0; u < kScanPer; ++u) {
+        v[u] = lo + u < hi ? __ldcg(col + lo + u) : 0;
+        sum += v[u];
+    }
+    const int incl = warp_incl_scan(sum);
+    int run = carry0 + incl - sum;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            int incl = warp_incl_scan(v[u]);
-            int64_t q = q0 + u * 32 + lane;
-            if (q < Q) col[q] = carry + incl - v[u];
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
+    for (int u = 0; u < kScanPer; ++u) {
+        if (lo + u < hi) col[lo + u] = run;
+        run += v[u];
     }
 }
 
@@ -304,6 +318,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     if (tid == 0) s_misc[4] = 0;
     // keep/spill: each home rank keeps rows in local-expert order up to C
     const int total = scan(s_cnt, s_x, N);
+    #pragma unroll 1
     for (int e = tid; e < N; e += NT) {
         const int h = e / L;
         const int hx = s_x[e] - s_x[h * L];
@@ -319,6 +334,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[lay.seg_off + h * SEG + (e - h * L)] = ho;
         ws[lay.seg_len + h * SEG + (e - h * L)] = k;
     }
+    #pragma unroll 1
     for (int h = tid; h < R; h += NT) {
         const int lo = s_x[h * L];
         const int hi = h + 1 < R ? s_x[(h + 1) * L] : total;
@@ -333,6 +349,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     // the spill stream and its chunks
     const int total_spill = scan(s_sp, s_x, N);  // s_x = A_e
     const int M = scan(s_y, s_y, N);             // s_y = chunk index
+    #pragma unroll 1
     for (int e = tid; e < N; e += NT)
         if (s_sp[e] > 0) {
             s_ce[s_y[e]] = s_x[e] + s_sp[e];
@@ -400,6 +417,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         }
 #endif
         int i0 = 0;
+        #pragma unroll 1
         for (int r = 0; r < R && !walked; ++r) {
             const int d = s_def[r];
             int take = 0, np = 0, ir = i0;
@@ -456,9 +474,11 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
             s_misc[3] = nrx;
         }
     }
+    #pragma unroll 1
     for (int e = tid; e < N; e += NT) s_y[e] = 0;  // pieces per expert
     sync();
     const int p_end = s_misc[0], P = s_misc[1], NSLOT = s_misc[2], nrx = s_misc[3];
+    #pragma unroll 1
     for (int r = tid; r < R; r += NT) {
         ws[lay.fill + r] = C - s_def[r] + s_rt[r];
         ws[lay.slots_used + r] = min(s_rnp[r], B);
@@ -469,8 +489,10 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
 
     // pieces (a warp per receiver), their slots and slot segments, route
     // entries and alloc entries
+    #pragma unroll 1
     for (int r = warp; r < R; r += NW) {
         const int npr = s_rnp[r];
+        #pragma unroll 1
         for (int b = lane; b < npr; b += 32) {
             const int i = s_ri0[r] + b;
             const int e = s_ch[i];
@@ -506,6 +528,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         }
     }
     // slots no piece took
+    #pragma unroll 1
     for (int idx = tid; idx < R * B; idx += NT) {
         const int r = idx / B, b = idx - r * B;
         if (b < s_rnp[r]) continue;
@@ -518,8 +541,10 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
         ws[lay.seg_off + sg] = fill;
         ws[lay.seg_len + sg] = 0;
     }
+    #pragma unroll 1
     for (int x = tid; x < nrx; x += NT) ws[lay.rx_expert + x] = s_ch[x];
     // fallback rows: the stream beyond the walk's end, per chunk (s_x: A_e -> fb_cnt)
+    #pragma unroll 1
     for (int e = tid; e < N; e += NT) {
         int fb = 0;
         if (s_sp[e] > 0) {
@@ -534,6 +559,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     scan(s_y, s_y, N);   // s_y = rep_ptr
     scan(s_x, s_ce, N);  // s_ce = exclusive prefix of fb_cnt
     int cap_err = 0;
+    #pragma unroll 1
     for (int e = tid; e < N; e += NT) {
         const int h = e / L;
         const int fbo = C + (s_ce[e] - s_ce[h * L]);
@@ -652,7 +678,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     // are loaded in one batch of up to kIdBatch per thread, so a block costs
     // about one memory latency however many ranges it holds.  The totals go
     // to blk[e][b] and into the global tokens_per_expert (cnt).  Then one
-    // thread per expert walks the block's ranges in order: base[e][q] =
+    // thread per expert walks the block's ranges in order: base[q][e] =
     // copies of e in the block's earlier ranges (stored only where range q
     // has a copy of e: a range of a few tokens routes to few experts, and
     // dispatch reads no other entry).
@@ -681,11 +707,13 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     auto walk = [&](int64_t qa, int nr) {
         for (int e = tid; e < N; e += kPlanThreads) {
             int run = 0;
+            int32_t *dst = ws + lay.base + qa * N + e;
+            const int *src = sm + e;
 #pragma unroll 8
-            for (int r = 0; r < nr; ++r) {
-                // dispatch reads base[e][q] only where range q routes to e
-                const int c = sm[r * N + e];
-                if (c) ws[lay.base + (int64_t)e * p.Q + qa + r] = run;
+            for (int r = 0; r < nr; ++r, dst += N, src += N) {
+                // dispatch reads base[q][e] only where range q routes to e
+                const int c = *src;
+                if (c) *dst = run;
                 run += c;
             }
         }
