@@ -41,9 +41,31 @@ def _torch():
 
 
 def peer_table(tensors, device):
-    """Device int64 array of the tensors' data pointers (a peer table)."""
+    """Device int64 array of the tensors' data pointers (a peer table).  The
+    table holds plain addresses: the caller keeps the tensors referenced for
+    as long as it is used (see PeerTable)."""
     torch = _torch()
     return torch.tensor([int(t.data_ptr()) for t in tensors], dtype=torch.int64, device=device)
+
+
+class PeerTable:
+    """A peer table together with the tensors it points into.  Keeping this
+    object keeps the tensors, and so the memory the kernels reach through the
+    table, alive: a tensor mapped from another process (exchange_buffers)
+    unmaps that process's memory when it is freed, after which a kernel given
+    the bare address would fault.  Pass the object itself wherever a peer
+    table is expected."""
+
+    def __init__(self, tensors, device):
+        self.tensors = list(tensors)
+        self.table = peer_table(self.tensors, device)
+
+    def data_ptr(self):
+        return self.table.data_ptr()
+
+
+def _table(t):
+    return t.table if isinstance(t, PeerTable) else t
 
 
 class RankBuffers:
@@ -91,26 +113,31 @@ class RankBuffers:
     def plan(self, flags=0, stream=None):
         mp.moonep_ep_plan(self.cfg, flags, self.rank, self.counts_all, self.ws, stream)
 
+    # peer tables: a PeerTable, or a device int64 tensor of addresses whose
+    # memory the caller keeps alive
     def dispatch(self, recv_peers, stream=None):
-        mp.moonep_ep_dispatch(self.cfg, self.rank, self.ws, self.x, self.ids, recv_peers, self.dest, stream)
+        mp.moonep_ep_dispatch(self.cfg, self.rank, self.ws, self.x, self.ids, _table(recv_peers), self.dest, stream)
 
     def combine(self, y_peers, stream=None):
-        mp.moonep_ep_combine(self.cfg, self.rank, self.ws, y_peers, self.dest, self.w, self.out, stream)
+        mp.moonep_ep_combine(self.cfg, self.rank, self.ws, _table(y_peers), self.dest, self.w, self.out, stream)
 
     def combine_backward(self, grad_out, y_peers, grad_y_peers, grad_w=None, stream=None):
         """grad_out [S][H] bf16 (int16) of this rank; grad_w [S][K] fp32 or None."""
-        mp.moonep_ep_combine_backward(self.cfg, self.rank, self.ws, grad_out, y_peers, self.dest, self.w,
-                                      grad_y_peers, grad_w, stream)
+        mp.moonep_ep_combine_backward(self.cfg, self.rank, self.ws, grad_out, _table(y_peers), self.dest, self.w,
+                                      _table(grad_y_peers), grad_w, stream)
 
     def dispatch_backward(self, grad_recv_peers, grad_x, stream=None):
         """grad_x [S][H] bf16 (int16) of this rank, from every rank's grad_recv."""
-        mp.moonep_ep_dispatch_backward(self.cfg, self.rank, self.ws, grad_recv_peers, self.dest, grad_x, stream)
+        mp.moonep_ep_dispatch_backward(self.cfg, self.rank, self.ws, _table(grad_recv_peers), self.dest, grad_x,
+                                       stream)
 
     def prefetch(self, w_home_peers, stream=None):
-        mp.moonep_ep_prefetch(self.cfg, self.rank, self.ws, w_home_peers, self.w_slot, self.w_elems, stream)
+        mp.moonep_ep_prefetch(self.cfg, self.rank, self.ws, _table(w_home_peers), self.w_slot, self.w_elems,
+                              stream)
 
     def reduce_grad(self, g_rep_peers, stream=None):
-        mp.moonep_ep_reduce_grad(self.cfg, self.rank, self.ws, self.g_home, g_rep_peers, self.g_elems, stream)
+        mp.moonep_ep_reduce_grad(self.cfg, self.rank, self.ws, self.g_home, _table(g_rep_peers), self.g_elems,
+                                 stream)
 
     def read_plan(self, tables=True):
         return mp.moonep_plan_read(self.cfg, self.ws, tables=tables)
@@ -146,7 +173,10 @@ def exchange_buffers(tensor, group=None):
     """Maps every rank's `tensor` into this process: returns a list of R
     tensors, entry q aliasing rank q's buffer (this rank's own tensor at its
     own index).  Uses CUDA IPC handles sent over the process group; every
-    rank's tensor must be a whole CUDA tensor of the same shape and dtype."""
+    rank's tensor must be a whole CUDA tensor of the same shape and dtype.
+    A mapped tensor unmaps the peer's memory when it is freed: keep the list
+    (or the PeerTable of map_peers) for as long as kernels use the
+    addresses."""
     import torch.distributed as dist
     from torch.multiprocessing.reductions import reduce_tensor
     me = dist.get_rank(group)
@@ -157,6 +187,12 @@ def exchange_buffers(tensor, group=None):
     for q, (f, a) in enumerate(got):
         out.append(tensor if q == me else f(*a))
     return out
+
+
+def map_peers(tensor, device, group=None):
+    """exchange_buffers and the device table of the mapped addresses, kept
+    together (a PeerTable)."""
+    return PeerTable(exchange_buffers(tensor, group), device)
 
 
 # ---------------------------------------------------------------------------
