@@ -514,7 +514,11 @@ __global__ void __launch_bounds__(kRgThreads, MOONEP_RG_MINB) reduce_grad_pipe_k
 
 }  // namespace
 
+#ifndef MOONEP_PREFETCH_CTAS_PER_SM
+#define MOONEP_PREFETCH_CTAS_PER_SM 1
+#endif
 cudaError_t launch_prefetch(const CopyParams &p, int grid, cudaStream_t s) {
+    grid *= MOONEP_PREFETCH_CTAS_PER_SM;
     const size_t smem = (size_t)kPfStages * kPfChunk + kPfStages * 8;
     if (p.peers) {
         static std::atomic<size_t> smem_set_ep[64];
