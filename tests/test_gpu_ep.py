@@ -325,3 +325,63 @@ def test_ep_empty_ranks(env):
         info = rb.read_plan(tables=False)
         assert info["status"] & mp.ST_ERROR_MASK == 0
         assert info["n_replicas"] == 0 and info["fallback_rows"] == 0
+
+
+@pytest.mark.parametrize("kernel", ["dispatch", "combine", "combine_backward", "prefetch"])
+def test_ep_wait_timeout_is_reported_and_recoverable(env, kernel):
+    # the expert-parallel forms give up after wait_limit polls (0 here) like
+    # the single-GPU ones: each rank either finishes or records
+    # MOONEP_ST_TIMEOUT in its own workspace and returns; the next plan
+    # clears the status and the step then matches the oracle
+    torch, mp, ep, harness = env
+    cfg = cfg_of(4, 4, 512, 4, 4096, 4, headroom=1.0)
+    R, S, K, H, Cm = 4, 512, 4, 4096, cfg["C_max"]
+    r = inputs.routing(4, 4, 512, 4, 0, alpha=1.0)
+    E = 64 * 1024
+    em = ep.Emulation(cfg, w_elems=E, poison=True)
+    em.set_routing(r.topk_idx, r.topk_w)
+    for q, rb in enumerate(em.ranks):
+        inputs.cb_fill_torch(rb.x.view(torch.bfloat16), 0, inputs.STREAM_X, offset=q * S * H)
+        inputs.cb_fill_torch(rb.w_home.view(torch.bfloat16), 0, inputs.STREAM_W, offset=q * 4 * E)
+    grad_y = [torch.zeros_like(rb.recv) for rb in em.ranks]
+    gy_peers = ep.PeerTable(grad_y, "cuda")
+
+    def run():
+        if kernel == "dispatch":
+            em.dispatch()
+            return [rb.dest.clone() for rb in em.ranks] + [rb.recv.clone() for rb in em.ranks]
+        if kernel == "combine":
+            em.combine()
+            return [rb.out.clone() for rb in em.ranks]
+        if kernel == "combine_backward":
+            em.combine_backward([rb.x for rb in em.ranks], gy_peers)
+            return [g.clone() for g in grad_y]
+        em.prefetch()
+        return [rb.w_slot.clone() for rb in em.ranks]
+
+    em.plan()
+    if kernel != "dispatch":
+        em.dispatch()
+    torch.cuda.synchronize()
+    try:
+        mp.moonep_set_wait_limit(0)
+        got = run()
+        torch.cuda.synchronize()
+        status = [rb.read_plan(tables=False)["status"] for rb in em.ranks]
+    finally:
+        mp.moonep_set_wait_limit(1 << 22)
+    for st in status:
+        assert st & mp.ST_ERROR_MASK & ~mp.ST_TIMEOUT == 0
+    em.plan()
+    em.dispatch()
+    ref = run()
+    torch.cuda.synchronize()
+    for rb in em.ranks:
+        assert rb.read_plan(tables=False)["status"] & mp.ST_ERROR_MASK == 0
+    if not any(st & mp.ST_TIMEOUT for st in status):
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)
+    # after recovery the step matches the oracle
+    opl = oracle.plan(cfg, r.topk_idx)
+    for q, rb in enumerate(em.ranks):
+        assert np.array_equal(rb.dest[:S * K].cpu().numpy(), opl["dest"][q].reshape(-1)), q
