@@ -22,9 +22,9 @@ mapped from each home rank):
 The data path runs in the library's kernels; this module only allocates,
 builds the peer-pointer tables and moves the counts between ranks.  Peers are
 reached through their buffers' device addresses as this GPU sees them: CUDA
-IPC mappings for one process per GPU (`exchange_buffers`), or plain local
-addresses when all ranks share one device (`Emulation`, used by the tests on
-one GPU).  The kernels never wait for another rank: the caller orders the
+IPC mappings for one process per GPU (`map_peers`, whose PeerTable keeps the
+mappings alive), or plain local addresses when all ranks share one device
+(`Emulation`, used by the tests on one GPU).  The kernels never wait for another rank: the caller orders the
 ranks between calls (stream order on one device; collectives or barriers
 across processes).
 """
