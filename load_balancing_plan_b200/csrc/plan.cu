@@ -168,6 +168,78 @@ __device__ int block_excl_scan(const int *in, int *out, int n, int *s_tmp) {
     return total;
 }
 
+// Two exclusive scans at once (a and b of n ints each; a's input and output
+// may alias, as may b's, but not one with the other): the same runs per
+// thread and the same barriers as one scan.  Returns both totals.
+__device__ int2 warp_excl_scan2(const int *ia, int *oa, const int *ib, int *ob, int n) {
+    const int lane = threadIdx.x & 31;
+    const int per = (n + 31) >> 5;
+    const int lo = min(lane * per, n), hi = min(lo + per, n);
+    int sa = 0, sb = 0;
+#pragma unroll 1
+    for (int i = lo; i < hi; ++i) {
+        sa += ia[i];
+        sb += ib[i];
+    }
+    const int xa = warp_incl_scan(sa), xb = warp_incl_scan(sb);
+    const int2 tot = make_int2(__shfl_sync(0xffffffffu, xa, 31), __shfl_sync(0xffffffffu, xb, 31));
+    int ra = xa - sa, rb = xb - sb;
+#pragma unroll 1
+    for (int i = lo; i < hi; ++i) {
+        const int a = ia[i], b = ib[i];
+        oa[i] = ra;
+        ob[i] = rb;
+        ra += a;
+        rb += b;
+    }
+    __syncwarp();
+    return tot;
+}
+
+// s_tmp holds 66 ints
+__device__ int2 block_excl_scan2(const int *ia, int *oa, const int *ib, int *ob, int n, int *s_tmp) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (n + kPlanThreads - 1) / kPlanThreads;
+    const int lo = min(tid * per, n), hi = min(lo + per, n);
+    int sa = 0, sb = 0;
+#pragma unroll 1
+    for (int i = lo; i < hi; ++i) {
+        sa += ia[i];
+        sb += ib[i];
+    }
+    const int xa = warp_incl_scan(sa), xb = warp_incl_scan(sb);
+    if (lane == 31) {
+        s_tmp[warp] = xa;
+        s_tmp[33 + warp] = xb;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int va = lane < kWarps ? s_tmp[lane] : 0, vb = lane < kWarps ? s_tmp[33 + lane] : 0;
+        const int ja = warp_incl_scan(va), jb = warp_incl_scan(vb);
+        if (lane < kWarps) {
+            s_tmp[lane] = ja - va;
+            s_tmp[33 + lane] = jb - vb;
+        }
+        if (lane == kWarps - 1) {
+            s_tmp[32] = ja;
+            s_tmp[65] = jb;
+        }
+    }
+    __syncthreads();
+    int ra = s_tmp[warp] + xa - sa, rb = s_tmp[33 + warp] + xb - sb;
+#pragma unroll 1
+    for (int i = lo; i < hi; ++i) {
+        const int a = ia[i], b = ib[i];
+        oa[i] = ra;
+        ob[i] = rb;
+        ra += a;
+        rb += b;
+    }
+    const int2 tot = make_int2(s_tmp[32], s_tmp[65]);
+    __syncthreads();
+    return tot;
+}
+
 // first m in [0, M) with a[m] > v, or M (a strictly increasing); one thread
 __device__ __forceinline__ int first_above(const int *a, int M, int v) {
     int lo = 0, hi = M;
@@ -300,7 +372,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     int *s_y = sm + 5 * N;    // chunk index, then pieces per expert -> rep_ptr
     int *s_hoff = sm + 6 * N; // row of the expert's local segment
     __shared__ int s_def[kMaxR], s_rp[kMaxR], s_rt[kMaxR], s_ri0[kMaxR], s_rnp[kMaxR], s_rpb[kMaxR], s_spb[kMaxR];
-    __shared__ int s_tmp[33];
+    __shared__ int s_tmp[66];
     __shared__ int s_misc[6];  // 0 p_end, 1 P, 2 NSLOT, 3 nrx, 4 capacity error
     const bool remote = (p.flags & MOONEP_PLAN_REMOTE_WEIGHTS) != 0;
     const bool one_group = (p.flags & MOONEP_PLAN_ONE_GROUP) != 0;
@@ -312,6 +384,9 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     };
     auto scan = [&](const int *in, int *out, int n) {
         return NT == 32 ? warp_excl_scan(in, out, n) : block_excl_scan(in, out, n, s_tmp);
+    };
+    auto scan2 = [&](const int *ia, int *oa, const int *ib, int *ob, int n) {
+        return NT == 32 ? warp_excl_scan2(ia, oa, ib, ob, n) : block_excl_scan2(ia, oa, ib, ob, n, s_tmp);
     };
 
     TRACE(ws, 3);
@@ -347,8 +422,9 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     sync();
 
     // the spill stream and its chunks
-    const int total_spill = scan(s_sp, s_x, N);  // s_x = A_e
-    const int M = scan(s_y, s_y, N);             // s_y = chunk index
+    // s_x = A_e (the spill stream's starts), s_y = chunk index
+    const int2 t2 = scan2(s_sp, s_x, s_y, s_y, N);
+    const int total_spill = t2.x, M = t2.y;
     #pragma unroll 1
     for (int e = tid; e < N; e += NT)
         if (s_sp[e] > 0) {
@@ -556,8 +632,7 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     }
     sync();
     TRACE(ws, 6);
-    scan(s_y, s_y, N);   // s_y = rep_ptr
-    scan(s_x, s_ce, N);  // s_ce = exclusive prefix of fb_cnt
+    scan2(s_y, s_y, s_x, s_ce, N);  // s_y = rep_ptr, s_ce = exclusive prefix of fb_cnt
     int cap_err = 0;
     #pragma unroll 1
     for (int e = tid; e < N; e += NT) {
