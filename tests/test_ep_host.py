@@ -85,3 +85,24 @@ def test_ranks_with_different_configurations_both_refuse():
     res = _run(_differ)
     for _, _, _, err in res:
         assert err is not None and "disagree" in err
+
+
+def test_peer_table_keeps_its_tensors():
+    # the table holds plain addresses; the PeerTable object holds the tensors
+    # behind them, so they live as long as the table is in use
+    import gc
+    import weakref
+    import torch
+    from load_balancing_plan_b200 import ep
+    ts = [torch.zeros(4, dtype=torch.int32) for _ in range(3)]
+    refs = [weakref.ref(t) for t in ts]
+    pt = ep.PeerTable(ts, "cpu")
+    assert pt.table.tolist() == [t.data_ptr() for t in ts]
+    assert pt.data_ptr() == pt.table.data_ptr()
+    assert ep._table(pt) is pt.table and ep._table(pt.table) is pt.table
+    del ts
+    gc.collect()
+    assert all(r() is not None for r in refs)
+    del pt
+    gc.collect()
+    assert all(r() is None for r in refs)
