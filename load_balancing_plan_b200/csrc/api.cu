@@ -11,6 +11,11 @@
 
 #include "moonep_internal.cuh"
 
+#ifndef MOONEP_DISPATCH_MAX_CTAS
+#define MOONEP_DISPATCH_MAX_CTAS 2  // resident dispatch CTAs per SM the shared memory is sized for
+                                    // (4 and 5 give smaller pieces and ran 3-4% slower)
+#endif
+
 using namespace moonep;
 
 namespace {
@@ -240,9 +245,11 @@ int moonep_dispatch(const moonep_cfg_t *cfg, void *ws, const void *x, const int3
     p.Q = p.lay.n_ranges;
     p.row_bytes = (uint32_t)cfg->H * 2;
     size_t smem = 0;
-    // two resident CTAs per SM; ranges beyond those run in later waves
+    // shared memory sized for two resident CTAs per SM (at H = 7168 this
+    // comes to 66 KB, so the SM holds three); ranges beyond those run in
+    // later waves
     int ctas_per_sm = (int)((p.Q + d->sms - 1) / d->sms);
-    if (ctas_per_sm > 2) ctas_per_sm = 2;
+    if (ctas_per_sm > MOONEP_DISPATCH_MAX_CTAS) ctas_per_sm = MOONEP_DISPATCH_MAX_CTAS;
     cudaError_t e = dispatch_smem_config(N, p.row_bytes, ctas_per_sm < 1 ? 1 : ctas_per_sm, &p.piece_bytes, &p.npc,
                                          &smem);
     if (e != cudaSuccess) return fail(MOONEP_ERR_ARG, "dispatch: no shared-memory configuration for H=%d", cfg->H);
@@ -536,7 +543,7 @@ int moonep_ep_dispatch(const moonep_cfg_t *cfg, int32_t rank, void *ws, const vo
     p.row_bytes = (uint32_t)cfg->H * 2;
     size_t smem = 0;
     int ctas_per_sm = (int)((p.Q + d->sms - 1) / d->sms);
-    if (ctas_per_sm > 2) ctas_per_sm = 2;
+    if (ctas_per_sm > MOONEP_DISPATCH_MAX_CTAS) ctas_per_sm = MOONEP_DISPATCH_MAX_CTAS;
     cudaError_t e = dispatch_smem_config(N, p.row_bytes, ctas_per_sm < 1 ? 1 : ctas_per_sm, &p.piece_bytes, &p.npc,
                                          &smem, true);
     if (e != cudaSuccess) return fail(MOONEP_ERR_ARG, "dispatch: no shared-memory configuration for H=%d", cfg->H);

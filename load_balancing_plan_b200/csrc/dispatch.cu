@@ -384,6 +384,9 @@ __global__ void __launch_bounds__(32 * (1 + kLoaderWarps), 1)
 
 }  // namespace
 
+#ifndef MOONEP_DISPATCH_FILL_SMEM
+#define MOONEP_DISPATCH_FILL_SMEM 0  // 1: at most ctas_per_sm resident CTAs (two: 25% slower than three)
+#endif
 // Shared memory: kStages pieces + barriers + ring + N counters (+ the peer
 // table under expert parallelism), sized so that `ctas_per_sm` CTAs fit one
 // SM (227 KB usable per SM on sm_100).
@@ -406,6 +409,11 @@ cudaError_t dispatch_smem_config(int N, uint32_t row_bytes, int ctas_per_sm, uin
     *piece_bytes = pb;
     *npc = n;
     *smem = (size_t)kStages * pb + fixed;
+#if MOONEP_DISPATCH_FILL_SMEM
+    // take the whole per-CTA budget, so that no more than ctas_per_sm CTAs
+    // are resident on an SM
+    if (*smem < budget) *smem = budget;
+#endif
     return cudaSuccess;
 }
 

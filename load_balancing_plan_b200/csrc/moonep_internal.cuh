@@ -43,7 +43,10 @@ enum : int {
 // with 16-token ranges and 734 with one 110-token range per resident CTA.  Q
 // is a whole number of such waves, so the last wave is full, and at most
 // kBaseWords / N so that the per-(expert, range) table stays small.
-constexpr int64_t kMinRanges = 296;
+#ifndef MOONEP_MIN_RANGES
+#define MOONEP_MIN_RANGES 296
+#endif
+constexpr int64_t kMinRanges = MOONEP_MIN_RANGES;
 #ifndef MOONEP_RANGE_TOKENS
 #define MOONEP_RANGE_TOKENS 4
 #endif
