@@ -720,9 +720,10 @@ def run_mid(args, peak):
 def run_ep(args, peak, workload="mid"):
     """A workload's step (mid by default) through the expert-parallel calls,
     its R ranks emulated on this GPU (each rank's own buffers, peers through
-    peer-pointer tables, the count all-gather a device copy): per rank count
-    -> (gather) -> plan -> prefetch -> dispatch -> combine -> combine_backward
-    -> dispatch_backward -> reduce_grad, rank after rank for each call.  Every kernel is launched once per rank;
+    peer-pointer tables; each rank's counting launch stores its counts into
+    every rank's counts_all): per rank count -> plan -> prefetch -> dispatch
+    -> combine -> combine_backward -> dispatch_backward -> reduce_grad, rank
+    after rank for each call.  Every kernel is launched once per rank;
     the figures are the sums over the ranks' launches (CUDA events around
     each phase on the launching stream).  One GPU per rank is not measured
     here."""
@@ -746,7 +747,7 @@ def run_ep(args, peak, workload="mid"):
     grad_w = [torch.empty_like(rb.w) for rb in em.ranks]
     grad_x = [torch.empty_like(rb.x) for rb in em.ranks]
     grad_out = [rb.out for rb in em.ranks]
-    phases = [("plan", em.plan), ("prefetch", em.prefetch), ("dispatch", em.dispatch),
+    phases = [("plan", lambda: em.plan(exchange=True)), ("prefetch", em.prefetch), ("dispatch", em.dispatch),
               ("combine", em.combine),
               ("combine_backward", lambda: em.combine_backward(grad_out, grad_y_peers, grad_w)),
               ("dispatch_backward", lambda: em.dispatch_backward(grad_y_peers, grad_x)),
@@ -777,8 +778,8 @@ def run_ep(args, peak, workload="mid"):
     dc = ab["dispatch"] + ab["combine"]
     value = dc / ((us["dispatch"] + us["combine"]) * 1e-6) / 1e9
     out = {"workload": wl_desc(wl, route, ", seed 0; %d ranks emulated on one GPU" % wl.R),
-           "step": "per rank: count -> (all-gather) -> plan -> prefetch -> dispatch -> combine -> combine_backward "
-                   "-> dispatch_backward -> reduce_grad",
+           "step": "per rank: count with the counts' exchange (moonep_ep_count_exchange) -> plan -> prefetch -> "
+                   "dispatch -> combine -> combine_backward -> dispatch_backward -> reduce_grad",
            "value": round(value, 2), "unit": UNIT, "dispatch_combine_frac_of_peak": round(value / peak, 4),
            "ms_per_step": round(total_ms, 4), "launch": "eager, one launch per rank and call",
            "phase_us": {k: round(v, 2) for k, v in us.items()},

@@ -370,6 +370,17 @@ MOONEP_API size_t moonep_ep_workspace_bytes(const moonep_cfg_t *cfg);
 MOONEP_API int moonep_ep_count(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_idx, void *ws,
                                int32_t *counts, void *stream);
 
+/* Steps 1 and 2 in one launch: moonep_ep_count, and the rank's finished
+ * counts [N + 1] stored into row `rank` of every rank's counts_all.
+ * counts_all_peers: device table of R pointers, entry q to rank q's
+ * counts_all (device int32 [R][N + 1]) as this GPU addresses it.  The last
+ * counting CTA to finish stores the row (plain stores, no multicast; no CTA
+ * waits for another); once every rank's launch has completed (the caller's
+ * barrier), each rank's counts_all is what the all-gather of step 2 would
+ * have left.  Also launches with S = 0, to store the rank's zero row. */
+MOONEP_API int moonep_ep_count_exchange(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_idx, void *ws,
+                                        int32_t *counts, int32_t *const *counts_all_peers, void *stream);
+
 /* Step 3.  counts_all: device int32 [R][N + 1], row q = rank q's counts.
  * flags as in moonep_plan_ex.  The tables equal moonep_plan_ex's on the
  * concatenated ids. */

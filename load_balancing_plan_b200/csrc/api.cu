@@ -461,7 +461,8 @@ size_t moonep_ep_workspace_bytes(const moonep_cfg_t *cfg) {
 
 // the plan kernel in one of its expert-parallel modes
 static int ep_plan_launch(const moonep_cfg_t *cfg, int32_t mode, int32_t flags, int32_t rank, const int32_t *ids,
-                          void *ws, int32_t *counts_out, const int32_t *counts_all, void *stream) {
+                          void *ws, int32_t *counts_out, const int32_t *counts_all, void *stream,
+                          int32_t *const *counts_peers = nullptr) {
     const int N = cfg->R * cfg->L;
     DeviceInfo *d = nullptr;
     TRY(device_info(N, &d));
@@ -482,13 +483,14 @@ static int ep_plan_launch(const moonep_cfg_t *cfg, int32_t mode, int32_t flags, 
     p.rank = rank;
     p.counts_out = counts_out;
     p.counts_all = counts_all;
+    p.counts_peers = counts_peers;
     cudaError_t e = launch_plan(p, d->plan_grid, d->plan_smem, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "plan kernel launch");
     return MOONEP_OK;
 }
 
-int moonep_ep_count(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_idx, void *ws, int32_t *counts,
-                    void *stream) {
+static int ep_count_impl(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_idx, void *ws, int32_t *counts,
+                         int32_t *const *counts_all_peers, void *stream) {
     TRY(check_cfg(cfg));
     TRY(check_rank(cfg, rank));
     TRY(check_ptr(topk_idx, 4, "topk_idx", cfg->S > 0));
@@ -500,11 +502,24 @@ int moonep_ep_count(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_i
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(header)");
     e = cudaMemsetAsync(counts, 0, (size_t)(N + 1) * 4, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counts)");
-    if (cfg->S == 0) {
+    if (cfg->S == 0 && !counts_all_peers) {
         DeviceInfo *d = nullptr;
         return device_info(N, &d);
     }
-    return ep_plan_launch(cfg, kPlanCount, 0, rank, topk_idx, ws, counts, nullptr, stream);
+    // with peers the launch runs even without tokens: it stores the rank's
+    // (zero) counts into every rank's counts_all
+    return ep_plan_launch(cfg, kPlanCount, 0, rank, topk_idx, ws, counts, nullptr, stream, counts_all_peers);
+}
+
+int moonep_ep_count(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_idx, void *ws, int32_t *counts,
+                    void *stream) {
+    return ep_count_impl(cfg, rank, topk_idx, ws, counts, nullptr, stream);
+}
+
+int moonep_ep_count_exchange(const moonep_cfg_t *cfg, int32_t rank, const int32_t *topk_idx, void *ws,
+                             int32_t *counts, int32_t *const *counts_all_peers, void *stream) {
+    TRY(check_ptr(counts_all_peers, 8, "counts_all_peers", true));
+    return ep_count_impl(cfg, rank, topk_idx, ws, counts, counts_all_peers, stream);
 }
 
 int moonep_ep_plan(const moonep_cfg_t *cfg, int32_t flags, int32_t rank, const int32_t *counts_all, void *ws,

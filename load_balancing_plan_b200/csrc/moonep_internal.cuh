@@ -31,6 +31,7 @@ enum : int {
     HDR_EP = 19,           // 0: the workspace of a single-GPU plan; rank + 1: of expert-parallel rank `rank`
     HDR_TOTAL_SPILL = 20,
     HDR_PEND = 21,
+    HDR_COUNT_DONE = 22,   // counting CTAs finished (moonep_ep_count_exchange)
 };
 
 // Token ranges of the dispatch grid.  The plan counts copies per (expert,
@@ -188,6 +189,7 @@ struct PlanParams {
     int32_t rank;              // expert-parallel rank (kPlanCount, kPlanFromCounts)
     int32_t *counts_out;       // kPlanCount: [N + 1] (counts, then status bits)
     const int32_t *counts_all; // kPlanFromCounts: [R][N + 1], every rank's counts_out
+    int32_t *const *counts_peers; // kPlanCount: device table [R] of every rank's counts_all, or NULL
     uint64_t mK, mT;           // floor((2^64 - 1) / d) + 1 for d = K and d = T (set at launch)
 };
 

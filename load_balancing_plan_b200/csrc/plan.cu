@@ -678,6 +678,37 @@ __device__ void plan_tables(const PlanParams &p, int *sm) {
     }
 }
 
+// Expert parallelism, the counts' exchange fused into the counting launch:
+// the last counting CTA to finish copies the rank's finished counts [N + 1]
+// into row `rank` of every rank's counts_all, through the peer table (plain
+// stores, no multicast).  Each CTA releases its atomics and counts itself
+// done; the one that sees every other CTA done acquires and copies, so no CTA
+// waits for another.  After every rank's launch has completed (the caller's
+// barrier), each counts_all holds all R rows, as an all-gather would leave it.
+// (Not inlined: it runs only under expert parallelism, and the single-GPU
+// plan's code stays as it was.)
+__device__ __noinline__ void push_counts(const PlanParams &p) {
+    __shared__ int s_last;
+    const int N = p.N;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int done = atomicAdd(p.ws + HDR_COUNT_DONE, 1);
+        s_last = done == (int)gridDim.x - 1;
+        if (s_last) __threadfence();
+    }
+    __syncthreads();
+    if (!s_last) return;
+    const int64_t row = (int64_t)p.rank * (N + 1);
+    for (int i = threadIdx.x; i <= N; i += blockDim.x) {
+        const int v = __ldcg(p.counts_out + i);
+        for (int q = 0; q < p.cfg.R; ++q) {
+            int32_t *dst = reinterpret_cast<int32_t *>(__ldg(reinterpret_cast<const uint64_t *>(p.counts_peers) + q));
+            dst[row + i] = v;
+        }
+    }
+}
+
 // Expert parallelism: the plan from every rank's counts ([R][N + 1]: the
 // copies of each expert among the rank's tokens, then the rank's status
 // bits).  CTA 0 sums the columns into tokens_per_expert (cnt) and plans
@@ -867,6 +898,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_kernel(const __grid_cons
     if (p.mode == kPlanCount) {
         // the status travels with the counts, so every rank learns of it
         if (bad) atomicOr(p.counts_out + N, MOONEP_ST_EXPERT_ID);
+        if (p.counts_peers) push_counts(p);
         return;
     }
     // the allocation table is only written after the barrier: clear it now,

@@ -7,6 +7,9 @@ mapped from each home rank):
 
     moonep_ep_count      histogram of the rank's own ids -> counts [N + 1]
     gather_counts        all-gather -> counts_all [R][N + 1] on every rank
+      (or both in one launch: moonep_ep_count_exchange stores the rank's
+      counts into row r of every rank's counts_all through a peer table;
+      then a barrier)
     moonep_ep_plan       every rank derives the same tables from counts_all
     moonep_ep_prefetch   slot weights read from the home ranks
     moonep_ep_dispatch   rows written into the destination ranks' buffers
@@ -107,8 +110,14 @@ class RankBuffers:
             self.w[:n].copy_(torch.from_numpy(np.ascontiguousarray(topk_w, np.float32).reshape(-1)))
 
     # one rank's calls (peer tables built by the caller)
-    def count(self, stream=None):
-        mp.moonep_ep_count(self.cfg, self.rank, self.ids, self.ws, self.counts, stream)
+    def count(self, stream=None, counts_all_peers=None):
+        """The rank's counts; with counts_all_peers (every rank's counts_all)
+        also stored into row `rank` of each of them."""
+        if counts_all_peers is None:
+            mp.moonep_ep_count(self.cfg, self.rank, self.ids, self.ws, self.counts, stream)
+        else:
+            mp.moonep_ep_count_exchange(self.cfg, self.rank, self.ids, self.ws, self.counts,
+                                        _table(counts_all_peers), stream)
 
     def plan(self, flags=0, stream=None):
         mp.moonep_ep_plan(self.cfg, flags, self.rank, self.counts_all, self.ws, stream)
@@ -212,6 +221,7 @@ class Emulation:
         self.R = cfg["R"]
         self.ranks = [RankBuffers(cfg, r, device, w_elems, g_elems, poison) for r in range(self.R)]
         self.recv_peers = peer_table([rb.recv for rb in self.ranks], device)
+        self.counts_all_peers = peer_table([rb.counts_all for rb in self.ranks], device)
         if w_elems:
             self.w_home_peers = peer_table([rb.w_home for rb in self.ranks], device)
         if g_elems:
@@ -223,12 +233,20 @@ class Emulation:
         for r, rb in enumerate(self.ranks):
             rb.set_routing(np.asarray(topk_idx)[r], np.asarray(topk_w)[r])
 
-    def plan(self, flags=0, stream=None):
+    def plan(self, flags=0, stream=None, exchange=False):
+        """Every rank's count, the exchange of the counts (a copy, or with
+        exchange=True the ranks' own stores into every counts_all), then every
+        rank's plan."""
+        if exchange:
+            for rb in self.ranks:
+                rb.count(stream, self.counts_all_peers)
+        else:
+            for rb in self.ranks:
+                rb.count(stream)
+            allc = self.torch.stack([rb.counts for rb in self.ranks])
+            for rb in self.ranks:
+                rb.counts_all.copy_(allc)
         for rb in self.ranks:
-            rb.count(stream)
-        allc = self.torch.stack([rb.counts for rb in self.ranks])
-        for rb in self.ranks:
-            rb.counts_all.copy_(allc)
             rb.plan(flags, stream)
 
     def dispatch(self, stream=None):

@@ -84,6 +84,7 @@ _sig = {
     "moonep_ep_ws_layout": ([_CP, ctypes.POINTER(WsLayout)], ctypes.c_int),
     "moonep_ep_workspace_bytes": ([_CP], ctypes.c_size_t),
     "moonep_ep_count": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moonep_ep_count_exchange": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_ep_plan": ([_CP, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp], ctypes.c_int),
     "moonep_ep_dispatch": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moonep_ep_combine": ([_CP, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
@@ -254,6 +255,11 @@ def moonep_ep_workspace_bytes(cfg) -> int:
 def moonep_ep_count(cfg, rank, topk_idx, ws, counts, stream=None) -> None:
     _check(_lib.moonep_ep_count(ctypes.byref(cfg_of(cfg)), int(rank), _p(topk_idx), _p(ws), _p(counts),
                                 _stream(stream)))
+
+
+def moonep_ep_count_exchange(cfg, rank, topk_idx, ws, counts, counts_all_peers, stream=None) -> None:
+    _check(_lib.moonep_ep_count_exchange(ctypes.byref(cfg_of(cfg)), int(rank), _p(topk_idx), _p(ws), _p(counts),
+                                         _p(counts_all_peers), _stream(stream)))
 
 
 def moonep_ep_plan(cfg, flags, rank, counts_all, ws, stream=None) -> None:

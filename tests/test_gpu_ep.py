@@ -52,7 +52,7 @@ def scale_rows(torch, harness, rb, row_expert, scale):
         rb.recv[rows] = (xr * s[re[rows]][:, None]).to(torch.bfloat16).view(torch.int16)
 
 
-def run_ep_compare(env, cfg, ids, w, seed=0, E=256, mode=0):
+def run_ep_compare(env, cfg, ids, w, seed=0, E=256, mode=0, exchange=False):
     torch, mp, ep, harness = env
     R, L, S, K, H, B, Cm = (cfg[n] for n in ("R", "L", "S", "K", "H", "B", "C_max"))
     N, T = R * L, R * S
@@ -69,7 +69,11 @@ def run_ep_compare(env, cfg, ids, w, seed=0, E=256, mode=0):
         if B:
             rb.g_rep.copy_(torch.from_numpy(np.ascontiguousarray(gr[r])))
     flags = {0: 0, oracle.MODE_REMOTE: mp.PLAN_REMOTE_WEIGHTS, oracle.MODE_ONE_GROUP: mp.PLAN_ONE_GROUP}[mode]
-    em.plan(flags)
+    if exchange:
+        # the ranks' counts_all start as garbage: only the ranks' own stores fill them
+        for rb in em.ranks:
+            rb.counts_all.fill_(-5)
+    em.plan(flags, exchange=exchange)
     em.prefetch()
     em.dispatch()
     torch.cuda.synchronize()
@@ -170,11 +174,21 @@ def ep_backward_compare(env, em, cfg, opl, y_o, w, seed):
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
-def test_ep_tiny_workload(env, seed):
+@pytest.mark.parametrize("exchange", [False, True])
+def test_ep_tiny_workload(env, seed, exchange):
+    # exchange: each rank's counting launch stores its counts into every
+    # rank's counts_all (moonep_ep_count_exchange) instead of an all-gather
     wl = inputs.WORKLOADS["tiny"]
     r = inputs.routing(wl.R, wl.L, wl.S, wl.K, seed, alpha=1.0)
-    em, opl = run_ep_compare(env, wl.cfg(), r.topk_idx, r.topk_w, seed=seed)
+    em, opl = run_ep_compare(env, wl.cfg(), r.topk_idx, r.topk_w, seed=seed, exchange=exchange)
     assert opl["n_replicas"] > 0
+    if exchange:
+        N = wl.R * wl.L
+        for q, rb in enumerate(em.ranks):
+            ca = rb.counts_all.cpu().numpy()
+            for rr in range(wl.R):
+                assert np.array_equal(ca[rr, :N], np.bincount(r.topk_idx[rr].reshape(-1), minlength=N)), (q, rr)
+            assert not ca[:, N].any()
 
 
 @pytest.mark.parametrize("case", [
@@ -189,6 +203,7 @@ def test_ep_tiny_workload(env, seed):
 ])
 def test_ep_small_cases(env, case):
     R, L, S, K, H, B, headroom, mode = case
+    exchange = R in (4, 64)  # the fallback case and the one with R at its maximum: counts exchanged in the launch
     cfg = cfg_of(R, L, S, K, H, B, headroom)
     if (R, L) == (4, 2):
         ids = pc.ids_from_counts(np.array([2, 3, 2, 3, 2, 3, 1, 0]), R, S, K)
@@ -196,7 +211,7 @@ def test_ep_small_cases(env, case):
     else:
         rt = inputs.routing(R, L, S, K, 3, alpha=1.5)
         ids, w = rt.topk_idx, rt.topk_w
-    em, opl = run_ep_compare(env, cfg, ids, w, seed=1, mode=mode)
+    em, opl = run_ep_compare(env, cfg, ids, w, seed=1, mode=mode, exchange=exchange)
     if (R, L) == (4, 2):
         assert opl["fallback_rows"] > 0
     if mode == oracle.MODE_ONE_GROUP:
@@ -204,8 +219,9 @@ def test_ep_small_cases(env, case):
 
 
 def test_ep_mid_workload_plan_and_rows(env):
-    # the mid workload split over 8 ranks: every rank's tables and
-    # destinations in full, and sampled dispatched rows and combined tokens
+    # the mid workload split over 8 ranks, the counts exchanged in the
+    # counting launches: every rank's tables and destinations in full, and
+    # sampled dispatched rows and combined tokens
     torch, mp, ep, harness = env
     wl = inputs.WORKLOADS["mid"]
     cfg = wl.cfg()
@@ -215,7 +231,7 @@ def test_ep_mid_workload_plan_and_rows(env):
     em.set_routing(r.topk_idx, r.topk_w)
     for q, rb in enumerate(em.ranks):
         inputs.cb_fill_torch(rb.x.view(torch.bfloat16), 0, inputs.STREAM_X, offset=q * S * H)
-    em.plan()
+    em.plan(exchange=True)
     em.dispatch()
     em.combine()
     torch.cuda.synchronize()
@@ -244,7 +260,8 @@ def test_ep_mid_workload_plan_and_rows(env):
         assert np.array_equal(harness.to_u16(rb.out[torch.from_numpy(ts).cuda()]), out_o), q
 
 
-def test_ep_bad_id_on_one_rank_stops_every_rank(env):
+@pytest.mark.parametrize("exchange", [False, True])
+def test_ep_bad_id_on_one_rank_stops_every_rank(env, exchange):
     torch, mp, ep, harness = env
     wl = inputs.WORKLOADS["tiny"]
     cfg = wl.cfg()
@@ -253,7 +270,7 @@ def test_ep_bad_id_on_one_rank_stops_every_rank(env):
     ids[2, 5, 1] = wl.N + 3            # one bad id, on rank 2
     em = ep.Emulation(cfg, poison=True)
     em.set_routing(ids, r.topk_w)
-    em.plan()
+    em.plan(exchange=exchange)
     em.dispatch()
     torch.cuda.synchronize()
     for rb in em.ranks:
@@ -310,12 +327,17 @@ def test_ep_edge_cases(env, case):
         assert opl["n_replicas"] == 0 and opl["fallback_rows"] > 0
 
 
-def test_ep_empty_ranks(env):
+@pytest.mark.parametrize("exchange", [False, True])
+def test_ep_empty_ranks(env, exchange):
     # S = 0: nothing to count, plan or move; every call returns without error
+    # (with the exchange, each rank still stores its zero row everywhere)
     torch, mp, ep, harness = env
     cfg = cfg_of(4, 2, 0, 2, 16, 2)
     em = ep.Emulation(cfg, w_elems=64, g_elems=64)
-    em.plan()
+    if exchange:
+        for rb in em.ranks:
+            rb.counts_all.fill_(-5)
+    em.plan(exchange=exchange)
     em.prefetch()
     em.dispatch()
     em.combine()
@@ -325,6 +347,7 @@ def test_ep_empty_ranks(env):
         info = rb.read_plan(tables=False)
         assert info["status"] & mp.ST_ERROR_MASK == 0
         assert info["n_replicas"] == 0 and info["fallback_rows"] == 0
+        assert not rb.counts_all.cpu().numpy().any()
 
 
 @pytest.mark.parametrize("kernel", ["dispatch", "combine", "combine_backward", "prefetch"])

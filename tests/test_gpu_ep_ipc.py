@@ -1,11 +1,13 @@
 """The expert-parallel step as separate processes, one per rank: each process
 owns its buffers, maps the other ranks' buffers through CUDA IPC
-(ep.exchange_buffers), all-gathers the counts over a process group and orders
-the ranks between calls with barriers, as one process per GPU does.  Here
-both processes share one GPU (the kernels of different ranks never wait for
-one another, so running them in two contexts on one device computes what two
-devices would; only NVLink is missing).  The process group is gloo, so the
-counts travel through host memory.  Each rank checks its own destinations,
+(ep.map_peers), gets every rank's counts (an all-gather over the process
+group, or each rank's counting launch storing its counts into every rank's
+mapped counts_all) and orders the ranks between calls with barriers, as one
+process per GPU does.  Here both processes share one GPU (the kernels of
+different ranks never wait for one another, so running them in two contexts
+on one device computes what two devices would; only NVLink is missing).  The
+process group is gloo, so the all-gathered counts travel through host
+memory.  Each rank checks its own destinations,
 receive rows, combined outputs, prefetched slots, backward gradients and
 reduced gradients against the oracle, bit for bit (grad_w within its fp32
 bound)."""
@@ -37,7 +39,7 @@ def _rank(rank, world, port, q, case):
     try:
         torch.cuda.set_device(0)
         dev = torch.device("cuda", 0)
-        L, S, K, H, B, hr, seed = case
+        L, S, K, H, B, hr, seed, exchange = case
         R = world
         C = S * K
         cfg = dict(R=R, L=L, S=S, K=K, H=H, B=B, C=C, C_max=int(np.floor((1 + hr) * C)))
@@ -61,21 +63,31 @@ def _rank(rank, world, port, q, case):
         G = inputs.cb_bf16_np(seed + 7, inputs.STREAM_Y, np.arange(T * H)).reshape(T, H)
         g_out = harness.as_i16(G[rank * S:(rank + 1) * S]).to(dev)
         torch.cuda.synchronize()
+
+        def between():
+            torch.cuda.synchronize()
+            dist.barrier()
+
         # peers: every rank's buffers mapped into this process (the PeerTable
         # objects keep the mappings alive)
         recv_peers = ep.map_peers(rb.recv, dev)
         w_home_peers = ep.map_peers(rb.w_home, dev)
         g_rep_peers = ep.map_peers(rb.g_rep, dev)
         grad_y_peers = ep.map_peers(grad_y, dev)
+        counts_all_peers = ep.map_peers(rb.counts_all, dev)
 
-        def between():
-            torch.cuda.synchronize()
-            dist.barrier()
-
-        rb.count()
-        counts_all = torch.zeros((R, N + 1), dtype=torch.int32)
-        ep.gather_counts(rb.counts.cpu(), counts_all)
-        rb.counts_all.copy_(counts_all)
+        if exchange:
+            # each rank's counting launch stores its counts into every rank's
+            # counts_all; the barrier then stands in for the all-gather
+            rb.counts_all.fill_(-5)
+            between()
+            rb.count(counts_all_peers=counts_all_peers)
+            between()
+        else:
+            rb.count()
+            counts_all = torch.zeros((R, N + 1), dtype=torch.int32)
+            ep.gather_counts(rb.counts.cpu(), counts_all)
+            rb.counts_all.copy_(counts_all)
         rb.plan()
         rb.prefetch(w_home_peers)
         rb.dispatch(recv_peers)
@@ -136,9 +148,9 @@ def _rank(rank, world, port, q, case):
 
 
 @pytest.mark.parametrize("case", [
-    # L, S, K, H, B, headroom, seed
-    (4, 64, 2, 64, 2, 0.5, 3),
-    (8, 300, 4, 136, 3, 1.0, 1),
+    # L, S, K, H, B, headroom, seed, counts exchanged in the counting launch
+    (4, 64, 2, 64, 2, 0.5, 3, False),
+    (8, 300, 4, 136, 3, 1.0, 1, True),
 ])
 def test_two_processes_on_cuda_ipc(case):
     import oracle
