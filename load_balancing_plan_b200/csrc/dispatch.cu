@@ -5,9 +5,10 @@
 // writes there, so no receive-buffer-to-compute-buffer copy exists;
 // agentlenshq "MoonshotAI/MoonEP", "How it works": fused permute).
 //
-// One CTA per token range (the ranges the plan counted: about 4 tokens each,
-// run in waves of two resident CTAs per SM, so that at any moment the stores
-// of all CTAs go to neighbouring rows of each expert's segment).  Warp 0
+// One CTA per token range (the ranges the plan counted: about 4 tokens each;
+// the grid is a whole number of waves of two CTAs per SM, and at H = 7168 a
+// CTA's 66 KB of shared memory lets three be resident; at any moment the
+// stores of all CTAs go to neighbouring rows of each expert's segment).  Warp 0
 // numbers the range's copies in ascending g: for each group of 32 ids it
 // finds equal experts with __match_any_sync, ranks lanes within a group by
 // popcount, and adds a per-expert running counter kept in shared memory
